@@ -1,0 +1,247 @@
+/*
+ * mxmoe.h -- C ABI of the MXFP8 routed-experts MLP library (libmxmoe.so).
+ *
+ * What the library computes (the routed-experts MLP of the torchtitan page
+ * "Wire the fully-fused grouped-GEMM MXFP8 plan behind fusion_plan", section
+ * "What it adds", and the page "fused gated-activation (SwiGLU) + MXFP8
+ * quantization kernel override", section "Summary"):
+ *
+ *   forward   h13 = x_e . W13[e]^T        (FC1 grouped GEMM, per expert e)
+ *             h   = silu(gate) * up       (fused SwiGLU + dual MXFP8 quant)
+ *             y   = h_e . W2[e]^T         (FC2 grouped GEMM)
+ *   backward  dh  = dy_e . W2[e]; dh13 = dSwiGLU(dh, h13)  (fused)
+ *             dW2[e] = dy_e^T . h_e, dx = dh13_e . W13[e], dW13[e] = dh13_e^T . x_e
+ *
+ * MXFP8 format (A2E MXFP8 pages, "quant_mode=4 ... E4M3 ... E8M0 MX scale"):
+ * each block of 32 consecutive elements is stored as 32 E4M3 codes (uint8)
+ * plus one E8M0 scale byte.  Scale rule (OCP MX v1.0): shared exponent
+ * floor(log2(amax)) - 8, byte = clamp(exp + 127, 0, 254); all-zero blocks get
+ * byte 0; a block holding NaN/Inf gets byte 0xFF and codes 0x7F|sign.
+ * Elements: x / 2^exp rounded to nearest-even E4M3, saturated to +-448.
+ *
+ * Conventions for every call:
+ *  - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *    never allocates device memory (composites take a caller workspace).
+ *  - bf16 tensors are passed as void* (IEEE bfloat16, row-major, dense).
+ *  - Every call is asynchronous on `stream` and returns an mxmoe_status; on
+ *    an error nothing is launched and mxmoe_last_error() names the argument.
+ *  - ROW quantization: blocks along the last (contiguous) dimension;
+ *    COL quantization: blocks over 32 consecutive rows of one column, stored
+ *    TRANSPOSED (codes [cols, rows]) so the contraction dimension is contiguous.
+ *  - Scale layouts:
+ *      MXFP8_SCALE_PLAIN: uint8 [R, ceil(C/32)] row-major for a matrix [R, C].
+ *      MXFP8_SCALE_MMA  : the tensor-core layout of a matrix [R, C] with
+ *        R % 128 == 0 and C % 128 == 0: 512-byte atoms, atom (R/128, C/128)
+ *        at byte ((r/128)*(C/128) + c/128)*512; inside it, the scale of row r
+ *        and 32-column block kb = c/32 sits at (r%32)*16 + ((r%128)/32)*4 + kb%4.
+ *      Grouped GEMM operands always use MXFP8_SCALE_MMA.
+ *  - expert_offsets: DEVICE int32 [E+1], offsets[0] == 0, non-decreasing,
+ *    every offset a multiple of pad_multiple (itself a multiple of 128), and
+ *    offsets[E] <= M.  Rows at or past offsets[E] are never read or written.
+ *    The GEMM kernels re-check this on the device; a bad table makes them do
+ *    nothing and raises MXMOE_ERR_OFFSETS in mxmoe_device_error().
+ */
+#ifndef MXMOE_H
+#define MXMOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MXMOE_OK = 0,
+  MXMOE_ERR_NULL = 1,           /* a required pointer is NULL                       */
+  MXMOE_ERR_SHAPE = 2,          /* a dimension is zero/negative or not a multiple   */
+  MXMOE_ERR_ALIGN = 3,          /* a pointer is not 16-byte aligned                  */
+  MXMOE_ERR_OFFSETS = 4,        /* expert_offsets table invalid (device-detected)    */
+  MXMOE_ERR_ARCH = 5,           /* current device is not sm_100                      */
+  MXMOE_ERR_CUDA = 6,           /* a CUDA runtime/driver call failed                 */
+  MXMOE_ERR_DEVICE_TIMEOUT = 7, /* a bounded device-side wait expired                */
+  MXMOE_ERR_WORKSPACE = 8,      /* workspace missing or too small                    */
+  MXMOE_ERR_ARG = 9             /* an enum/flag argument is out of range             */
+} mxmoe_status;
+
+#define MXFP8_ROW 1
+#define MXFP8_COL 2
+#define MXFP8_SCALE_PLAIN 0
+#define MXFP8_SCALE_MMA 1
+
+/* Text of the last host-side error of the calling thread ("" if none). */
+const char* mxmoe_last_error(void);
+
+/* Device-side error word of the current device (a GEMM kernel that found a
+ * bad offsets table or whose bounded mbarrier wait expired sets it).
+ * Synchronizes `stream`, returns the first error code recorded (MXMOE_OK if
+ * none) in *code and, if reset != 0, clears it.  Returns MXMOE_ERR_CUDA if
+ * the read itself failed. */
+int mxmoe_device_error(cudaStream_t stream, int reset, int* code);
+
+/* Library version string and number of SMs the kernels size grids for. */
+const char* mxmoe_version(void);
+
+/* -------------------------------------------------------------------------
+ * mxfp8_quantize -- bf16 -> MXFP8 cast, row-wise and/or column-wise.
+ * (Standalone cast kernels of the SwiGLU-boundary page, "Summary": the
+ * unfused path launches 6 + 6 of them per MLP; A2E MXFP8 page: the
+ * attention side quantizes the activation so "the payload halves".)
+ *
+ *  x        bf16 [batch, rows, cols]
+ *  modes    MXFP8_ROW | MXFP8_COL (at least one)
+ *  ROW out  row_codes  uint8 [batch, rows, cols];
+ *           row_scales PLAIN [batch*rows, ceil(cols/32)] (short last block
+ *           allowed when cols % 32 != 0) or MMA layout of [batch*rows, cols].
+ *  COL out  col_codes  uint8 [batch, cols, rows] (each batch transposed);
+ *           col_scales PLAIN [batch*cols, rows/32] or MMA layout of the
+ *           [batch*cols, rows] matrix.  Needs rows % 32 == 0.
+ *  MMA layout needs rows % 128 == 0 and cols % 128 == 0.
+ * Unused output pointers may be NULL.
+ * ------------------------------------------------------------------------- */
+int mxfp8_quantize(const void* x, int64_t batch, int64_t rows, int64_t cols,
+                   int modes, int scale_layout,
+                   uint8_t* row_codes, uint8_t* row_scales,
+                   uint8_t* col_codes, uint8_t* col_scales,
+                   cudaStream_t stream);
+
+/* -------------------------------------------------------------------------
+ * mxfp8_swiglu_quant -- fused SwiGLU + dual MXFP8 quantization.
+ * (SwiGLU-boundary page, "Summary": fused SwiGLU + dual MXFP8 quantization;
+ * the bf16 post-activation is never materialized.)
+ *
+ *  h13   bf16 [rows, 2F]; columns 0..F-1 gate (a), F..2F-1 up (b)
+ *  h     = bf16(silu(a) * b) computed in fp32, never written to memory
+ *  outputs as mxfp8_quantize of h [rows, F] with batch = 1.
+ *  Needs F % 32 == 0; COL needs rows % 32 == 0; MMA layout needs rows and F
+ *  multiples of 128.
+ * ------------------------------------------------------------------------- */
+int mxfp8_swiglu_quant(const void* h13, int64_t rows, int64_t F,
+                       int modes, int scale_layout,
+                       uint8_t* row_codes, uint8_t* row_scales,
+                       uint8_t* col_codes, uint8_t* col_scales,
+                       cudaStream_t stream);
+
+/* -------------------------------------------------------------------------
+ * mxfp8_dequantize -- MXFP8 (ROW, PLAIN scales) -> bf16.
+ * (A2E transport page, review "[P2] Handle the two E8M0 endpoint encodings":
+ * byte 0x00 is 2^-127, byte 0xFF is NaN.)  out = bf16(code * 2^(byte-127)).
+ *  codes [rows, cols], scales [rows, ceil(cols/32)], out bf16 [rows, cols].
+ * ------------------------------------------------------------------------- */
+int mxfp8_dequantize(const uint8_t* codes, const uint8_t* scales,
+                     int64_t rows, int64_t cols, void* out, cudaStream_t stream);
+
+/* -------------------------------------------------------------------------
+ * mxfp8_grouped_gemm -- ragged-M grouped GEMM (FC2 / dgrad form).
+ * (Fully-fused plan page, "What it adds": FC2 GEMM.)
+ *
+ *  out[m, n] = sum_k A[m, k] * W[e, n, k] for offsets[e] <= m < offsets[e+1],
+ *  with both operands dequantized from MXFP8 and accumulated in fp32 on the
+ *  tensor cores; out is bf16 [M, N] (rows >= offsets[E] untouched).
+ *  a, a_scales : codes [M, K], MMA scales of [M, K]
+ *  w, w_scales : codes [E, N, K], MMA scales of [E*N, K]
+ *  Needs M, N, K multiples of 128.
+ * ------------------------------------------------------------------------- */
+int mxfp8_grouped_gemm(const uint8_t* a, const uint8_t* a_scales, int64_t M, int64_t K,
+                       const uint8_t* w, const uint8_t* w_scales, int E, int64_t N,
+                       const int32_t* expert_offsets, int pad_multiple,
+                       void* out, cudaStream_t stream);
+
+/* -------------------------------------------------------------------------
+ * mxfp8_grouped_gemm_wgrad -- ragged-K grouped GEMM (weight gradients).
+ * (Fully-fused plan page, "What it adds": wgrad; "Evidence": zero-token
+ * experts give exact-zero grads.)
+ *
+ *  dw[e, n, j] = sum over m in expert e's rows of G[m, n] * X[m, j]
+ *  gt, gt_scales : COL codes of G, [N, M], MMA scales of [N, M]
+ *  xt, xt_scales : COL codes of X, [Kx, M], MMA scales of [Kx, M]
+ *  dw            : bf16 [E, N, Kx]; an expert with no rows gets exact zeros.
+ *  Needs N, Kx, M multiples of 128.
+ * ------------------------------------------------------------------------- */
+int mxfp8_grouped_gemm_wgrad(const uint8_t* gt, const uint8_t* gt_scales, int64_t N,
+                             const uint8_t* xt, const uint8_t* xt_scales, int64_t Kx,
+                             int64_t M, const int32_t* expert_offsets, int E, int pad_multiple,
+                             void* dw, cudaStream_t stream);
+
+/* -------------------------------------------------------------------------
+ * mxfp8_grouped_gemm_swiglu_quant -- FC1 grouped GEMM with the SwiGLU + dual
+ * quantization epilogue in one launch (fully-fused plan page, "What it adds":
+ * "FC1 grouped GEMM + SwiGLU + dual MXFP8 quantization in one launch").
+ *
+ *  h13 = x_e . W13[e]^T (fp32 accumulate, rounded to bf16), h = bf16(silu(a)*b)
+ *  a, a_scales     : x codes [M, K], MMA scales
+ *  w13, w13_scales : codes [E, 2F, K] (rows 0..F-1 gate, F..2F-1 up), MMA scales of [E*2F, K]
+ *  h13_out         : bf16 [M, 2F] (saved for the backward), may be NULL
+ *  h_row_codes/scales : [M, F], MMA scales of [M, F]    (FC2 operand)
+ *  h_col_codes/scales : [F, M], MMA scales of [F, M]    (dW2 operand)
+ *  Needs M, K, F multiples of 128.
+ * ------------------------------------------------------------------------- */
+int mxfp8_grouped_gemm_swiglu_quant(const uint8_t* a, const uint8_t* a_scales,
+                                    int64_t M, int64_t K,
+                                    const uint8_t* w13, const uint8_t* w13_scales,
+                                    int E, int64_t F,
+                                    const int32_t* expert_offsets, int pad_multiple,
+                                    void* h13_out,
+                                    uint8_t* h_row_codes, uint8_t* h_row_scales,
+                                    uint8_t* h_col_codes, uint8_t* h_col_scales,
+                                    cudaStream_t stream);
+
+/* -------------------------------------------------------------------------
+ * mxfp8_grouped_gemm_dswiglu_quant -- FC2 dgrad with the fused dSwiGLU +
+ * dual quantization epilogue (fully-fused plan page: "fused dSwiGLU backward").
+ *
+ *  dh = bf16(dy_e . W2[e]) (contraction over D), then with a, b from h13:
+ *  s = sigmoid(a); dgate = dh*b*s*(1 + a*(1-s)); dup = dh*a*s (fp32, -> bf16)
+ *  dy, dy_scales   : codes [M, D], MMA scales
+ *  w2t, w2t_scales : COL codes of W2 per expert, [E, F, D], MMA scales of [E*F, D]
+ *  h13             : bf16 [M, 2F] saved by the forward
+ *  g_row_codes/scales : dh13 codes [M, 2F], MMA scales of [M, 2F]   (dx operand)
+ *  g_col_codes/scales : dh13 codes [2F, M], MMA scales of [2F, M]   (dW13 operand)
+ *  Needs M, D, F multiples of 128.
+ * ------------------------------------------------------------------------- */
+int mxfp8_grouped_gemm_dswiglu_quant(const uint8_t* dy, const uint8_t* dy_scales,
+                                     int64_t M, int64_t D,
+                                     const uint8_t* w2t, const uint8_t* w2t_scales,
+                                     int E, int64_t F,
+                                     const int32_t* expert_offsets, int pad_multiple,
+                                     const void* h13,
+                                     uint8_t* g_row_codes, uint8_t* g_row_scales,
+                                     uint8_t* g_col_codes, uint8_t* g_col_scales,
+                                     cudaStream_t stream);
+
+/* -------------------------------------------------------------------------
+ * Composites.  All buffers caller-owned.  x, dy: bf16 [M, D] (pad rows zero);
+ * w13: bf16 [E, 2F, D]; w2: bf16 [E, D, F].  The saved tensors are what the
+ * backward needs: h13 (bf16 [M, 2F]), the COL-quantized h ([F, M] codes + MMA
+ * scales) and the COL-quantized x ([D, M] codes + MMA scales).  The bf16
+ * post-activation h is never written.
+ * Workspace: mxmoe_workspace_size(which = 1 fwd, 2 bwd) bytes, 256-aligned.
+ * ------------------------------------------------------------------------- */
+typedef struct {
+  void* h13;               /* bf16 [M, 2F]                     */
+  uint8_t* h_col_codes;    /* [F, M]                            */
+  uint8_t* h_col_scales;   /* MMA scales of [F, M]              */
+  uint8_t* x_col_codes;    /* [D, M]                            */
+  uint8_t* x_col_scales;   /* MMA scales of [D, M]              */
+} mxmoe_saved;
+
+size_t mxmoe_workspace_size(int64_t M, int64_t D, int E, int64_t F, int which);
+
+int moe_mlp_fwd(const void* x, int64_t M, int64_t D,
+                const void* w13, const void* w2, int E, int64_t F,
+                const int32_t* expert_offsets, int pad_multiple,
+                void* y, const mxmoe_saved* saved,
+                void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+int moe_mlp_bwd(const void* dy, int64_t M, int64_t D,
+                const void* w13, const void* w2, int E, int64_t F,
+                const int32_t* expert_offsets, int pad_multiple,
+                const mxmoe_saved* saved,
+                void* dx, void* dw13, void* dw2,
+                void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MXMOE_H */

@@ -1,0 +1,296 @@
+"""Python binding of libmxmoe (MXFP8 routed-experts MLP for sm_100a).
+
+Argument marshalling only: tensors are checked, output buffers allocated with
+torch on the tensor's device, and the C ABI of include/mxmoe.h is called on
+the current torch CUDA stream.  Every step of the computation runs in the
+library's CUDA kernels; there is no CPU or PyTorch fallback, and a missing or
+unbuilt library raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+__all__ = [
+    "ROW", "COL", "PLAIN", "MMA", "lib", "MXMOEError",
+    "mxfp8_quantize", "mxfp8_swiglu_quant", "mxfp8_dequantize",
+    "mxfp8_grouped_gemm", "mxfp8_grouped_gemm_wgrad",
+    "mxfp8_grouped_gemm_swiglu_quant", "mxfp8_grouped_gemm_dswiglu_quant",
+    "moe_mlp_fwd", "moe_mlp_bwd", "device_error", "header_functions",
+]
+
+ROW, COL = 1, 2
+PLAIN, MMA = 0, 1
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmxmoe.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "mxmoe.h")
+
+
+class MXMOEError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"mxmoe status {status}: {msg}")
+        self.status = status
+
+
+class _Saved(ctypes.Structure):
+    _fields_ = [("h13", ctypes.c_void_p), ("h_col_codes", ctypes.c_void_p), ("h_col_scales", ctypes.c_void_p),
+                ("x_col_codes", ctypes.c_void_p), ("x_col_scales", ctypes.c_void_p)]
+
+
+_P, _I, _L, _S = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+_SIGS = {
+    "mxmoe_last_error": ([], ctypes.c_char_p),
+    "mxmoe_version": ([], ctypes.c_char_p),
+    "mxmoe_device_error": ([_P, _I, ctypes.POINTER(ctypes.c_int)], _I),
+    "mxfp8_quantize": ([_P, _L, _L, _L, _I, _I, _P, _P, _P, _P, _P], _I),
+    "mxfp8_swiglu_quant": ([_P, _L, _L, _I, _I, _P, _P, _P, _P, _P], _I),
+    "mxfp8_dequantize": ([_P, _P, _L, _L, _P, _P], _I),
+    "mxfp8_grouped_gemm": ([_P, _P, _L, _L, _P, _P, _I, _L, _P, _I, _P, _P], _I),
+    "mxfp8_grouped_gemm_wgrad": ([_P, _P, _L, _P, _P, _L, _L, _P, _I, _I, _P, _P], _I),
+    "mxfp8_grouped_gemm_swiglu_quant": ([_P, _P, _L, _L, _P, _P, _I, _L, _P, _I, _P, _P, _P, _P, _P, _P], _I),
+    "mxfp8_grouped_gemm_dswiglu_quant": ([_P, _P, _L, _L, _P, _P, _I, _L, _P, _I, _P, _P, _P, _P, _P, _P], _I),
+    "mxmoe_workspace_size": ([_L, _L, _I, _L, _I], _S),
+    "moe_mlp_fwd": ([_P, _L, _L, _P, _P, _I, _L, _P, _I, _P, ctypes.POINTER(_Saved), _P, _S, _P], _I),
+    "moe_mlp_bwd": ([_P, _L, _L, _P, _P, _I, _L, _P, _I, ctypes.POINTER(_Saved), _P, _P, _P, _P, _S, _P], _I),
+}
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libmxmoe.so from the package directory (raises if it is not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is not built; run `python -m mxfp8_block_scaled_routed_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (args, ret) in _SIGS.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = ret
+        _lib = L
+    return _lib
+
+
+def header_functions() -> list[str]:
+    """Names of the functions declared in include/mxmoe.h."""
+    src = open(HEADER_PATH).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\**\s+\**(\w+)\s*\(", src, flags=re.M)))
+
+
+def _check(status: int):
+    if status != 0:
+        raise MXMOEError(status, lib().mxmoe_last_error().decode())
+
+
+def _stream(t: torch.Tensor):
+    return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _need(t: torch.Tensor, dtype, name: str):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (no CPU path)")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _u8(shape, dev):
+    return torch.empty(shape, dtype=torch.uint8, device=dev)
+
+
+def device_error(reset: bool = True, device=None) -> int:
+    """First device-side error code recorded by the kernels (0 if none)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    code = ctypes.c_int(0)
+    _check(lib().mxmoe_device_error(ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream),
+                                    int(reset), ctypes.byref(code)))
+    return code.value
+
+
+# ----------------------------------------------------------------------------- casts
+def mxfp8_quantize(x: torch.Tensor, modes: int = ROW | COL, scale_layout: int = PLAIN):
+    """bf16 [rows, cols] or [batch, rows, cols] -> dict of MXFP8 tensors.
+
+    Keys: row_codes [.., rows, cols], row_scales, col_codes [.., cols, rows],
+    col_scales.  PLAIN scales are [.., rows, ceil(cols/32)] / [.., cols, rows/32];
+    MMA scales are flat uint8 vectors in the tensor-core atom layout.
+    """
+    _need(x, torch.bfloat16, "x")
+    if x.dim() not in (2, 3):
+        raise ValueError("x must be 2-D or 3-D")
+    batch = x.shape[0] if x.dim() == 3 else 1
+    rows, cols = x.shape[-2], x.shape[-1]
+    lead = (batch,) if x.dim() == 3 else ()
+    out = {}
+    if modes & ROW:
+        out["row_codes"] = _u8(lead + (rows, cols), x.device)
+        out["row_scales"] = (_u8(lead + (rows, (cols + 31) // 32), x.device) if scale_layout == PLAIN
+                             else _u8((batch * rows * cols // 32,), x.device))
+    if modes & COL:
+        out["col_codes"] = _u8(lead + (cols, rows), x.device)
+        out["col_scales"] = (_u8(lead + (cols, rows // 32), x.device) if scale_layout == PLAIN
+                             else _u8((batch * rows * cols // 32,), x.device))
+    _check(lib().mxfp8_quantize(_ptr(x), batch, rows, cols, modes, scale_layout,
+                                _ptr(out.get("row_codes")), _ptr(out.get("row_scales")),
+                                _ptr(out.get("col_codes")), _ptr(out.get("col_scales")), _stream(x)))
+    return out
+
+
+def mxfp8_swiglu_quant(h13: torch.Tensor, modes: int = ROW | COL, scale_layout: int = PLAIN):
+    """bf16 h13 [rows, 2F] -> MXFP8 of h = silu(gate) * up, as mxfp8_quantize."""
+    _need(h13, torch.bfloat16, "h13")
+    rows, F2 = h13.shape
+    F = F2 // 2
+    out = {}
+    if modes & ROW:
+        out["row_codes"] = _u8((rows, F), h13.device)
+        out["row_scales"] = (_u8((rows, F // 32), h13.device) if scale_layout == PLAIN
+                             else _u8((rows * F // 32,), h13.device))
+    if modes & COL:
+        out["col_codes"] = _u8((F, rows), h13.device)
+        out["col_scales"] = (_u8((F, rows // 32), h13.device) if scale_layout == PLAIN
+                             else _u8((rows * F // 32,), h13.device))
+    _check(lib().mxfp8_swiglu_quant(_ptr(h13), rows, F, modes, scale_layout,
+                                    _ptr(out.get("row_codes")), _ptr(out.get("row_scales")),
+                                    _ptr(out.get("col_codes")), _ptr(out.get("col_scales")), _stream(h13)))
+    return out
+
+
+def mxfp8_dequantize(codes: torch.Tensor, scales: torch.Tensor) -> torch.Tensor:
+    """MXFP8 ROW (plain scales) -> bf16."""
+    _need(codes, torch.uint8, "codes")
+    _need(scales, torch.uint8, "scales")
+    rows, cols = codes.shape
+    out = torch.empty(rows, cols, dtype=torch.bfloat16, device=codes.device)
+    _check(lib().mxfp8_dequantize(_ptr(codes), _ptr(scales), rows, cols, _ptr(out), _stream(codes)))
+    return out
+
+
+# ----------------------------------------------------------------------------- GEMMs
+def _offs(offsets: torch.Tensor):
+    _need(offsets, torch.int32, "expert_offsets")
+    return offsets.numel() - 1
+
+
+def mxfp8_grouped_gemm(a, a_scales, w, w_scales, offsets, pad_multiple=128, out=None):
+    """Ragged-M grouped GEMM: a [M, K] codes, w [E, N, K] codes (MMA scales)."""
+    E = _offs(offsets)
+    M, K = a.shape
+    _, N, _ = w.shape
+    if out is None:
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=a.device)
+    for t, n in ((a, "a"), (a_scales, "a_scales"), (w, "w"), (w_scales, "w_scales")):
+        _need(t, torch.uint8, n)
+    _check(lib().mxfp8_grouped_gemm(_ptr(a), _ptr(a_scales), M, K, _ptr(w), _ptr(w_scales), E, N,
+                                    _ptr(offsets), pad_multiple, _ptr(out), _stream(a)))
+    return out
+
+
+def mxfp8_grouped_gemm_wgrad(gt, gt_scales, xt, xt_scales, offsets, pad_multiple=128, out=None):
+    """Ragged-K grouped GEMM: gt [N, M], xt [Kx, M] COL codes -> dw bf16 [E, N, Kx]."""
+    E = _offs(offsets)
+    N, M = gt.shape
+    Kx = xt.shape[0]
+    if out is None:
+        out = torch.empty(E, N, Kx, dtype=torch.bfloat16, device=gt.device)
+    _check(lib().mxfp8_grouped_gemm_wgrad(_ptr(gt), _ptr(gt_scales), N, _ptr(xt), _ptr(xt_scales), Kx, M,
+                                          _ptr(offsets), E, pad_multiple, _ptr(out), _stream(gt)))
+    return out
+
+
+def mxfp8_grouped_gemm_swiglu_quant(a, a_scales, w13, w13_scales, offsets, pad_multiple=128, want_h13=True):
+    """FC1 + SwiGLU + dual quantization; returns dict(h13, h_row_codes, h_row_scales, h_col_codes, h_col_scales)."""
+    E = _offs(offsets)
+    M, K = a.shape
+    F = w13.shape[1] // 2
+    dev = a.device
+    o = dict(h13=torch.empty(M, 2 * F, dtype=torch.bfloat16, device=dev) if want_h13 else None,
+             h_row_codes=_u8((M, F), dev), h_row_scales=_u8((M * F // 32,), dev),
+             h_col_codes=_u8((F, M), dev), h_col_scales=_u8((M * F // 32,), dev))
+    _check(lib().mxfp8_grouped_gemm_swiglu_quant(
+        _ptr(a), _ptr(a_scales), M, K, _ptr(w13), _ptr(w13_scales), E, F, _ptr(offsets), pad_multiple,
+        _ptr(o["h13"]), _ptr(o["h_row_codes"]), _ptr(o["h_row_scales"]), _ptr(o["h_col_codes"]),
+        _ptr(o["h_col_scales"]), _stream(a)))
+    return o
+
+
+def mxfp8_grouped_gemm_dswiglu_quant(dy, dy_scales, w2t, w2t_scales, offsets, h13, pad_multiple=128):
+    """FC2 dgrad + dSwiGLU + dual quantization; returns dict(g_row_codes, g_row_scales, g_col_codes, g_col_scales)."""
+    E = _offs(offsets)
+    M, D = dy.shape
+    F = w2t.shape[1]
+    dev = dy.device
+    _need(h13, torch.bfloat16, "h13")
+    o = dict(g_row_codes=_u8((M, 2 * F), dev), g_row_scales=_u8((M * 2 * F // 32,), dev),
+             g_col_codes=_u8((2 * F, M), dev), g_col_scales=_u8((M * 2 * F // 32,), dev))
+    _check(lib().mxfp8_grouped_gemm_dswiglu_quant(
+        _ptr(dy), _ptr(dy_scales), M, D, _ptr(w2t), _ptr(w2t_scales), E, F, _ptr(offsets), pad_multiple,
+        _ptr(h13), _ptr(o["g_row_codes"]), _ptr(o["g_row_scales"]), _ptr(o["g_col_codes"]),
+        _ptr(o["g_col_scales"]), _stream(dy)))
+    return o
+
+
+# ----------------------------------------------------------------------------- composites
+def workspace_bytes(M, D, E, F, which):
+    return int(lib().mxmoe_workspace_size(M, D, E, F, which))
+
+
+def make_saved(M, D, F, device):
+    return dict(h13=torch.empty(M, 2 * F, dtype=torch.bfloat16, device=device),
+                h_col_codes=_u8((F, M), device), h_col_scales=_u8((M * F // 32,), device),
+                x_col_codes=_u8((D, M), device), x_col_scales=_u8((M * D // 32,), device))
+
+
+def _saved_struct(s):
+    return _Saved(s["h13"].data_ptr(), s["h_col_codes"].data_ptr(), s["h_col_scales"].data_ptr(),
+                  s["x_col_codes"].data_ptr(), s["x_col_scales"].data_ptr())
+
+
+def moe_mlp_fwd(x, w13, w2, offsets, pad_multiple=128, y=None, saved=None, workspace=None):
+    """Forward of the routed-experts MLP. Returns (y bf16 [M, D], saved dict)."""
+    E = _offs(offsets)
+    for t, n in ((x, "x"), (w13, "w13"), (w2, "w2")):
+        _need(t, torch.bfloat16, n)
+    M, D = x.shape
+    F = w13.shape[1] // 2
+    dev = x.device
+    y = torch.empty(M, D, dtype=torch.bfloat16, device=dev) if y is None else y
+    saved = make_saved(M, D, F, dev) if saved is None else saved
+    nb = workspace_bytes(M, D, E, F, 1)
+    ws = _u8((nb,), dev) if workspace is None else workspace
+    st = _saved_struct(saved)
+    _check(lib().moe_mlp_fwd(_ptr(x), M, D, _ptr(w13), _ptr(w2), E, F, _ptr(offsets), pad_multiple, _ptr(y),
+                             ctypes.byref(st), _ptr(ws), ws.numel(), _stream(x)))
+    return y, saved
+
+
+def moe_mlp_bwd(dy, w13, w2, offsets, saved, pad_multiple=128, dx=None, dw13=None, dw2=None, workspace=None):
+    """Backward of the routed-experts MLP. Returns (dx, dw13, dw2) in bf16."""
+    E = _offs(offsets)
+    for t, n in ((dy, "dy"), (w13, "w13"), (w2, "w2")):
+        _need(t, torch.bfloat16, n)
+    M, D = dy.shape
+    F = w13.shape[1] // 2
+    dev = dy.device
+    dx = torch.empty(M, D, dtype=torch.bfloat16, device=dev) if dx is None else dx
+    dw13 = torch.empty_like(w13) if dw13 is None else dw13
+    dw2 = torch.empty_like(w2) if dw2 is None else dw2
+    nb = workspace_bytes(M, D, E, F, 2)
+    ws = _u8((nb,), dev) if workspace is None else workspace
+    st = _saved_struct(saved)
+    _check(lib().moe_mlp_bwd(_ptr(dy), M, D, _ptr(w13), _ptr(w2), E, F, _ptr(offsets), pad_multiple,
+                             ctypes.byref(st), _ptr(dx), _ptr(dw13), _ptr(dw2), _ptr(ws), ws.numel(), _stream(dy)))
+    return dx, dw13, dw2

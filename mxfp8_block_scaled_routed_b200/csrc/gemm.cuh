@@ -1,0 +1,473 @@
+// Persistent MXFP8 grouped GEMM on the sm_100a tensor cores (tcgen05
+// block-scaled MMA, fp32 accumulators in TMEM, TMA-fed shared-memory tiles).
+//
+// Covers the four grouped-GEMM ops of the fully-fused plan (torchtitan page
+// "Wire the fully-fused grouped-GEMM MXFP8 plan behind fusion_plan", section
+// "What it adds"): FC1 + SwiGLU + dual quantization, FC2, the dgrad with the
+// fused dSwiGLU backward, and the wgrad over the ragged token dimension.
+//
+// Two schedules over the expert-major padded token layout:
+//  * ragged M: out[m, :] = A[m, :] . B[e]^T for the rows m of expert e
+//    (A = tokens x K, B = per-expert weights [E, N, K]); an M tile of 128
+//    rows never straddles two experts because segments are padded to 128.
+//    Zero-token experts own no M tile and are skipped.
+//  * ragged K: out[e] = A_e^T . B_e over expert e's token rows, with both
+//    operands column-quantized and stored transposed ([N, M] and [Kx, M]) so
+//    the token dimension is the contiguous contraction.  Experts without rows
+//    write exact zeros.
+//
+// CTA = 8 warps: warp 0 issues TMA/bulk copies, warp 1 issues tcgen05.mma,
+// warp 2 owns the TMEM allocation, warps 4..7 run the epilogue (warp 4+q
+// reads TMEM lanes 32q..32q+31, i.e. rows 32q.. of the 128-row tile).
+// Tile: 128 x BN x 128 (M x N x K bytes), 128-byte swizzled K-major operands.
+// The E8M0 scales arrive as 512-byte atoms (MMA scale layout), are copied to
+// TMEM with tcgen05.cp and consumed by the block-scaled MMA (scale id = the
+// 32-wide K step inside the 128-wide K block).
+#pragma once
+#include <cuda.h>
+#include "mx_common.cuh"
+#include "sm100.cuh"
+
+namespace mxmoe::gemm {
+
+using namespace mxmoe::sm100;
+
+enum Mode : int { kRaggedM = 0, kRaggedK = 1 };
+enum Epi : int { kEpiBF16 = 0, kEpiSwiGLU = 1, kEpiDSwiGLU = 2 };
+
+constexpr int kErrOffsets = 4;
+constexpr int kErrTimeout = 7;
+
+struct Params {
+  int E;
+  int64_t rows_a;     // ragged M: M (token rows); ragged K: N (rows of A^T)
+  int64_t kext;       // K extent of A and B (ragged M: K; ragged K: M)
+  int64_t n_out;      // ragged M: N (B rows per expert; 2F for SwiGLU); ragged K: Kx
+  int64_t M;          // token rows of the buffer (bounds the offsets)
+  const int32_t* offsets;
+  int pad;
+  const uint8_t* a_scales;
+  const uint8_t* b_scales;
+  // epilogue
+  uint16_t* out;          // bf16 output (BF16 epilogue), h13 out (SwiGLU, may be null)
+  const uint16_t* h13;    // dSwiGLU input
+  int64_t F;              // SwiGLU / dSwiGLU intermediate size
+  uint8_t* row_codes;
+  uint8_t* row_scales;
+  uint8_t* col_codes;
+  uint8_t* col_scales;
+};
+
+template <int kMode, int kEpi, int BN>
+struct Cfg {
+  static constexpr int BM = 128, BK = 128;
+  static constexpr int kAcc = (BN == 256) ? 1 : 2;
+  static constexpr int kStages = (BN == 256) ? 4 : 6;
+  static constexpr int A_BYTES = BM * BK;
+  static constexpr int B_BYTES = BN * BK;
+  static constexpr int SFA_BYTES = 512;
+  static constexpr int SFB_BYTES = (BN / 128) * 512;
+  static constexpr int SF_COLS = 4 + BN / 32;           // TMEM columns for one SF buffer
+  static constexpr int ACC_COLS = kAcc * BN;
+  static constexpr int TMEM_COLS = 512;
+  static_assert(ACC_COLS + 2 * SF_COLS <= TMEM_COLS, "TMEM budget");
+  // shared memory map (offsets from a 1024-aligned base)
+  static constexpr int OFF_A = 0;
+  static constexpr int OFF_B = OFF_A + kStages * A_BYTES;
+  static constexpr int OFF_SFA = OFF_B + kStages * B_BYTES;
+  static constexpr int OFF_SFB = OFF_SFA + kStages * SFA_BYTES;
+  static constexpr int OFF_EPI = OFF_SFB + kStages * SFB_BYTES;
+  static constexpr int EPI_BYTES = 4 * 32 * 17 * 4;        // per-warp 32x32 bf16 transpose buffer
+  static constexpr int OFF_BAR = OFF_EPI + EPI_BYTES;
+  static constexpr int NUM_BARS = 2 * kStages + 2 * kAcc;
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+  static constexpr int OFF_OFFS = OFF_MISC + 16;
+  static constexpr int MAX_E = 1024;
+  static constexpr int SMEM_BYTES = OFF_OFFS + (MAX_E + 1) * 4 + 1024;  // + alignment slack
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+// ---------------------------------------------------------------- tile schedule
+struct Tile {
+  int e;
+  int nk;           // K blocks of 128
+  int64_t a_row;    // first A row of the tile
+  int64_t b_row0;   // first B row of box 0
+  int64_t b_row1;   // first B row of box 1 (BN == 256)
+  int64_t k0;       // first K element
+  int64_t out_r0;   // first output row
+  int64_t out_c0;   // first output column (SwiGLU: first f)
+};
+
+template <int kMode, int kEpi, int BN>
+__device__ __forceinline__ int64_t num_tiles(const Params& p, const int32_t* offs) {
+  if constexpr (kMode == kRaggedM) {
+    const int64_t nt = (kEpi == kEpiSwiGLU) ? p.F / 128 : p.n_out / BN;
+    return (int64_t(offs[p.E]) / 128) * nt;
+  } else {
+    return int64_t(p.E) * (p.rows_a / 128) * (p.n_out / BN);
+  }
+}
+
+template <int kMode, int kEpi, int BN>
+__device__ __forceinline__ Tile get_tile(const Params& p, const int32_t* offs, int64_t t) {
+  Tile T;
+  if constexpr (kMode == kRaggedM) {
+    const int64_t nt = (kEpi == kEpiSwiGLU) ? p.F / 128 : p.n_out / BN;
+    const int64_t mt = t / nt, ntile = t % nt;
+    const int64_t m0 = mt * 128;
+    int lo = 0, hi = p.E;  // last e with offs[e] <= m0
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (offs[mid] <= m0) lo = mid; else hi = mid;
+    }
+    T.e = lo;
+    T.nk = int(p.kext / 128);
+    T.k0 = 0;
+    T.a_row = m0;
+    T.out_r0 = m0;
+    if constexpr (kEpi == kEpiSwiGLU) {
+      const int64_t f0 = ntile * 128;
+      T.b_row0 = int64_t(T.e) * 2 * p.F + f0;          // gate rows
+      T.b_row1 = int64_t(T.e) * 2 * p.F + p.F + f0;    // up rows
+      T.out_c0 = f0;
+    } else {
+      T.b_row0 = int64_t(T.e) * p.n_out + ntile * BN;
+      T.b_row1 = T.b_row0 + 128;
+      T.out_c0 = ntile * BN;
+    }
+  } else {
+    const int64_t nn = p.rows_a / 128, nj = p.n_out / BN;
+    const int64_t e = t / (nn * nj), rem = t % (nn * nj);
+    const int64_t nt = rem / nj, jt = rem % nj;
+    T.e = int(e);
+    T.k0 = offs[e];
+    T.nk = int((offs[e + 1] - offs[e]) / 128);
+    T.a_row = nt * 128;
+    T.b_row0 = jt * BN;
+    T.b_row1 = jt * BN + 128;
+    T.out_r0 = nt * 128;
+    T.out_c0 = jt * BN;
+  }
+  return T;
+}
+
+// ---------------------------------------------------------------- epilogue helpers
+// Warp-level 32x32 transpose through shared memory: each lane gives one row
+// of 16 packed bf16 pairs; each lane gets one column as 16 packed pairs.
+__device__ __forceinline__ void warp_transpose32(uint32_t* buf, const uint32_t (&row)[16], uint32_t (&col)[16],
+                                                 int lane) {
+#pragma unroll
+  for (int j = 0; j < 16; ++j) buf[lane * 17 + j] = row[j];
+  __syncwarp();
+  const int w = lane >> 1, sh = (lane & 1) * 16;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const uint32_t lo = (buf[(2 * j) * 17 + w] >> sh) & 0xFFFFu;
+    const uint32_t hi = (buf[(2 * j + 1) * 17 + w] >> sh) & 0xFFFFu;
+    col[j] = lo | (hi << 16);
+  }
+  __syncwarp();
+}
+
+// Quantize 32 packed bf16 (16 words) of one block: returns the scale byte and
+// writes 32 codes to dst (16-byte aligned).
+__device__ __forceinline__ uint32_t quant32_store(const uint32_t (&v)[16], uint8_t* dst) {
+  uint4 q[4];
+  uint32_t am = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    q[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+    am = max(am, absmax_bits8(q[i]));
+  }
+  const uint32_t byte = scale_byte_from_bits(am);
+  uint2 c0 = encode8(q[0], byte), c1 = encode8(q[1], byte);
+  uint2 c2 = encode8(q[2], byte), c3 = encode8(q[3], byte);
+  reinterpret_cast<uint4*>(dst)[0] = make_uint4(c0.x, c0.y, c1.x, c1.y);
+  reinterpret_cast<uint4*>(dst)[1] = make_uint4(c2.x, c2.y, c3.x, c3.y);
+  return byte;
+}
+
+__device__ __forceinline__ void store64(uint16_t* dst, const uint32_t (&v)[16]) {
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) d[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+}
+
+__device__ __forceinline__ void load64(const uint16_t* src, uint32_t (&v)[16]) {
+  const uint4* s = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint4 t = s[i];
+    v[4 * i] = t.x; v[4 * i + 1] = t.y; v[4 * i + 2] = t.z; v[4 * i + 3] = t.w;
+  }
+}
+
+// ROW + COL quantization of a 32x32 bf16 block held one row per lane.
+// ROW: codes at row_codes[(row) * ld_row + col0], scale (row, col0/32) of a
+// [*, ld_row] matrix.  COL: codes at col_codes[(col0 + lane) * M + m_blk],
+// scale (col0 + lane, m_blk/32) of a [*, M] matrix.
+__device__ __forceinline__ void dual_quant_block(const uint32_t (&v)[16], int lane, uint32_t* tbuf,
+                                                 int64_t row, int64_t col0, int64_t ld_row, int64_t m_blk,
+                                                 int64_t M, uint8_t* row_codes, uint8_t* row_scales,
+                                                 uint8_t* col_codes, uint8_t* col_scales) {
+  const uint32_t rb = quant32_store(v, row_codes + row * ld_row + col0);
+  row_scales[mma_scale_offset(row, col0 >> 5, ld_row)] = uint8_t(rb);
+  uint32_t c[16];
+  warp_transpose32(tbuf, v, c, lane);
+  const int64_t crow = col0 + lane;
+  const uint32_t cb = quant32_store(c, col_codes + crow * M + m_blk);
+  col_scales[mma_scale_offset(crow, m_blk >> 5, M)] = uint8_t(cb);
+}
+
+// ---------------------------------------------------------------- the kernel
+template <int kMode, int kEpi, int BN>
+__global__ void __launch_bounds__(256, 1)
+grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                    const Params p) {
+  using C = Cfg<kMode, kEpi, BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  auto full_bar = [&](int s) { return smem_u32(&bars[s]); };
+  auto empty_bar = [&](int s) { return smem_u32(&bars[C::kStages + s]); };
+  auto tfull_bar = [&](int a) { return smem_u32(&bars[2 * C::kStages + a]); };
+  auto tempty_bar = [&](int a) { return smem_u32(&bars[2 * C::kStages + C::kAcc + a]); };
+  volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(smem + C::OFF_MISC);
+  int32_t* offs = reinterpret_cast<int32_t*>(smem + C::OFF_OFFS);
+
+  // ---- offsets into shared memory + validation (every CTA checks)
+  bool bad = p.E > C::MAX_E;
+  if (!bad) {
+    for (int i = threadIdx.x; i <= p.E; i += blockDim.x) offs[i] = p.offsets[i];
+  }
+  __syncthreads();
+  if (!bad) {
+    for (int i = threadIdx.x; i <= p.E; i += blockDim.x) {
+      const int32_t o = offs[i];
+      if (o < 0 || (o % p.pad) != 0 || int64_t(o) > p.M) bad = true;
+      if (i == 0 && o != 0) bad = true;
+      if (i < p.E && offs[i + 1] < o) bad = true;
+    }
+  }
+  if (__syncthreads_or(bad)) {
+    if (threadIdx.x == 0 && blockIdx.x == 0) raise_device_error(kErrOffsets);
+    return;
+  }
+
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmap_a);
+    prefetch_tmap(&tmap_b);
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int a = 0; a < C::kAcc; ++a) {
+      mbar_init(tfull_bar(a), 1);
+      mbar_init(tempty_bar(a), 128);
+    }
+    misc[1] = 0;  // abort flag
+    fence_mbar_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(smem_u32(const_cast<uint32_t*>(misc)), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = misc[0];
+  const int64_t ntiles = num_tiles<kMode, kEpi, BN>(p, offs);
+
+  if (warp == 0) {
+    // ================= producer =================
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        const Tile T = get_tile<kMode, kEpi, BN>(p, offs, t);
+        for (int kb = 0; kb < T.nk; ++kb) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1)) { ok = false; break; }
+          const uint32_t fb = full_bar(stage);
+          mbar_arrive_expect_tx(fb, C::A_BYTES + C::B_BYTES + C::SFA_BYTES + C::SFB_BYTES);
+          const int64_t k = T.k0 + int64_t(kb) * 128;
+          tma_load_2d(sbase + C::OFF_A + stage * C::A_BYTES, &tmap_a, fb, int(k), int(T.a_row));
+          tma_load_2d(sbase + C::OFF_B + stage * C::B_BYTES, &tmap_b, fb, int(k), int(T.b_row0));
+          if constexpr (BN == 256)
+            tma_load_2d(sbase + C::OFF_B + stage * C::B_BYTES + 16384, &tmap_b, fb, int(k), int(T.b_row1));
+          const int64_t katoms = p.kext / 128, kat = k / 128;
+          bulk_load(sbase + C::OFF_SFA + stage * C::SFA_BYTES,
+                    p.a_scales + ((T.a_row / 128) * katoms + kat) * 512, 512, fb);
+          bulk_load(sbase + C::OFF_SFB + stage * C::SFB_BYTES,
+                    p.b_scales + ((T.b_row0 / 128) * katoms + kat) * 512, 512, fb);
+          if constexpr (BN == 256)
+            bulk_load(sbase + C::OFF_SFB + stage * C::SFB_BYTES + 512,
+                      p.b_scales + ((T.b_row1 / 128) * katoms + kat) * 512, 512, fb);
+          if (++stage == C::kStages) { stage = 0; phase ^= 1; }
+        }
+      }
+      if (!ok) { misc[1] = 1; raise_device_error(kErrTimeout); }
+    }
+  } else if (warp == 1) {
+    // ================= MMA issuer =================
+    if (lane == 0) {
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      uint32_t sfbuf = 0;
+      bool ok = true;
+      const uint32_t sf_col0 = C::ACC_COLS;
+      for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        const Tile T = get_tile<kMode, kEpi, BN>(p, offs, t);
+        if (T.nk == 0) continue;
+        if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = 0; kb < T.nk; ++kb) {
+          if (!mbar_wait(full_bar(stage), phase)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sfa_t = tmem_base + sf_col0 + sfbuf * C::SF_COLS;
+          const uint32_t sfb_t = sfa_t + 4;
+          const uint32_t sfa_s = sbase + C::OFF_SFA + stage * C::SFA_BYTES;
+          const uint32_t sfb_s = sbase + C::OFF_SFB + stage * C::SFB_BYTES;
+          utccp_32x128b_warpx4(sfa_t, smem_desc(sfa_s, 0, 128, 0));
+#pragma unroll
+          for (int j = 0; j < BN / 128; ++j)
+            utccp_32x128b_warpx4(sfb_t + 4 * j, smem_desc(sfb_s + 512 * j, 0, 128, 0));
+          const uint32_t a_s = sbase + C::OFF_A + stage * C::A_BYTES;
+          const uint32_t b_s = sbase + C::OFF_B + stage * C::B_BYTES;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint64_t ad = smem_desc(a_s + k * 32, 0, 1024, 2);
+            const uint64_t bd = smem_desc(b_s + k * 32, 0, 1024, 2);
+            mma_mxf8(d_tmem, ad, bd, mxf8_idesc(128, BN, k), sfa_t, sfb_t, (kb | k) != 0);
+          }
+          mma_commit(empty_bar(stage));
+          sfbuf ^= 1;
+          if (++stage == C::kStages) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        mma_commit(tfull_bar(acc));
+        if (++acc == C::kAcc) { acc = 0; acc_phase ^= 1; }
+      }
+      if (!ok) { misc[1] = 1; raise_device_error(kErrTimeout); }
+    }
+  } else if (warp >= 4) {
+    // ================= epilogue =================
+    const int q = warp - 4;                 // TMEM lane quarter
+    const int r_in = q * 32 + lane;         // row inside the 128-row tile
+    uint32_t* tbuf = reinterpret_cast<uint32_t*>(smem + C::OFF_EPI) + q * 32 * 17;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x) {
+      const Tile T = get_tile<kMode, kEpi, BN>(p, offs, t);
+      if constexpr (kMode == kRaggedK) {
+        if (T.nk == 0) {
+          // expert without rows: its weight gradient is exactly zero
+          uint16_t* o = p.out + (int64_t(T.e) * p.rows_a + T.out_r0 + r_in) * p.n_out + T.out_c0;
+          for (int c = 0; c < BN; c += 8) *reinterpret_cast<uint4*>(o + c) = make_uint4(0, 0, 0, 0);
+          continue;
+        }
+      }
+      // warp-uniform outcome: the tcgen05.ld below are .sync.aligned
+      if (!__all_sync(0xffffffffu, mbar_wait(tfull_bar(acc), acc_phase))) {
+        raise_device_error(kErrTimeout);
+        break;
+      }
+      tc_fence_after();
+      const uint32_t t_row = tmem_base + (uint32_t(q * 32) << 16) + acc * BN;
+      if constexpr (kEpi == kEpiBF16) {
+        uint16_t* o;
+        if constexpr (kMode == kRaggedK)
+          o = p.out + (int64_t(T.e) * p.rows_a + T.out_r0 + r_in) * p.n_out + T.out_c0;
+        else
+          o = p.out + (T.out_r0 + r_in) * p.n_out + T.out_c0;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(t_row + c, r);
+          tmem_wait_ld();
+          uint32_t w[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) w[j] = pack_bf16x2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
+          store64(o + c, w);
+        }
+      } else if constexpr (kEpi == kEpiSwiGLU) {
+        const int64_t m = T.out_r0 + r_in;
+        const int64_t F = p.F;
+#pragma unroll 1
+        for (int c = 0; c < 128; c += 32) {
+          uint32_t g[32], u[32];
+          tmem_ld_32x32b_x32(t_row + c, g);
+          tmem_ld_32x32b_x32(t_row + 128 + c, u);
+          tmem_wait_ld();
+          uint32_t a2[16], b2[16], h2[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            a2[j] = pack_bf16x2(__uint_as_float(g[2 * j]), __uint_as_float(g[2 * j + 1]));
+            b2[j] = pack_bf16x2(__uint_as_float(u[2 * j]), __uint_as_float(u[2 * j + 1]));
+            h2[j] = pack_bf16x2(silu_mul(bf16lo_to_f32(a2[j]), bf16lo_to_f32(b2[j])),
+                                silu_mul(bf16hi_to_f32(a2[j]), bf16hi_to_f32(b2[j])));
+          }
+          const int64_t f = T.out_c0 + c;
+          if (p.out != nullptr) {
+            store64(p.out + m * 2 * F + f, a2);
+            store64(p.out + m * 2 * F + F + f, b2);
+          }
+          dual_quant_block(h2, lane, tbuf, m, f, F, T.out_r0 + q * 32, p.M, p.row_codes, p.row_scales,
+                           p.col_codes, p.col_scales);
+        }
+      } else {  // kEpiDSwiGLU
+        const int64_t m = T.out_r0 + r_in;
+        const int64_t F = p.F;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          const int64_t f = T.out_c0 + c;
+          uint32_t ha[16], hb[16];
+          load64(p.h13 + m * 2 * F + f, ha);
+          load64(p.h13 + m * 2 * F + F + f, hb);
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(t_row + c, r);
+          tmem_wait_ld();
+          uint32_t dg[16], du[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            float d[2], a[2], b[2], og[2], ou[2];
+            d[0] = round_bf16(__uint_as_float(r[2 * j]));
+            d[1] = round_bf16(__uint_as_float(r[2 * j + 1]));
+            a[0] = bf16lo_to_f32(ha[j]); a[1] = bf16hi_to_f32(ha[j]);
+            b[0] = bf16lo_to_f32(hb[j]); b[1] = bf16hi_to_f32(hb[j]);
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+              const float s = 1.0f / (1.0f + expf(-a[i]));
+              og[i] = d[i] * b[i] * s * (1.0f + a[i] * (1.0f - s));
+              ou[i] = d[i] * a[i] * s;
+            }
+            dg[j] = pack_bf16x2(og[0], og[1]);
+            du[j] = pack_bf16x2(ou[0], ou[1]);
+          }
+          dual_quant_block(dg, lane, tbuf, m, f, 2 * F, T.out_r0 + q * 32, p.M, p.row_codes, p.row_scales,
+                           p.col_codes, p.col_scales);
+          dual_quant_block(du, lane, tbuf, m, F + f, 2 * F, T.out_r0 + q * 32, p.M, p.row_codes,
+                           p.row_scales, p.col_codes, p.col_scales);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(tempty_bar(acc));
+      if (++acc == C::kAcc) { acc = 0; acc_phase ^= 1; }
+    }
+  }
+
+  // ---- teardown: every role has left its loop (all waits are bounded)
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+}  // namespace mxmoe::gemm

@@ -1,0 +1,110 @@
+// Device-side MXFP8 helpers shared by the cast and GEMM-epilogue kernels.
+//
+// MXFP8 block (A2E MXFP8 pages: E4M3 elements with an E8M0 block scale):
+// 32 elements share one power-of-two scale 2^s with s = floor(log2(amax)) - 8,
+// stored as the byte s + 127 clamped to [0, 254]; elements are x / 2^s rounded
+// to nearest-even E4M3 and saturated to +-448.  A block holding NaN/Inf gets
+// byte 0xFF and codes 0x7F | sign.
+#pragma once
+#include <cstdint>
+#include <cuda_bf16.h>
+
+namespace mxmoe {
+
+constexpr int kBlock = 32;
+
+// Device-side error word, one per device that loaded the library.
+__device__ int g_device_error;
+
+__device__ __forceinline__ void raise_device_error(int code) {
+  atomicCAS(&g_device_error, 0, code);
+}
+
+// ---------------------------------------------------------------- bf16 bits
+__device__ __forceinline__ float bf16lo_to_f32(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi_to_f32(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Round-to-nearest-even fp32 -> bf16 (hardware cvt), packed pair (lo = a).
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(b), "f"(a));
+  return r;
+}
+__device__ __forceinline__ float round_bf16(float a) {
+  return __bfloat162float(__float2bfloat16_rn(a));
+}
+
+// max over |x| of eight packed bf16 (uint4) as a 15-bit magnitude pattern.
+// For non-negative floats the integer order of the bit patterns is the
+// numeric order, and NaN/Inf (>= 0x7F80) sort above every finite value.
+__device__ __forceinline__ uint32_t absmax_bits8(uint4 v) {
+  const uint32_t m = 0x7FFF7FFFu;
+  uint32_t a = __vmaxu2(v.x & m, v.y & m);
+  uint32_t b = __vmaxu2(v.z & m, v.w & m);
+  a = __vmaxu2(a, b);
+  return max(a & 0xFFFFu, a >> 16);
+}
+
+// E8M0 byte from the 15-bit magnitude pattern of the block maximum.
+// floor(log2(amax)) is the unbiased exponent field, so the byte is
+// max(expfield - 8, 0); subnormal or zero maxima land on 0 via the clamp.
+// Returns 0xFF for NaN/Inf blocks.
+__device__ __forceinline__ uint32_t scale_byte_from_bits(uint32_t amax_bits) {
+  if (amax_bits >= 0x7F80u) return 0xFFu;
+  int e = int(amax_bits >> 7) - 8;
+  return uint32_t(e < 0 ? 0 : e);
+}
+
+// 2^-(byte-127) as fp32 (exact; byte in [0, 254] -> exponent in [-127, 127]).
+__device__ __forceinline__ float inv_scale_from_byte(uint32_t byte) {
+  return __uint_as_float((254u - byte) << 23);
+}
+
+// Two fp32 -> two E4M3 codes (nearest-even, saturating), lo byte = a.
+__device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(b), "f"(a));
+  return r;
+}
+
+// Eight packed bf16 -> eight E4M3 codes (uint2), scaled by inv (a power of two).
+__device__ __forceinline__ uint2 quant8_bf16(uint4 v, float inv) {
+  uint2 out;
+  out.x = e4m3x2(bf16lo_to_f32(v.x) * inv, bf16hi_to_f32(v.x) * inv) |
+          (e4m3x2(bf16lo_to_f32(v.y) * inv, bf16hi_to_f32(v.y) * inv) << 16);
+  out.y = e4m3x2(bf16lo_to_f32(v.z) * inv, bf16hi_to_f32(v.z) * inv) |
+          (e4m3x2(bf16lo_to_f32(v.w) * inv, bf16hi_to_f32(v.w) * inv) << 16);
+  return out;
+}
+
+// NaN codes (0x7F | sign) for eight packed bf16.
+__device__ __forceinline__ uint2 nan8_bf16(uint4 v) {
+  auto s = [](uint32_t w) {
+    return ((w >> 8) & 0x80u) | ((w >> 16) & 0x8000u);
+  };
+  uint2 out;
+  out.x = (s(v.x) | (s(v.y) << 16)) | 0x7F7F7F7Fu;
+  out.y = (s(v.z) | (s(v.w) << 16)) | 0x7F7F7F7Fu;
+  return out;
+}
+
+// Quantize 8 packed bf16 given the block's scale byte.
+__device__ __forceinline__ uint2 encode8(uint4 v, uint32_t byte) {
+  return byte == 0xFFu ? nan8_bf16(v) : quant8_bf16(v, inv_scale_from_byte(byte));
+}
+
+// ---------------------------------------------------------------- layouts
+// Byte offset of the scale of row r, 32-column block kb in the MMA (tensor
+// core) scale layout of a matrix with `kcols` columns (kcols % 128 == 0).
+__device__ __forceinline__ int64_t mma_scale_offset(int64_t r, int64_t kb, int64_t kcols) {
+  const int64_t atom = (r >> 7) * (kcols >> 7) + (kb >> 2);
+  return atom * 512 + ((r & 31) << 4) + (((r >> 5) & 3) << 2) + (kb & 3);
+}
+
+// ---------------------------------------------------------------- SwiGLU
+// h = bf16(silu(a) * b) in fp32 with IEEE division and expf.
+__device__ __forceinline__ float silu_mul(float a, float b) {
+  return a / (1.0f + expf(-a)) * b;
+}
+
+}  // namespace mxmoe

@@ -1,0 +1,569 @@
+// libmxmoe: C ABI of the MXFP8 routed-experts MLP (declared in include/mxmoe.h).
+//
+// One translation unit: the cast kernels (quant.cuh), the tcgen05 grouped
+// GEMM (gemm.cuh) and the host code below, which validates every argument,
+// encodes the TMA tensor maps, launches on the caller's stream and chains
+// the forward/backward composites.  Nothing here allocates device memory.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/mxmoe.h"
+#include "gemm.cuh"
+#include "quant.cuh"
+
+using namespace mxmoe;
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+int fail(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(MXMOE_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+#define MX_CHECK_CUDA(call, what)              \
+  do {                                         \
+    cudaError_t e_ = (call);                   \
+    if (e_ != cudaSuccess) return cuda_fail(e_, what); \
+  } while (0)
+
+#define MX_TRY(expr)          \
+  do {                        \
+    int s_ = (expr);          \
+    if (s_ != MXMOE_OK) return s_; \
+  } while (0)
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+constexpr int kMaxDevices = 64;
+struct DevInfo {
+  int checked = 0;   // 1 ok, -1 wrong arch
+  int sms = 0;
+  unsigned attr_set = 0;  // bitmask of kernel instantiations with smem attribute set
+};
+DevInfo g_dev[kMaxDevices];
+std::mutex g_mu;
+
+int device_info(DevInfo** out) {
+  int dev = 0;
+  MX_CHECK_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(MXMOE_ERR_CUDA, "device index %d out of range", dev);
+  std::lock_guard<std::mutex> lk(g_mu);
+  DevInfo& d = g_dev[dev];
+  if (d.checked == 0) {
+    int major = 0, minor = 0, sms = 0;
+    MX_CHECK_CUDA(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev), "attr");
+    MX_CHECK_CUDA(cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev), "attr");
+    MX_CHECK_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev), "attr");
+    d.sms = sms;
+    d.checked = (major == 10 && minor == 0) ? 1 : -1;
+  }
+  if (d.checked < 0) return fail(MXMOE_ERR_ARCH, "device %d is not sm_100 (this library is built for sm_100a)", dev);
+  *out = &d;
+  return MXMOE_OK;
+}
+
+// ---------------------------------------------------------------- TMA tensor maps
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+int get_encode(EncodeTiledFn* fn) {
+  static EncodeTiledFn cached = nullptr;
+  static std::once_flag once;
+  static cudaError_t err = cudaSuccess;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    err = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+    if (err == cudaSuccess && q == cudaDriverEntryPointSuccess) cached = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  if (!cached) return fail(MXMOE_ERR_CUDA, "cuTensorMapEncodeTiled unavailable (%s)", cudaGetErrorString(err));
+  *fn = cached;
+  return MXMOE_OK;
+}
+
+// 2-D uint8 K-major operand [rows, kext], box 128 x 128 bytes, 128-byte swizzle.
+int make_operand_map(CUtensorMap* map, const uint8_t* base, int64_t rows, int64_t kext) {
+  EncodeTiledFn enc;
+  MX_TRY(get_encode(&enc));
+  cuuint64_t dims[2] = {cuuint64_t(kext), cuuint64_t(rows)};
+  cuuint64_t strides[1] = {cuuint64_t(kext)};
+  cuuint32_t box[2] = {128, 128};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MXMOE_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
+  return MXMOE_OK;
+}
+
+// ---------------------------------------------------------------- GEMM launch
+template <int kMode, int kEpi, int BN>
+int launch_gemm(const uint8_t* a, int64_t a_rows, const uint8_t* b, int64_t b_rows, gemm::Params p,
+                int64_t max_tiles, cudaStream_t stream, int attr_bit) {
+  using C = gemm::Cfg<kMode, kEpi, BN>;
+  DevInfo* d;
+  MX_TRY(device_info(&d));
+  auto kern = gemm::grouped_gemm_kernel<kMode, kEpi, BN>;
+  if (!(d->attr_set & (1u << attr_bit))) {
+    MX_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES),
+                  "cudaFuncSetAttribute");
+    std::lock_guard<std::mutex> lk(g_mu);
+    d->attr_set |= (1u << attr_bit);
+  }
+  if (p.E > C::MAX_E) return fail(MXMOE_ERR_SHAPE, "E=%d exceeds the supported maximum %d", p.E, C::MAX_E);
+  CUtensorMap ma, mb;
+  MX_TRY(make_operand_map(&ma, a, a_rows, p.kext));
+  MX_TRY(make_operand_map(&mb, b, b_rows, p.kext));
+  if (max_tiles <= 0) return MXMOE_OK;
+  const int grid = int(max_tiles < d->sms ? max_tiles : d->sms);
+  kern<<<grid, 256, C::SMEM_BYTES, stream>>>(ma, mb, p);
+  MX_CHECK_CUDA(cudaGetLastError(), "grouped GEMM launch");
+  return MXMOE_OK;
+}
+
+int check_offsets_args(const int32_t* offsets, int E, int pad) {
+  if (!offsets) return fail(MXMOE_ERR_NULL, "expert_offsets is NULL");
+  if (E <= 0) return fail(MXMOE_ERR_SHAPE, "E=%d must be positive", E);
+  if (pad < 128 || pad % 128 != 0)
+    return fail(MXMOE_ERR_SHAPE, "pad_multiple=%d must be a positive multiple of 128", pad);
+  return MXMOE_OK;
+}
+
+int check_mult(const char* name, int64_t v, int64_t m) {
+  if (v <= 0 || v % m != 0) return fail(MXMOE_ERR_SHAPE, "%s=%lld must be a positive multiple of %lld", name,
+                                        (long long)v, (long long)m);
+  return MXMOE_OK;
+}
+
+int check_ptrs(std::initializer_list<std::pair<const char*, const void*>> ps) {
+  for (auto& kv : ps) {
+    if (!kv.second) return fail(MXMOE_ERR_NULL, "%s is NULL", kv.first);
+    if (!aligned16(kv.second)) return fail(MXMOE_ERR_ALIGN, "%s is not 16-byte aligned", kv.first);
+  }
+  return MXMOE_OK;
+}
+
+// ---------------------------------------------------------------- casts
+int quantize_impl(const void* x, int64_t batch, int64_t rows, int64_t cols, int modes, int layout,
+                  uint8_t* rc, uint8_t* rs, uint8_t* cc, uint8_t* cs, cudaStream_t stream,
+                  bool swiglu = false) {
+  if (modes < 1 || modes > 3) return fail(MXMOE_ERR_ARG, "modes=%d must be MXFP8_ROW, MXFP8_COL or both", modes);
+  if (layout != MXFP8_SCALE_PLAIN && layout != MXFP8_SCALE_MMA)
+    return fail(MXMOE_ERR_ARG, "scale_layout=%d invalid", layout);
+  if (batch <= 0 || rows <= 0 || cols <= 0)
+    return fail(MXMOE_ERR_SHAPE, "batch=%lld rows=%lld cols=%lld must be positive", (long long)batch,
+                (long long)rows, (long long)cols);
+  if (!x) return fail(MXMOE_ERR_NULL, "input is NULL");
+  const bool row = modes & MXFP8_ROW, col = modes & MXFP8_COL;
+  if (row && (!rc || !rs)) return fail(MXMOE_ERR_NULL, "row_codes/row_scales NULL with MXFP8_ROW");
+  if (col && (!cc || !cs)) return fail(MXMOE_ERR_NULL, "col_codes/col_scales NULL with MXFP8_COL");
+  if (col && rows % 32 != 0) return fail(MXMOE_ERR_SHAPE, "MXFP8_COL needs rows %% 32 == 0 (rows=%lld)", (long long)rows);
+  if (layout == MXFP8_SCALE_MMA && (rows % 128 != 0 || cols % 128 != 0))
+    return fail(MXMOE_ERR_SHAPE, "MMA scale layout needs rows and cols multiples of 128 (%lld x %lld)",
+                (long long)rows, (long long)cols);
+  const bool vec_ok = cols % 32 == 0 && aligned16(x) && (!row || aligned16(rc)) && (!col || aligned16(cc)) &&
+                      (!col || rows % 16 == 0);
+  if (swiglu && !vec_ok) return fail(MXMOE_ERR_SHAPE, "SwiGLU quant needs F %% 32 == 0 and 16-byte aligned buffers");
+  const uint16_t* in = static_cast<const uint16_t*>(x);
+  DevInfo* d;
+  MX_TRY(device_info(&d));
+  if (!vec_ok) {
+    if (col) return fail(MXMOE_ERR_SHAPE, "MXFP8_COL needs cols %% 32 == 0 and 16-byte aligned buffers");
+    if (layout == MXFP8_SCALE_MMA) return fail(MXMOE_ERR_SHAPE, "MMA layout needs aligned buffers");
+    const int64_t R = batch * rows;
+    const int64_t warps = R * ((cols + 31) / 32);
+    const int64_t blocks = (warps * 32 + 255) / 256;
+    if (blocks > 0x7FFFFFFF) return fail(MXMOE_ERR_SHAPE, "tensor too large");
+    mx_row_generic_kernel<<<unsigned(blocks), 256, 0, stream>>>(in, R, cols, rc, rs);
+    MX_CHECK_CUDA(cudaGetLastError(), "cast launch");
+    return MXMOE_OK;
+  }
+  TileArgs a;
+  a.in = in;
+  a.rows = rows;
+  a.cols = cols;
+  a.ld_in = swiglu ? 2 * cols : cols;
+  a.up_off = swiglu ? cols : 0;
+  a.modes = modes;
+  a.mma_layout = layout;
+  a.row_codes = rc;
+  a.row_scales = rs;
+  a.col_codes = cc;
+  a.col_scales = cs;
+  a.dev_rows = nullptr;
+  dim3 grid(unsigned((cols + 127) / 128), unsigned((rows + 127) / 128), unsigned(batch));
+  if (grid.y > 65535 || grid.z > 65535) return fail(MXMOE_ERR_SHAPE, "tensor too large for the cast grid");
+  if (swiglu)
+    mx_tile_kernel<true><<<grid, kTileThreads, 0, stream>>>(a);
+  else
+    mx_tile_kernel<false><<<grid, kTileThreads, 0, stream>>>(a);
+  MX_CHECK_CUDA(cudaGetLastError(), "cast launch");
+  return MXMOE_OK;
+}
+
+// Cast of the token buffer used inside the composites: rows at or past
+// offsets[E] (read on the device) are neither read nor written.
+int quantize_tokens(const void* x, int64_t rows, int64_t cols, const int32_t* rows_dev, uint8_t* rc, uint8_t* rs,
+                    uint8_t* cc, uint8_t* cs, cudaStream_t stream) {
+  TileArgs a;
+  a.in = static_cast<const uint16_t*>(x);
+  a.rows = rows;
+  a.cols = cols;
+  a.ld_in = cols;
+  a.up_off = 0;
+  a.modes = MXFP8_ROW | MXFP8_COL;
+  a.mma_layout = 1;
+  a.row_codes = rc;
+  a.row_scales = rs;
+  a.col_codes = cc;
+  a.col_scales = cs;
+  a.dev_rows = rows_dev;
+  dim3 grid(unsigned(cols / 128), unsigned(rows / 128), 1);
+  mx_tile_kernel<false><<<grid, kTileThreads, 0, stream>>>(a);
+  MX_CHECK_CUDA(cudaGetLastError(), "cast launch");
+  return MXMOE_OK;
+}
+
+int gemm_ragged_m(const uint8_t* a, const uint8_t* as, int64_t M, int64_t K, const uint8_t* w,
+                  const uint8_t* ws, int E, int64_t N, const int32_t* offsets, int pad, void* out,
+                  cudaStream_t stream) {
+  gemm::Params p{};
+  p.E = E;
+  p.rows_a = M;
+  p.kext = K;
+  p.n_out = N;
+  p.M = M;
+  p.offsets = offsets;
+  p.pad = pad;
+  p.a_scales = as;
+  p.b_scales = ws;
+  p.out = static_cast<uint16_t*>(out);
+  if (N % 256 == 0)
+    return launch_gemm<gemm::kRaggedM, gemm::kEpiBF16, 256>(a, M, w, int64_t(E) * N, p, (M / 128) * (N / 256),
+                                                            stream, 0);
+  return launch_gemm<gemm::kRaggedM, gemm::kEpiBF16, 128>(a, M, w, int64_t(E) * N, p, (M / 128) * (N / 128),
+                                                          stream, 1);
+}
+
+int gemm_ragged_k(const uint8_t* gt, const uint8_t* gs, int64_t N, const uint8_t* xt, const uint8_t* xs,
+                  int64_t Kx, int64_t M, const int32_t* offsets, int E, int pad, void* dw, cudaStream_t stream) {
+  gemm::Params p{};
+  p.E = E;
+  p.rows_a = N;
+  p.kext = M;
+  p.n_out = Kx;
+  p.M = M;
+  p.offsets = offsets;
+  p.pad = pad;
+  p.a_scales = gs;
+  p.b_scales = xs;
+  p.out = static_cast<uint16_t*>(dw);
+  if (Kx % 256 == 0)
+    return launch_gemm<gemm::kRaggedK, gemm::kEpiBF16, 256>(gt, N, xt, Kx, p, int64_t(E) * (N / 128) * (Kx / 256),
+                                                            stream, 2);
+  return launch_gemm<gemm::kRaggedK, gemm::kEpiBF16, 128>(gt, N, xt, Kx, p, int64_t(E) * (N / 128) * (Kx / 128),
+                                                          stream, 3);
+}
+
+int gemm_swiglu(const uint8_t* a, const uint8_t* as, int64_t M, int64_t K, const uint8_t* w13, const uint8_t* ws,
+                int E, int64_t F, const int32_t* offsets, int pad, void* h13, uint8_t* hrc, uint8_t* hrs,
+                uint8_t* hcc, uint8_t* hcs, cudaStream_t stream) {
+  gemm::Params p{};
+  p.E = E;
+  p.rows_a = M;
+  p.kext = K;
+  p.n_out = 2 * F;
+  p.M = M;
+  p.offsets = offsets;
+  p.pad = pad;
+  p.a_scales = as;
+  p.b_scales = ws;
+  p.out = static_cast<uint16_t*>(h13);
+  p.F = F;
+  p.row_codes = hrc;
+  p.row_scales = hrs;
+  p.col_codes = hcc;
+  p.col_scales = hcs;
+  return launch_gemm<gemm::kRaggedM, gemm::kEpiSwiGLU, 256>(a, M, w13, int64_t(E) * 2 * F, p, (M / 128) * (F / 128),
+                                                            stream, 4);
+}
+
+int gemm_dswiglu(const uint8_t* dy, const uint8_t* ds, int64_t M, int64_t D, const uint8_t* w2t,
+                 const uint8_t* w2ts, int E, int64_t F, const int32_t* offsets, int pad, const void* h13,
+                 uint8_t* grc, uint8_t* grs, uint8_t* gcc, uint8_t* gcs, cudaStream_t stream) {
+  gemm::Params p{};
+  p.E = E;
+  p.rows_a = M;
+  p.kext = D;
+  p.n_out = F;
+  p.M = M;
+  p.offsets = offsets;
+  p.pad = pad;
+  p.a_scales = ds;
+  p.b_scales = w2ts;
+  p.h13 = static_cast<const uint16_t*>(h13);
+  p.F = F;
+  p.row_codes = grc;
+  p.row_scales = grs;
+  p.col_codes = gcc;
+  p.col_scales = gcs;
+  if (F % 256 == 0)
+    return launch_gemm<gemm::kRaggedM, gemm::kEpiDSwiGLU, 256>(dy, M, w2t, int64_t(E) * F, p, (M / 128) * (F / 256),
+                                                               stream, 5);
+  return launch_gemm<gemm::kRaggedM, gemm::kEpiDSwiGLU, 128>(dy, M, w2t, int64_t(E) * F, p, (M / 128) * (F / 128),
+                                                             stream, 6);
+}
+
+// ---------------------------------------------------------------- workspace
+struct Carver {
+  uint8_t* base;
+  size_t off = 0;
+  template <class T>
+  T* take(size_t bytes) {
+    off = (off + 255) & ~size_t(255);
+    T* r = reinterpret_cast<T*>(base ? base + off : nullptr);
+    off += bytes;
+    return r;
+  }
+};
+
+struct FwdWs {
+  uint8_t *x_rc, *x_rs, *w13_c, *w13_s, *w2_c, *w2_s, *h_rc, *h_rs;
+};
+struct BwdWs {
+  uint8_t *dy_rc, *dy_rs, *dy_cc, *dy_cs, *w2t_c, *w2t_s, *w13t_c, *w13t_s, *g_rc, *g_rs, *g_cc, *g_cs;
+};
+
+size_t carve_fwd(uint8_t* base, int64_t M, int64_t D, int E, int64_t F, FwdWs* w) {
+  Carver c{base};
+  w->x_rc = c.take<uint8_t>(M * D);
+  w->x_rs = c.take<uint8_t>(M * D / 32);
+  w->w13_c = c.take<uint8_t>(int64_t(E) * 2 * F * D);
+  w->w13_s = c.take<uint8_t>(int64_t(E) * 2 * F * D / 32);
+  w->w2_c = c.take<uint8_t>(int64_t(E) * D * F);
+  w->w2_s = c.take<uint8_t>(int64_t(E) * D * F / 32);
+  w->h_rc = c.take<uint8_t>(M * F);
+  w->h_rs = c.take<uint8_t>(M * F / 32);
+  return c.off + 256;
+}
+
+size_t carve_bwd(uint8_t* base, int64_t M, int64_t D, int E, int64_t F, BwdWs* w) {
+  Carver c{base};
+  w->dy_rc = c.take<uint8_t>(M * D);
+  w->dy_rs = c.take<uint8_t>(M * D / 32);
+  w->dy_cc = c.take<uint8_t>(M * D);
+  w->dy_cs = c.take<uint8_t>(M * D / 32);
+  w->w2t_c = c.take<uint8_t>(int64_t(E) * D * F);
+  w->w2t_s = c.take<uint8_t>(int64_t(E) * D * F / 32);
+  w->w13t_c = c.take<uint8_t>(int64_t(E) * 2 * F * D);
+  w->w13t_s = c.take<uint8_t>(int64_t(E) * 2 * F * D / 32);
+  w->g_rc = c.take<uint8_t>(M * 2 * F);
+  w->g_rs = c.take<uint8_t>(M * 2 * F / 32);
+  w->g_cc = c.take<uint8_t>(M * 2 * F);
+  w->g_cs = c.take<uint8_t>(M * 2 * F / 32);
+  return c.off + 256;
+}
+
+int check_mlp_shapes(int64_t M, int64_t D, int E, int64_t F, const int32_t* offsets, int pad) {
+  MX_TRY(check_offsets_args(offsets, E, pad));
+  MX_TRY(check_mult("M", M, 128));
+  MX_TRY(check_mult("D", D, 128));
+  MX_TRY(check_mult("F", F, 128));
+  return MXMOE_OK;
+}
+
+uint8_t* align_ws(void* ws) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(ws) + 255) & ~uintptr_t(255));
+}
+
+}  // namespace
+
+// =====================================================================================
+extern "C" {
+
+const char* mxmoe_last_error(void) { return g_err; }
+
+const char* mxmoe_version(void) { return "mxmoe 0.1 (sm_100a, tcgen05 block-scaled MXFP8)"; }
+
+int mxmoe_device_error(cudaStream_t stream, int reset, int* code) {
+  if (!code) return fail(MXMOE_ERR_NULL, "code is NULL");
+  MX_CHECK_CUDA(cudaStreamSynchronize(stream), "cudaStreamSynchronize");
+  int v = 0;
+  MX_CHECK_CUDA(cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int)), "read device error");
+  if (reset) {
+    const int z = 0;
+    MX_CHECK_CUDA(cudaMemcpyToSymbol(g_device_error, &z, sizeof(int)), "reset device error");
+  }
+  *code = v;
+  return MXMOE_OK;
+}
+
+int mxfp8_quantize(const void* x, int64_t batch, int64_t rows, int64_t cols, int modes, int scale_layout,
+                   uint8_t* row_codes, uint8_t* row_scales, uint8_t* col_codes, uint8_t* col_scales,
+                   cudaStream_t stream) {
+  return quantize_impl(x, batch, rows, cols, modes, scale_layout, row_codes, row_scales, col_codes, col_scales,
+                       stream);
+}
+
+int mxfp8_swiglu_quant(const void* h13, int64_t rows, int64_t F, int modes, int scale_layout, uint8_t* row_codes,
+                       uint8_t* row_scales, uint8_t* col_codes, uint8_t* col_scales, cudaStream_t stream) {
+  if (F % 32 != 0) return fail(MXMOE_ERR_SHAPE, "F=%lld must be a multiple of 32", (long long)F);
+  return quantize_impl(h13, 1, rows, F, modes, scale_layout, row_codes, row_scales, col_codes, col_scales, stream,
+                       true);
+}
+
+int mxfp8_dequantize(const uint8_t* codes, const uint8_t* scales, int64_t rows, int64_t cols, void* out,
+                     cudaStream_t stream) {
+  if (!codes || !scales || !out) return fail(MXMOE_ERR_NULL, "codes/scales/out is NULL");
+  if (rows <= 0 || cols <= 0) return fail(MXMOE_ERR_SHAPE, "rows and cols must be positive");
+  DevInfo* d;
+  MX_TRY(device_info(&d));
+  const int64_t n = rows * cols;
+  const int64_t blocks = (n + 255) / 256;
+  if (blocks > 0x7FFFFFFF) return fail(MXMOE_ERR_SHAPE, "tensor too large");
+  mx_dequant_kernel<<<unsigned(blocks), 256, 0, stream>>>(codes, scales, rows, cols, static_cast<uint16_t*>(out));
+  MX_CHECK_CUDA(cudaGetLastError(), "dequant launch");
+  return MXMOE_OK;
+}
+
+int mxfp8_grouped_gemm(const uint8_t* a, const uint8_t* a_scales, int64_t M, int64_t K, const uint8_t* w,
+                       const uint8_t* w_scales, int E, int64_t N, const int32_t* expert_offsets, int pad_multiple,
+                       void* out, cudaStream_t stream) {
+  MX_TRY(check_offsets_args(expert_offsets, E, pad_multiple));
+  MX_TRY(check_mult("M", M, 128));
+  MX_TRY(check_mult("K", K, 128));
+  MX_TRY(check_mult("N", N, 128));
+  MX_TRY(check_ptrs({{"a", a}, {"a_scales", a_scales}, {"w", w}, {"w_scales", w_scales}, {"out", out}}));
+  return gemm_ragged_m(a, a_scales, M, K, w, w_scales, E, N, expert_offsets, pad_multiple, out, stream);
+}
+
+int mxfp8_grouped_gemm_wgrad(const uint8_t* gt, const uint8_t* gt_scales, int64_t N, const uint8_t* xt,
+                             const uint8_t* xt_scales, int64_t Kx, int64_t M, const int32_t* expert_offsets, int E,
+                             int pad_multiple, void* dw, cudaStream_t stream) {
+  MX_TRY(check_offsets_args(expert_offsets, E, pad_multiple));
+  MX_TRY(check_mult("M", M, 128));
+  MX_TRY(check_mult("N", N, 128));
+  MX_TRY(check_mult("Kx", Kx, 128));
+  MX_TRY(check_ptrs({{"gt", gt}, {"gt_scales", gt_scales}, {"xt", xt}, {"xt_scales", xt_scales}, {"dw", dw}}));
+  return gemm_ragged_k(gt, gt_scales, N, xt, xt_scales, Kx, M, expert_offsets, E, pad_multiple, dw, stream);
+}
+
+int mxfp8_grouped_gemm_swiglu_quant(const uint8_t* a, const uint8_t* a_scales, int64_t M, int64_t K,
+                                    const uint8_t* w13, const uint8_t* w13_scales, int E, int64_t F,
+                                    const int32_t* expert_offsets, int pad_multiple, void* h13_out,
+                                    uint8_t* h_row_codes, uint8_t* h_row_scales, uint8_t* h_col_codes,
+                                    uint8_t* h_col_scales, cudaStream_t stream) {
+  MX_TRY(check_offsets_args(expert_offsets, E, pad_multiple));
+  MX_TRY(check_mult("M", M, 128));
+  MX_TRY(check_mult("K", K, 128));
+  MX_TRY(check_mult("F", F, 128));
+  MX_TRY(check_ptrs({{"a", a}, {"a_scales", a_scales}, {"w13", w13}, {"w13_scales", w13_scales},
+                     {"h_row_codes", h_row_codes}, {"h_row_scales", h_row_scales}, {"h_col_codes", h_col_codes},
+                     {"h_col_scales", h_col_scales}}));
+  if (h13_out && !aligned16(h13_out)) return fail(MXMOE_ERR_ALIGN, "h13_out is not 16-byte aligned");
+  return gemm_swiglu(a, a_scales, M, K, w13, w13_scales, E, F, expert_offsets, pad_multiple, h13_out, h_row_codes,
+                     h_row_scales, h_col_codes, h_col_scales, stream);
+}
+
+int mxfp8_grouped_gemm_dswiglu_quant(const uint8_t* dy, const uint8_t* dy_scales, int64_t M, int64_t D,
+                                     const uint8_t* w2t, const uint8_t* w2t_scales, int E, int64_t F,
+                                     const int32_t* expert_offsets, int pad_multiple, const void* h13,
+                                     uint8_t* g_row_codes, uint8_t* g_row_scales, uint8_t* g_col_codes,
+                                     uint8_t* g_col_scales, cudaStream_t stream) {
+  MX_TRY(check_offsets_args(expert_offsets, E, pad_multiple));
+  MX_TRY(check_mult("M", M, 128));
+  MX_TRY(check_mult("D", D, 128));
+  MX_TRY(check_mult("F", F, 128));
+  MX_TRY(check_ptrs({{"dy", dy}, {"dy_scales", dy_scales}, {"w2t", w2t}, {"w2t_scales", w2t_scales},
+                     {"h13", h13}, {"g_row_codes", g_row_codes}, {"g_row_scales", g_row_scales},
+                     {"g_col_codes", g_col_codes}, {"g_col_scales", g_col_scales}}));
+  return gemm_dswiglu(dy, dy_scales, M, D, w2t, w2t_scales, E, F, expert_offsets, pad_multiple, h13, g_row_codes,
+                      g_row_scales, g_col_codes, g_col_scales, stream);
+}
+
+size_t mxmoe_workspace_size(int64_t M, int64_t D, int E, int64_t F, int which) {
+  if (M <= 0 || D <= 0 || E <= 0 || F <= 0) return 0;
+  FwdWs f;
+  BwdWs b;
+  if (which == 1) return carve_fwd(nullptr, M, D, E, F, &f);
+  if (which == 2) return carve_bwd(nullptr, M, D, E, F, &b);
+  return 0;
+}
+
+int moe_mlp_fwd(const void* x, int64_t M, int64_t D, const void* w13, const void* w2, int E, int64_t F,
+                const int32_t* expert_offsets, int pad_multiple, void* y, const mxmoe_saved* saved, void* workspace,
+                size_t workspace_bytes, cudaStream_t stream) {
+  MX_TRY(check_mlp_shapes(M, D, E, F, expert_offsets, pad_multiple));
+  if (!saved) return fail(MXMOE_ERR_NULL, "saved is NULL");
+  MX_TRY(check_ptrs({{"x", x}, {"w13", w13}, {"w2", w2}, {"y", y}, {"saved.h13", saved->h13},
+                     {"saved.h_col_codes", saved->h_col_codes}, {"saved.h_col_scales", saved->h_col_scales},
+                     {"saved.x_col_codes", saved->x_col_codes}, {"saved.x_col_scales", saved->x_col_scales}}));
+  FwdWs w;
+  const size_t need = carve_fwd(nullptr, M, D, E, F, &w);
+  if (!workspace || workspace_bytes < need)
+    return fail(MXMOE_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed", workspace_bytes, need);
+  carve_fwd(align_ws(workspace), M, D, E, F, &w);
+  // a1: x -> ROW (FC1 operand) + COL (dW13 operand, saved)
+  MX_TRY(quantize_tokens(x, M, D, expert_offsets + E, w.x_rc, w.x_rs, saved->x_col_codes, saved->x_col_scales,
+                         stream));
+  // a2: weights, ROW along the contraction dimension of each forward GEMM
+  MX_TRY(quantize_impl(w13, 1, int64_t(E) * 2 * F, D, MXFP8_ROW, MXFP8_SCALE_MMA, w.w13_c, w.w13_s, nullptr,
+                       nullptr, stream));
+  MX_TRY(quantize_impl(w2, 1, int64_t(E) * D, F, MXFP8_ROW, MXFP8_SCALE_MMA, w.w2_c, w.w2_s, nullptr, nullptr,
+                       stream));
+  // a3: FC1 + SwiGLU + dual quantization
+  MX_TRY(gemm_swiglu(w.x_rc, w.x_rs, M, D, w.w13_c, w.w13_s, E, F, expert_offsets, pad_multiple, saved->h13,
+                     w.h_rc, w.h_rs, saved->h_col_codes, saved->h_col_scales, stream));
+  // a4: FC2
+  return gemm_ragged_m(w.h_rc, w.h_rs, M, F, w.w2_c, w.w2_s, E, D, expert_offsets, pad_multiple, y, stream);
+}
+
+int moe_mlp_bwd(const void* dy, int64_t M, int64_t D, const void* w13, const void* w2, int E, int64_t F,
+                const int32_t* expert_offsets, int pad_multiple, const mxmoe_saved* saved, void* dx, void* dw13,
+                void* dw2, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  MX_TRY(check_mlp_shapes(M, D, E, F, expert_offsets, pad_multiple));
+  if (!saved) return fail(MXMOE_ERR_NULL, "saved is NULL");
+  MX_TRY(check_ptrs({{"dy", dy}, {"w13", w13}, {"w2", w2}, {"dx", dx}, {"dw13", dw13}, {"dw2", dw2},
+                     {"saved.h13", saved->h13}, {"saved.h_col_codes", saved->h_col_codes},
+                     {"saved.h_col_scales", saved->h_col_scales}, {"saved.x_col_codes", saved->x_col_codes},
+                     {"saved.x_col_scales", saved->x_col_scales}}));
+  BwdWs w;
+  const size_t need = carve_bwd(nullptr, M, D, E, F, &w);
+  if (!workspace || workspace_bytes < need)
+    return fail(MXMOE_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed", workspace_bytes, need);
+  carve_bwd(align_ws(workspace), M, D, E, F, &w);
+  // a5: dY -> ROW (dh operand) + COL (dW2 operand)
+  MX_TRY(quantize_tokens(dy, M, D, expert_offsets + E, w.dy_rc, w.dy_rs, w.dy_cc, w.dy_cs, stream));
+  // a2 (backward): W2 COL along D, W13 COL along 2F, per expert
+  MX_TRY(quantize_impl(w2, E, D, F, MXFP8_COL, MXFP8_SCALE_MMA, nullptr, nullptr, w.w2t_c, w.w2t_s, stream));
+  MX_TRY(quantize_impl(w13, E, 2 * F, D, MXFP8_COL, MXFP8_SCALE_MMA, nullptr, nullptr, w.w13t_c, w.w13t_s, stream));
+  // a6: dh = dY . W2[e] with the fused dSwiGLU + dual quantization
+  MX_TRY(gemm_dswiglu(w.dy_rc, w.dy_rs, M, D, w.w2t_c, w.w2t_s, E, F, expert_offsets, pad_multiple, saved->h13,
+                      w.g_rc, w.g_rs, w.g_cc, w.g_cs, stream));
+  // a7: dW2[e] = dY_e^T . h_e
+  MX_TRY(gemm_ragged_k(w.dy_cc, w.dy_cs, D, saved->h_col_codes, saved->h_col_scales, F, M, expert_offsets, E,
+                       pad_multiple, dw2, stream));
+  // a8: dx = dh13 . W13[e]
+  MX_TRY(gemm_ragged_m(w.g_rc, w.g_rs, M, 2 * F, w.w13t_c, w.w13t_s, E, D, expert_offsets, pad_multiple, dx,
+                       stream));
+  // a9: dW13[e] = dh13_e^T . x_e
+  return gemm_ragged_k(w.g_cc, w.g_cs, 2 * F, saved->x_col_codes, saved->x_col_scales, D, M, expert_offsets, E,
+                       pad_multiple, dw13, stream);
+}
+
+}  // extern "C"

@@ -328,53 +328,32 @@ def quantize_weights_cols(w: np.ndarray):
 # ----------------------------------------------------------------------------
 # composites
 # ----------------------------------------------------------------------------
-def _seg_matmul(a, b_of_e, offsets, experts, n_out):
-    """out[seg_e] = a[seg_e] @ b_of_e(e) for each listed expert (float64)."""
-    out = np.full((a.shape[0], n_out), np.nan)
-    for e in _experts(offsets, experts):
-        lo, hi = int(offsets[e]), int(offsets[e + 1])
-        if hi > lo:
-            out[lo:hi] = a[lo:hi] @ b_of_e(e)
-    return out
+# Every quantization block of the composite lies inside one expert segment:
+# ROW blocks are within a row, COL blocks are 32-row groups and segments start
+# at multiples of the pad (itself a multiple of 128).  The composite is
+# therefore written per expert segment and the full-tensor forms below just
+# loop over the experts.
+def expert_fwd(x_e, w13_e, w2_e, exact=False):
+    """Forward for the rows x_e [n, D] routed to one expert.
 
-
-def _seg_wgrad(g, x, offsets, experts, E):
-    """dW[e] = g[seg_e]^T @ x[seg_e]; zero for an expert without rows."""
-    out = np.full((E, g.shape[1], x.shape[1]), np.nan)
-    for e in _experts(offsets, experts):
-        lo, hi = int(offsets[e]), int(offsets[e + 1])
-        out[e] = g[lo:hi].T @ x[lo:hi] if hi > lo else 0.0
-    return out
-
-
-def moe_mlp_fwd(x, w13, w2, offsets, experts=None, exact=False):
-    """Forward of the MXFP8 routed-experts MLP.
-
-    x [M, D] bf16 values, w13 [E, 2F, D] (rows 0..F-1 gate, F..2F-1 up),
-    w2 [E, D, F], given as float64 arrays.  Every GEMM operand is the
-    dequantized MX tensor: x and h ROW-quantized along the contraction
-    dimension, w13 and w2 ROW-quantized per expert along theirs.  h13 is
-    rounded to bf16, h = bf16(silu(gate) * up).  y is returned unrounded.
-
-    exact=True drops every quantization and bf16 rounding (a plain float64
-    MLP with the same structure); the tests use it to pin the composition.
+    h13 = x_e . w13_e^T with x ROW-quantized along D and w13_e [2F, D]
+    ROW-quantized along D; h13 rounded to bf16; h = bf16(silu(gate) * up);
+    y = h . w2_e^T with h ROW-quantized along F and w2_e [D, F] along F
+    (y is returned unrounded).  exact=True drops every quantization and bf16
+    rounding (a plain float64 MLP with the same structure).
     """
-    x = np.asarray(x, dtype=np.float64)
-    E = w13.shape[0]
-    F = w13.shape[1] // 2
-    D = x.shape[1]
+    x_e = np.asarray(x_e, dtype=np.float64)
+    F = w13_e.shape[0] // 2
     out = {}
     if exact:
-        xq, w13q, w2q = x, w13, w2
+        xq, w13q, w2q = x_e, w13_e, w2_e
     else:
-        x_rc, x_rs = quantize_rows(x)
-        out["x_row"] = (x_rc, x_rs)
-        out["x_col"] = quantize_cols(x)
-        xq = dequantize_rows(x_rc, x_rs)
-        w13q = np.stack([dequantize_rows(*quantize_rows(w13[e])) for e in range(E)])
-        w2q = np.stack([dequantize_rows(*quantize_rows(w2[e])) for e in range(E)])
-    h13 = _seg_matmul(xq, lambda e: w13q[e].T, offsets, experts, 2 * F)
-    h13 = np.nan_to_num(h13, nan=0.0)        # rows of experts not listed: inert
+        out["x_row"] = quantize_rows(x_e)
+        out["x_col"] = quantize_cols(x_e)
+        xq = dequantize_rows(*out["x_row"])
+        w13q = dequantize_rows(*quantize_rows(w13_e))
+        w2q = dequantize_rows(*quantize_rows(w2_e))
+    h13 = xq @ w13q.T
     if exact:
         a, b = h13[:, :F], h13[:, F:]
         h = a * _sigmoid(a) * b
@@ -382,49 +361,40 @@ def moe_mlp_fwd(x, w13, w2, offsets, experts=None, exact=False):
     else:
         h13 = round_to_bf16(h13)
         h = swiglu(h13)
-        h_rc, h_rs = quantize_rows(h)
-        out["h_row"] = (h_rc, h_rs)
+        out["h_row"] = quantize_rows(h)
         out["h_col"] = quantize_cols(h)
-        hq = dequantize_rows(h_rc, h_rs)
-    y = _seg_matmul(hq, lambda e: w2q[e].T, offsets, experts, D)
-    out.update(y=y, h13=h13, h=h)
+        hq = dequantize_rows(*out["h_row"])
+    out.update(y=hq @ w2q.T, h13=h13, h=h)
     return out
 
 
-def moe_mlp_bwd(dy, fwd, x, w13, w2, offsets, experts=None, exact=False):
-    """Backward of :func:`moe_mlp_fwd`: dx [M, D], dW13 [E, 2F, D], dW2 [E, D, F].
+def expert_bwd(dy_e, fwd_e, x_e, w13_e, w2_e, exact=False):
+    """Backward for one expert segment.
 
-    dh = dY . W2[e] with dY ROW-quantized and W2 COL-quantized along D;
-    dh is rounded to bf16 and turned into dh13 = [dgate | dup] (bf16) by
-    dSwiGLU.  dW2[e] = dY_e^T . h_e and dW13[e] = dh13_e^T . x_e over the
-    expert's rows with both operands COL-quantized along the token dimension;
-    dx = dh13 . W13[e] with dh13 ROW-quantized and W13 COL-quantized along 2F.
+    dh = dY . W2 with dY ROW-quantized along D and W2 [D, F] COL-quantized
+    along D; dh rounded to bf16; dh13 = [dgate | dup] = dSwiGLU(dh, h13) in
+    bf16; dW2 = dY^T . h and dW13 = dh13^T . x with both operands
+    COL-quantized along the token rows; dx = dh13 . W13 with dh13
+    ROW-quantized and W13 [2F, D] COL-quantized along 2F.
     """
-    dy = np.asarray(dy, dtype=np.float64)
-    x = np.asarray(x, dtype=np.float64)
-    E = w13.shape[0]
-    F = w13.shape[1] // 2
-    D = dy.shape[1]
-    h13 = fwd["h13"]
+    dy_e = np.asarray(dy_e, dtype=np.float64)
+    F = w13_e.shape[0] // 2
+    h13 = fwd_e["h13"]
     out = {}
     if exact:
-        dyr = dyc = dy
-        w2c = w2
-        w13c = w13
-        hc, xc = fwd["h"], x
+        dyr = dyc = dy_e
+        w2c, w13c = w2_e, w13_e
+        hc, xc = fwd_e["h"], np.asarray(x_e, dtype=np.float64)
     else:
-        dy_rc, dy_rs = quantize_rows(dy)
-        dy_cc, dy_cs = quantize_cols(dy)
-        dyr = dequantize_rows(dy_rc, dy_rs)
-        dyc = dequantize_rows(dy_cc, dy_cs).T
-        # W2[e] is [D, F]: COL blocks run along D (the contraction of dh)
-        w2c = np.stack([dequantize_rows(*quantize_cols(w2[e])).T for e in range(E)])
-        # W13[e] is [2F, D]: COL blocks run along 2F (the contraction of dx)
-        w13c = np.stack([dequantize_rows(*quantize_cols(w13[e])).T for e in range(E)])
-        hc = dequantize_rows(*fwd["h_col"]).T
-        xc = dequantize_rows(*fwd["x_col"]).T
-    dh = _seg_matmul(dyr, lambda e: w2c[e], offsets, experts, F)
-    dh = np.nan_to_num(dh, nan=0.0)
+        out["dy_row"] = quantize_rows(dy_e)
+        out["dy_col"] = quantize_cols(dy_e)
+        dyr = dequantize_rows(*out["dy_row"])
+        dyc = dequantize_rows(*out["dy_col"]).T
+        w2c = dequantize_rows(*quantize_cols(w2_e)).T       # [D, F], blocks along D
+        w13c = dequantize_rows(*quantize_cols(w13_e)).T     # [2F, D], blocks along 2F
+        hc = dequantize_rows(*fwd_e["h_col"]).T
+        xc = dequantize_rows(*fwd_e["x_col"]).T
+    dh = dyr @ w2c
     if exact:
         a, b = h13[:, :F], h13[:, F:]
         s = _sigmoid(a)
@@ -433,16 +403,62 @@ def moe_mlp_bwd(dy, fwd, x, w13, w2, offsets, experts=None, exact=False):
     else:
         dh = round_to_bf16(dh)
         dh13 = dswiglu(dh, h13)
-        g_rc, g_rs = quantize_rows(dh13)
-        g_cc, g_cs = quantize_cols(dh13)
-        out["dh13_row"] = (g_rc, g_rs)
-        out["dh13_col"] = (g_cc, g_cs)
-        out["dy_row"] = (dy_rc, dy_rs)
-        out["dy_col"] = (dy_cc, dy_cs)
-        gr = dequantize_rows(g_rc, g_rs)
-        gc = dequantize_rows(g_cc, g_cs).T
-    dw2 = _seg_wgrad(dyc, hc, offsets, experts, E)
-    dx = _seg_matmul(gr, lambda e: w13c[e], offsets, experts, D)
-    dw13 = _seg_wgrad(gc, xc, offsets, experts, E)
-    out.update(dx=dx, dw13=dw13, dw2=dw2, dh=dh, dh13=dh13)
+        out["dh13_row"] = quantize_rows(dh13)
+        out["dh13_col"] = quantize_cols(dh13)
+        gr = dequantize_rows(*out["dh13_row"])
+        gc = dequantize_rows(*out["dh13_col"]).T
+    out.update(dw2=dyc.T @ hc, dx=gr @ w13c, dw13=gc.T @ xc, dh=dh, dh13=dh13)
     return out
+
+
+def _segments(offsets, experts):
+    E = len(offsets) - 1
+    for e in (range(E) if experts is None else experts):
+        yield e, int(offsets[e]), int(offsets[e + 1])
+
+
+def moe_mlp_fwd(x, w13, w2, offsets, experts=None, exact=False):
+    """Forward of the routed-experts MLP over the expert-major padded layout.
+
+    x [M, D], w13 [E, 2F, D] (rows 0..F-1 gate = w1, F..2F-1 up = w3),
+    w2 [E, D, F], as float64 arrays of bf16 values.  Returns full-size arrays
+    y, h13, h (rows outside the listed experts' segments are NaN) and
+    'experts': {e: per-expert dict of expert_fwd}.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    M, D = x.shape
+    F = w13.shape[1] // 2
+    y = np.full((M, D), np.nan)
+    h13 = np.full((M, 2 * F), np.nan)
+    h = np.full((M, F), np.nan)
+    per = {}
+    for e, lo, hi in _segments(offsets, experts):
+        if hi == lo:
+            continue
+        r = expert_fwd(x[lo:hi], w13[e], w2[e], exact)
+        y[lo:hi], h13[lo:hi], h[lo:hi] = r["y"], r["h13"], r["h"]
+        per[e] = r
+    return dict(y=y, h13=h13, h=h, experts=per)
+
+
+def moe_mlp_bwd(dy, fwd, x, w13, w2, offsets, experts=None, exact=False):
+    """Backward: dx [M, D] (NaN outside the listed segments), dW13 [E, 2F, D],
+    dW2 [E, D, F] (NaN for experts not listed, exact zeros for listed experts
+    without rows), plus 'experts': {e: per-expert dict of expert_bwd}."""
+    dy = np.asarray(dy, dtype=np.float64)
+    x = np.asarray(x, dtype=np.float64)
+    M, D = dy.shape
+    E, F2, _ = w13.shape
+    dx = np.full((M, D), np.nan)
+    dw13 = np.full((E, F2, D), np.nan)
+    dw2 = np.full((E, D, F2 // 2), np.nan)
+    per = {}
+    for e, lo, hi in _segments(offsets, experts):
+        if hi == lo:
+            dw13[e] = 0.0
+            dw2[e] = 0.0
+            continue
+        r = expert_bwd(dy[lo:hi], fwd["experts"][e], x[lo:hi], w13[e], w2[e], exact)
+        dx[lo:hi], dw13[e], dw2[e] = r["dx"], r["dw13"], r["dw2"]
+        per[e] = r
+    return dict(dx=dx, dw13=dw13, dw2=dw2, experts=per)

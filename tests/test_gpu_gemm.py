@@ -1,0 +1,213 @@
+"""GPU parity of the tcgen05 grouped GEMMs against the oracle.
+
+Operands are quantized by the oracle from the same bf16 tensors the GPU
+quantizes itself (the casts are bit-exact, checked in test_gpu_quant), so
+both sides multiply identical MXFP8 operands.
+"""
+import numpy as np
+import pytest
+import torch
+
+import mxfp8_block_scaled_routed_b200 as mxk
+import synth
+from oracle import mx
+from mxtest import (assert_codes_close, assert_gemm_close, bf16_np, mma_to_plain, plain_to_mma, u8)
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).to(DEV)
+
+
+def _offsets(counts, pad):
+    padded = [((c + pad - 1) // pad) * pad for c in counts]
+    return np.concatenate([[0], np.cumsum(padded)]).astype(np.int32)
+
+
+def _bf16(a):
+    return synth.to_bf16(np.asarray(a, dtype=np.float32))
+
+
+def _mx_rows_dev(x_bf16: torch.Tensor):
+    """GPU ROW quantization with MMA scales (the GEMM operand form)."""
+    o = mxk.mxfp8_quantize(x_bf16.to(DEV), mxk.ROW, mxk.MMA)
+    return o["row_codes"].reshape(-1, x_bf16.shape[-1]), o["row_scales"]
+
+
+def _exact_pow2_ternary(g, shape, spread=3):
+    """t * 2^e with t in {-1,0,1} and e constant per 32-block: quantization is exact."""
+    t = g.choice(np.array([-1.0, 0.0, 1.0]), size=shape)
+    t[..., ::32] = 1.0                                   # every block has a nonzero
+    e = g.integers(-spread, spread + 1, size=shape[:-1] + (shape[-1] // 32,))
+    return t * np.repeat(np.ldexp(1.0, e), 32, axis=-1)
+
+
+# ------------------------------------------------------------------ ragged M
+@pytest.mark.parametrize("N", [256, 384])
+def test_grouped_gemm_exact_closed_form(N):
+    """Exactly representable operands: fp32 accumulation is exact, so the bf16
+    output must equal round_to_bf16 of the exact product bit for bit."""
+    g = np.random.default_rng(1)
+    E, K = 3, 512
+    off = _offsets([200, 0, 300], 128)
+    M = int(off[-1]) + 128
+    a = _exact_pow2_ternary(g, (M, K))
+    w = _exact_pow2_ternary(g, (E, N, K))
+    ac, as_ = _mx_rows_dev(_bf16(a))
+    wc, ws = _mx_rows_dev(_bf16(w.reshape(E * N, K)))
+    out = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device=DEV)
+    mxk.mxfp8_grouped_gemm(ac, as_, wc.reshape(E, N, K), ws, _dev(off), 128, out=out)
+    got = bf16_np(out)
+    for e in range(E):
+        lo, hi = off[e], off[e + 1]
+        np.testing.assert_array_equal(got[lo:hi], mx.round_to_bf16(a[lo:hi] @ w[e].T))
+    assert np.isnan(got[off[-1]:]).all()          # rows past offsets[E] untouched
+    assert mxk.device_error() == 0
+
+
+@pytest.mark.parametrize("pad,N,K", [(128, 512, 256), (256, 384, 640), (128, 256, 1408)])
+def test_grouped_gemm_random_vs_oracle(pad, N, K):
+    g = synth.rng(2)
+    E = 4
+    off = _offsets([130, 0, 77, 300], pad)
+    M = int(off[-1])
+    a = _bf16(synth.normal(g, (M, K)))
+    w = _bf16(synth.normal(g, (E, N, K), 0.02))
+    ac, as_ = _mx_rows_dev(a)
+    wc, ws = _mx_rows_dev(w.reshape(E * N, K))
+    out = mxk.mxfp8_grouped_gemm(ac, as_, wc.reshape(E, N, K), ws, _dev(off), pad)
+    arc, ars = mx.quantize_rows(bf16_np(a))
+    wrc, wrs = mx.quantize_weights_rows(bf16_np(w))
+    ref = mx.grouped_gemm(arc, ars, wrc, wrs, off)
+    assert_gemm_close(bf16_np(out), ref, "grouped_gemm")
+
+
+def test_grouped_gemm_nan_tail_not_read():
+    g = synth.rng(3)
+    E, N, K = 2, 256, 256
+    off = _offsets([100, 60], 128)
+    M = int(off[-1]) + 256
+    a = synth.normal(g, (M, K))
+    a[off[-1]:] = np.nan                                  # poisoned tail
+    at = _bf16(a)
+    w = _bf16(synth.normal(g, (E, N, K), 0.02))
+    ac, as_ = _mx_rows_dev(at)
+    wc, ws = _mx_rows_dev(w.reshape(E * N, K))
+    out = torch.full((M, N), 7.0, dtype=torch.bfloat16, device=DEV)
+    mxk.mxfp8_grouped_gemm(ac, as_, wc.reshape(E, N, K), ws, _dev(off), 128, out=out)
+    got = bf16_np(out)
+    assert np.isfinite(got[: off[-1]]).all()
+    assert (got[off[-1]:] == 7.0).all()
+
+
+def test_bad_offsets_raise_device_error_and_write_nothing():
+    E, N, K, M = 2, 256, 256, 256
+    a = torch.zeros(M, K, dtype=torch.uint8, device=DEV)
+    sa = torch.zeros(M * K // 32, dtype=torch.uint8, device=DEV)
+    w = torch.zeros(E, N, K, dtype=torch.uint8, device=DEV)
+    sw = torch.zeros(E * N * K // 32, dtype=torch.uint8, device=DEV)
+    out = torch.full((M, N), 3.0, dtype=torch.bfloat16, device=DEV)
+    assert mxk.device_error() == 0
+    for bad in ([0, 256, 128], [0, 64, 256], [0, 128, 512], [128, 128, 256]):
+        mxk.mxfp8_grouped_gemm(a, sa, w, sw, _dev(np.array(bad, np.int32)), 128, out=out)
+        assert mxk.device_error(reset=True) == 4, bad
+    assert (bf16_np(out) == 3.0).all()
+
+
+# ------------------------------------------------------------------ ragged K
+def _mx_cols_dev(x_bf16: torch.Tensor):
+    o = mxk.mxfp8_quantize(x_bf16.to(DEV), mxk.COL, mxk.MMA)
+    return o["col_codes"], o["col_scales"]
+
+
+def test_wgrad_exact_closed_form_and_empty_expert():
+    g = np.random.default_rng(4)
+    E, N, Kx = 3, 256, 384
+    off = _offsets([256, 0, 300], 128)
+    M = int(off[-1])
+    # COL quantization of G and X is exact when each 32-row block of a column
+    # is t * 2^e: build the transposes with the helper and transpose back.
+    Gt = _exact_pow2_ternary(g, (N, M))
+    Xt = _exact_pow2_ternary(g, (Kx, M))
+    gc, gs = _mx_cols_dev(_bf16(Gt.T))
+    xc, xs = _mx_cols_dev(_bf16(Xt.T))
+    out = torch.full((E, N, Kx), float("nan"), dtype=torch.bfloat16, device=DEV)
+    mxk.mxfp8_grouped_gemm_wgrad(gc, gs, xc, xs, _dev(off), 128, out=out)
+    got = bf16_np(out)
+    for e in range(E):
+        lo, hi = off[e], off[e + 1]
+        np.testing.assert_array_equal(got[e], mx.round_to_bf16(Gt[:, lo:hi] @ Xt[:, lo:hi].T))
+    assert (got[1] == 0).all() and not np.signbit(got[1]).any()
+
+
+@pytest.mark.parametrize("pad,N,Kx", [(128, 256, 256), (256, 384, 512)])
+def test_wgrad_random_vs_oracle(pad, N, Kx):
+    g = synth.rng(5)
+    E = 4
+    off = _offsets([300, 0, 129, 60], pad)
+    M = int(off[-1])
+    G = _bf16(synth.normal(g, (M, N), 1e-2))
+    X = _bf16(synth.normal(g, (M, Kx)))
+    gc, gs = _mx_cols_dev(G)
+    xc, xs = _mx_cols_dev(X)
+    out = mxk.mxfp8_grouped_gemm_wgrad(gc, gs, xc, xs, _dev(off), pad)
+    gcc, gcs = mx.quantize_cols(bf16_np(G))
+    xcc, xcs = mx.quantize_cols(bf16_np(X))
+    ref = mx.grouped_gemm_wgrad(gcc, gcs, xcc, xcs, off)
+    assert_gemm_close(bf16_np(out), ref, "wgrad")
+    assert (bf16_np(out)[1] == 0).all()
+
+
+# ------------------------------------------------------------------ fused epilogues
+def test_fc1_swiglu_dual_quant_vs_oracle_and_standalone():
+    g = synth.rng(6)
+    E, D, F = 3, 256, 384
+    off = _offsets([200, 0, 140], 128)
+    M = int(off[-1])
+    x = _bf16(synth.normal(g, (M, D)))
+    w13 = _bf16(synth.normal(g, (E, 2 * F, D), 0.05))
+    xc, xs = _mx_rows_dev(x)
+    wc, ws = _mx_rows_dev(w13.reshape(E * 2 * F, D))
+    o = mxk.mxfp8_grouped_gemm_swiglu_quant(xc, xs, wc.reshape(E, 2 * F, D), ws, _dev(off), 128)
+    # oracle: h13 per expert, then SwiGLU + dual quantization
+    xr = mx.quantize_rows(bf16_np(x))
+    wr = mx.quantize_weights_rows(bf16_np(w13))
+    h13_ref = mx.round_to_bf16(mx.grouped_gemm(*xr, *wr, off))
+    h13_got = bf16_np(o["h13"])
+    assert_gemm_close(h13_got, h13_ref, "h13")
+    rc, rs, cc, cs = mx.swiglu_quant(h13_ref)
+    got_rs = mma_to_plain(u8(o["h_row_scales"]), M, F)
+    got_cs = mma_to_plain(u8(o["h_col_scales"]), F, M)
+    assert_codes_close(u8(o["h_row_codes"]), rc, got_rs, rs, "FC1 h ROW")
+    assert_codes_close(u8(o["h_col_codes"]), cc, got_cs, cs, "FC1 h COL")
+    # the fused epilogue equals the standalone SwiGLU cast of its own h13, bit for bit
+    s = mxk.mxfp8_swiglu_quant(o["h13"], mxk.ROW | mxk.COL, mxk.MMA)
+    for k in ("row_codes", "row_scales", "col_codes", "col_scales"):
+        assert torch.equal(s[k].reshape(-1), o["h_" + k].reshape(-1)), k
+
+
+def test_fc2_dgrad_dswiglu_dual_quant_vs_oracle():
+    g = synth.rng(7)
+    E, D, F = 3, 384, 256
+    off = _offsets([150, 0, 250], 128)
+    M = int(off[-1])
+    dy = _bf16(synth.normal(g, (M, D), 1e-2))
+    w2 = _bf16(synth.normal(g, (E, D, F), 0.05))
+    h13 = _bf16(synth.normal(g, (M, 2 * F), 2.0))
+    dr, ds = _mx_rows_dev(dy)
+    w2t = mxk.mxfp8_quantize(w2.to(DEV), mxk.COL, mxk.MMA)        # [E, F, D]
+    o = mxk.mxfp8_grouped_gemm_dswiglu_quant(dr, ds, w2t["col_codes"], w2t["col_scales"], _dev(off),
+                                             h13.to(DEV), 128)
+    dyr = mx.quantize_rows(bf16_np(dy))
+    w2c = mx.quantize_weights_cols(bf16_np(w2))
+    dh = mx.round_to_bf16(np.nan_to_num(mx.grouped_gemm(*dyr, *w2c, off)))
+    dh13 = mx.dswiglu(dh, bf16_np(h13))
+    dh13[off[-1]:] = 0
+    rc, rs = mx.quantize_rows(dh13)
+    cc, cs = mx.quantize_cols(dh13)
+    got_rs = mma_to_plain(u8(o["g_row_scales"]), M, 2 * F)
+    got_cs = mma_to_plain(u8(o["g_col_scales"]), 2 * F, M)
+    assert_codes_close(u8(o["g_row_codes"]), rc, got_rs, rs, "dh13 ROW")
+    assert_codes_close(u8(o["g_col_codes"]), cc, got_cs, cs, "dh13 COL")
