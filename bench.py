@@ -1,0 +1,514 @@
+#!/usr/bin/env python
+"""Benchmark of the MXFP8 routed-experts MLP on B200.
+
+One step = one pass of the whole hot path over one batch of synthetic routed
+tokens: the DSv3-scale expert layer (E=256, D=7168, F=2048, 16384 tokens
+top-8, Zipf(1.0) routing padded to 256) forward and backward -- token and
+weight casts, FC1 + SwiGLU + dual quant, FC2, dY casts, FC2 dgrad + dSwiGLU +
+dual quant, dW2, dx, dW13 -- plus the standalone SwiGLU + dual quant of
+h13 [16384, 2x4096] and the bf16 -> MXFP8 cast of the [8192, 7168] transport
+payload.
+
+Prints one JSON line.  `value` is the useful (real routed rows) fwd+bwd
+TFLOP/s of the expert MLP with inputs resident in HBM; every input is larger
+than L2, so no flush is needed between steps.  `e2e` is the same metric
+through the public composite API with the step's token inputs copied from
+pinned host memory and a slice of the result read back inside the timed
+region.  `--impl reference` times the CPU oracle on a bounded sample.
+
+Launch: python bench.py [--gpus N --steps K --warmup W]; for N > 1 under
+torch.distributed.run (one rank per GPU; each rank runs its own batch, no
+collective on the data path: weak scaling).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+SWIGLU_ROWS, SWIGLU_F = 16384, 4096
+CAST_ROWS, CAST_COLS = 8192, 7168
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def src_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "mxfp8_block_scaled_routed_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:12]
+
+
+def ncu_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch recorded by an ncu capture in profiles/, if the
+    capture was taken from the current kernel sources."""
+    p = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
+    if not os.path.exists(p):
+        return None
+    txt = open(p).read()
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", txt)
+    h = re.search(r"source_hash:\s*([0-9a-f]+)", txt)
+    if not m or not h or h.group(1) != src_hash():
+        return None
+    return float(m.group(1))
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples every 200 ms; only samples taken inside [t0, t1]
+    (host wall clock around the timed region) are kept."""
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(1.0)              # let nvidia-smi start sampling before the timed region
+
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.3)
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        import datetime
+        sm, mx_, pw, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 10:
+                continue
+            try:
+                ts = datetime.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                if self.t0 is not None and not (self.t0 - 0.25 <= ts <= self.t1 + 0.25):
+                    continue
+                sm.append(float(f[2]))
+                mx_.append(float(f[3]))
+                pw.append(float(f[4]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[6:10]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(mx_) if mx_ else None,
+                "reasons": sorted(reasons), "samples": len(sm),
+                "power_w_median": float(np.median(pw)) if pw else None}
+
+
+# ----------------------------------------------------------------------------- the step
+class Step:
+    """All buffers of one fwd+bwd step, laid out once; run() issues the kernels.
+
+    The sequence is exactly the one moe_mlp_fwd / moe_mlp_bwd issue, written
+    out call by call so each kernel can be bracketed with CUDA events.
+    """
+
+    def __init__(self, inp, dev):
+        import mxfp8_block_scaled_routed_b200 as mxk
+        self.mxk, self.L = mxk, mxk.lib()
+        s = inp.spec
+        self.E, self.D, self.F = s.E, s.D, s.F
+        self.M = M = inp.routing.M
+        self.R = inp.routing.R
+        self.pad = s.pad
+        E, D, F = self.E, self.D, self.F
+        u8 = lambda *sh: torch.empty(*sh, dtype=torch.uint8, device=dev)
+        bf = lambda *sh: torch.empty(*sh, dtype=torch.bfloat16, device=dev)
+        self.x, self.w13, self.w2, self.dy = inp.x, inp.w13, inp.w2, inp.dy
+        self.off = torch.from_numpy(inp.routing.offsets).to(dev)
+        self.x_rc, self.x_rs, self.x_cc, self.x_cs = u8(M, D), u8(M * D // 32), u8(D, M), u8(M * D // 32)
+        self.w13_c, self.w13_s = u8(E * 2 * F, D), u8(E * 2 * F * D // 32)
+        self.w2_c, self.w2_s = u8(E * D, F), u8(E * D * F // 32)
+        self.h13 = bf(M, 2 * F)
+        self.h_rc, self.h_rs, self.h_cc, self.h_cs = u8(M, F), u8(M * F // 32), u8(F, M), u8(M * F // 32)
+        self.y = bf(M, D)
+        self.dy_rc, self.dy_rs, self.dy_cc, self.dy_cs = u8(M, D), u8(M * D // 32), u8(D, M), u8(M * D // 32)
+        self.w2t_c, self.w2t_s = u8(E, F, D), u8(E * F * D // 32)
+        self.w13t_c, self.w13t_s = u8(E, D, 2 * F), u8(E * D * 2 * F // 32)
+        self.g_rc, self.g_rs, self.g_cc, self.g_cs = u8(M, 2 * F), u8(M * 2 * F // 32), u8(2 * F, M), u8(M * 2 * F // 32)
+        self.dx, self.dw13, self.dw2 = bf(M, D), bf(E, 2 * F, D), bf(E, D, F)
+        # standalone boundary kernels
+        self.sw_in = inp.swiglu_h13
+        self.sw_rc, self.sw_rs = u8(SWIGLU_ROWS, SWIGLU_F), u8(SWIGLU_ROWS * SWIGLU_F // 32)
+        self.sw_cc, self.sw_cs = u8(SWIGLU_F, SWIGLU_ROWS), u8(SWIGLU_ROWS * SWIGLU_F // 32)
+        self.c_in = inp.cast_x
+        self.c_rc, self.c_rs = u8(CAST_ROWS, CAST_COLS), u8(CAST_ROWS, CAST_COLS // 32)
+        self.stream = torch.cuda.current_stream(dev)
+        self._build()
+
+    def _build(self):
+        L, p = self.L, (lambda t: torch.Tensor.data_ptr(t))
+        st = self.stream.cuda_stream
+        M, D, E, F, pad = self.M, self.D, self.E, self.F, self.pad
+        off = p(self.off)
+        self.ops = [
+            ("cast_x_dual", "hbm", 4.0625 * M * D,
+             lambda: L.mxfp8_quantize(p(self.x), 1, M, D, 3, 1, p(self.x_rc), p(self.x_rs), p(self.x_cc), p(self.x_cs), st)),
+            ("cast_w13_row", "hbm", 3.03125 * E * 2 * F * D,
+             lambda: L.mxfp8_quantize(p(self.w13), 1, E * 2 * F, D, 1, 1, p(self.w13_c), p(self.w13_s), None, None, st)),
+            ("cast_w2_row", "hbm", 3.03125 * E * D * F,
+             lambda: L.mxfp8_quantize(p(self.w2), 1, E * D, F, 1, 1, p(self.w2_c), p(self.w2_s), None, None, st)),
+            ("fc1_swiglu_quant", "tensor", 2.0 * M * 2 * F * D,
+             lambda: L.mxfp8_grouped_gemm_swiglu_quant(p(self.x_rc), p(self.x_rs), M, D, p(self.w13_c), p(self.w13_s), E, F,
+                                                       off, pad, p(self.h13), p(self.h_rc), p(self.h_rs), p(self.h_cc),
+                                                       p(self.h_cs), st)),
+            ("fc2", "tensor", 2.0 * M * D * F,
+             lambda: L.mxfp8_grouped_gemm(p(self.h_rc), p(self.h_rs), M, F, p(self.w2_c), p(self.w2_s), E, D, off, pad,
+                                          p(self.y), st)),
+            ("cast_dy_dual", "hbm", 4.0625 * M * D,
+             lambda: L.mxfp8_quantize(p(self.dy), 1, M, D, 3, 1, p(self.dy_rc), p(self.dy_rs), p(self.dy_cc), p(self.dy_cs), st)),
+            ("cast_w2_col", "hbm", 3.03125 * E * D * F,
+             lambda: L.mxfp8_quantize(p(self.w2), E, D, F, 2, 1, None, None, p(self.w2t_c), p(self.w2t_s), st)),
+            ("cast_w13_col", "hbm", 3.03125 * E * 2 * F * D,
+             lambda: L.mxfp8_quantize(p(self.w13), E, 2 * F, D, 2, 1, None, None, p(self.w13t_c), p(self.w13t_s), st)),
+            ("fc2_dgrad_dswiglu_quant", "tensor", 2.0 * M * F * D,
+             lambda: L.mxfp8_grouped_gemm_dswiglu_quant(p(self.dy_rc), p(self.dy_rs), M, D, p(self.w2t_c), p(self.w2t_s), E, F,
+                                                        off, pad, p(self.h13), p(self.g_rc), p(self.g_rs), p(self.g_cc),
+                                                        p(self.g_cs), st)),
+            ("wgrad_dw2", "tensor", 2.0 * M * D * F,
+             lambda: L.mxfp8_grouped_gemm_wgrad(p(self.dy_cc), p(self.dy_cs), D, p(self.h_cc), p(self.h_cs), F, M, off, E, pad,
+                                                p(self.dw2), st)),
+            ("dgrad_dx", "tensor", 2.0 * M * 2 * F * D,
+             lambda: L.mxfp8_grouped_gemm(p(self.g_rc), p(self.g_rs), M, 2 * F, p(self.w13t_c), p(self.w13t_s), E, D, off,
+                                          pad, p(self.dx), st)),
+            ("wgrad_dw13", "tensor", 2.0 * M * 2 * F * D,
+             lambda: L.mxfp8_grouped_gemm_wgrad(p(self.g_cc), p(self.g_cs), 2 * F, p(self.x_cc), p(self.x_cs), D, M, off, E,
+                                                pad, p(self.dw13), st)),
+            ("swiglu_quant_16384x4096", "hbm", 6.0625 * SWIGLU_ROWS * SWIGLU_F,
+             lambda: L.mxfp8_swiglu_quant(p(self.sw_in), SWIGLU_ROWS, SWIGLU_F, 3, 1, p(self.sw_rc), p(self.sw_rs),
+                                          p(self.sw_cc), p(self.sw_cs), st)),
+            ("cast_payload_8192x7168", "hbm", 3.03125 * CAST_ROWS * CAST_COLS,
+             lambda: L.mxfp8_quantize(p(self.c_in), 1, CAST_ROWS, CAST_COLS, 1, 0, p(self.c_rc), p(self.c_rs), None, None, st)),
+        ]
+        self.mlp_ops = 12
+
+    def run(self, events=None):
+        for i, (name, _, _, fn) in enumerate(self.ops):
+            s = fn()
+            if s != 0:
+                raise RuntimeError(f"{name}: {self.L.mxmoe_last_error().decode()}")
+            if events is not None:
+                events[i + 1].record(self.stream)
+
+    def flops(self, rows):
+        return 18.0 * rows * self.D * self.F
+
+
+# ----------------------------------------------------------------------------- inputs
+def make_inputs(workload: str, seed: int, dev):
+    import synth
+    inp = synth.device_moe_inputs(workload, seed, device=dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(seed + 7)
+    h = torch.randn(SWIGLU_ROWS, 2 * SWIGLU_F, generator=gen, device=dev)
+    n = h.numel()
+    idx = torch.randperm(n, generator=gen, device=dev)[: n // 100]
+    h.view(-1)[idx] *= 100.0
+    inp.swiglu_h13 = h.to(torch.bfloat16)
+    del h, idx
+    inp.cast_x = torch.randn(CAST_ROWS, CAST_COLS, generator=gen, device=dev).to(torch.bfloat16)
+    return inp
+
+
+# ----------------------------------------------------------------------------- CPU baseline (oracle)
+def oracle_sample(inp, budget_s=12.0, max_experts=None):
+    """Time the CPU oracle (fwd+bwd) on whole experts of the workload, the
+    smallest non-empty ones first, until about budget_s of work is done."""
+    from oracle import mx
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [os.cpu_count()])
+    except Exception:
+        cores = os.cpu_count()
+    counts = inp.routing.counts
+    off = inp.routing.offsets
+    order = [int(e) for e in np.argsort(counts) if counts[e] > 0]
+    order = order[len(order) // 2:] + order[: len(order) // 2]          # start from the median expert
+    f = lambda t: t.float().double().cpu().numpy()
+    flops, t_total, rows_done, experts = 0.0, 0.0, 0, []
+    for e in order:
+        lo, hi = int(off[e]), int(off[e + 1])
+        x, dy = f(inp.x[lo:hi]), f(inp.dy[lo:hi])
+        w13, w2 = f(inp.w13[e]), f(inp.w2[e])
+        t0 = time.perf_counter()
+        r = mx.expert_fwd(x, w13, w2)
+        mx.expert_bwd(dy, r, x, w13, w2)
+        t_total += time.perf_counter() - t0
+        flops += 18.0 * int(counts[e]) * inp.spec.D * inp.spec.F
+        rows_done += int(counts[e])
+        experts.append(e)
+        if t_total >= budget_s or (max_experts and len(experts) >= max_experts):
+            break
+    return dict(value=flops / t_total / 1e12, unit="TFLOP/s", cores=int(cores), kind="oracle",
+                sample=f"fwd+bwd of {len(experts)} whole expert(s) ({rows_done} real rows) of the "
+                       f"{inp.spec.name} layer, float64 numpy, {t_total:.1f} s"), t_total
+
+
+# ----------------------------------------------------------------------------- main
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        torch.distributed.init_process_group("nccl" if torch.cuda.is_available() else "gloo",
+                                             timeout=datetime.timedelta(seconds=600))
+    return world, rank, local
+
+
+def config_dict(spec, inp, extra=None):
+    d = {"workload": f"{spec.name}: E={spec.E} D={spec.D} F={spec.F} tokens={spec.tokens} top{spec.top_k} "
+                     f"Zipf({spec.zipf_s}) pad {spec.pad}, fwd+bwd; + SwiGLU quant 16384x2x4096 + cast 8192x7168",
+         "tokens": spec.tokens, "top_k": spec.top_k, "padded_rows": int(inp.routing.M), "real_rows": int(inp.routing.R),
+         "l2": "inputs larger than L2 (x, dy, weights >> 126 MB); no flush needed"}
+    if extra:
+        d.update(extra)
+    return d
+
+
+def run_reference(args, world, rank):
+    import synth
+    if rank != 0:
+        return 0
+    spec = synth.SPECS[args.workload]
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = synth.device_moe_inputs(spec, args.seed, device=dev)
+    for _ in range(args.warmup):
+        oracle_sample(inp, budget_s=2.0, max_experts=1)
+    times, vals = [], []
+    cpu = None
+    for _ in range(args.steps):
+        cpu, t = oracle_sample(inp, budget_s=4.0)
+        times.append(t)
+        vals.append(cpu["value"])
+    v = float(np.mean(vals))
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * float(np.mean(times)),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config_dict(spec, inp),
+            "cpu_baseline": dict(cpu, value=v),
+            "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+METRIC = "MoE expert-MLP MXFP8 fwd+bwd TFLOP/s (useful rows); SwiGLU+quant GB/s vs HBM peak"
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="dsv3", choices=["dsv3", "dsv3_16b", "tiny"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    world, rank, local = dist_setup(args)
+    if args.impl == "reference":
+        return run_reference(args, world, rank)
+
+    assert torch.cuda.is_available(), "bench.py needs a GPU"
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    import mxfp8_block_scaled_routed_b200 as mxk
+    import synth
+    spec = synth.SPECS[args.workload]
+    inp = make_inputs(args.workload, args.seed + rank, dev)
+    step = Step(inp, dev)
+    n_ops = len(step.ops)
+
+    # warm-up (at least 3 steps)
+    args.warmup = max(args.warmup, 3)
+    for _ in range(args.warmup):
+        step.run()
+    torch.cuda.synchronize()
+    if mxk.device_error() != 0:
+        raise RuntimeError("device error during warm-up")
+
+    # timed region: K steps, CUDA events around every kernel on the launch stream
+    gpu_index = local
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        try:
+            gpu_index = int(vis.split(",")[local])
+        except ValueError:
+            pass
+    clocks = ClockSampler(gpu_index)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ops + 1)] for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    clocks.mark_start()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(step.stream)
+    for k in range(args.steps):
+        evs[k][0].record(step.stream)
+        step.run(evs[k])
+    t_end.record(step.stream)
+    torch.cuda.synchronize()
+    clocks.mark_end()
+    clk = clocks.stop()
+    if world > 1:
+        torch.distributed.barrier()
+    ms_total = t_start.elapsed_time(t_end)
+    if mxk.device_error() != 0:
+        raise RuntimeError("device error during the timed region")
+    per = np.array([[evs[k][i].elapsed_time(evs[k][i + 1]) for i in range(n_ops)] for k in range(args.steps)])
+    mean_ms = per.mean(axis=0)
+    ms_step = ms_total / args.steps
+    if world > 1:
+        t = torch.tensor([ms_step], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms_step = float(t.item())
+
+    peaks, peak_src = load_peaks()
+    fp8_sus = 2.0 * peaks["bf16_tflops_sustained"]     # MXFP8 dense = 2 x bf16 (nominal 4.5 / 2.25 PF)
+    hbm = peaks["hbm_gbs"]
+    kernels = {}
+    for (name, bound, work, _), ms in zip(step.ops, mean_ms):
+        if bound == "tensor":
+            ach = work / (ms * 1e-3) / 1e12
+            kernels[name] = {"ms": round(float(ms), 4), "TFLOP/s": round(ach, 1), "frac": round(ach / fp8_sus, 3)}
+        else:
+            ach = work / (ms * 1e-3) / 1e9
+            kernels[name] = {"ms": round(float(ms), 4), "GB/s": round(ach, 1), "frac": round(ach / hbm, 3)}
+    mlp_ms = float(mean_ms[: step.mlp_ops].sum())
+    cast_w_ms = float(sum(mean_ms[i] for i, (n, *_r) in enumerate(step.ops) if n.startswith("cast_w")))
+    useful = step.flops(step.R)
+    executed = step.flops(step.M)
+    value = world * useful / (ms_step * 1e-3) / 1e12
+    fwd_ms = float(mean_ms[:5].sum())
+
+    # dominant kernel and its roofline
+    imax = int(np.argmax(mean_ms[: step.mlp_ops]))
+    dname, dbound, dwork, _ = step.ops[imax]
+    dms = float(mean_ms[imax])
+    if dbound == "tensor":
+        ach = dwork / (dms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "kernel": dname, "achieved": round(ach, 1), "peak": round(fp8_sus, 1),
+                "unit": "TFLOP/s", "frac": round(ach / fp8_sus, 3),
+                "peak_source": f"{peak_src} bf16 sustained x 2 (MXFP8 nominal ratio)",
+                "traffic": ncu_traffic(dname, args.workload)}
+    else:
+        ach = dwork / (dms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "kernel": dname, "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s",
+                "frac": round(ach / hbm, 3), "peak_source": f"{peak_src} hbm_gbs",
+                "traffic": ncu_traffic(dname, args.workload)}
+
+    # end to end through the public composite API, host buffers
+    e2e = None
+    if not args.no_e2e:
+        x_h = inp.x.cpu().pin_memory()
+        dy_h = inp.dy.cpu().pin_memory()
+        off_h = torch.from_numpy(inp.routing.offsets).pin_memory()
+        x_d, dy_d, off_d = torch.empty_like(inp.x), torch.empty_like(inp.dy), torch.empty_like(step.off)
+        out_h = torch.empty(2, spec.D, dtype=torch.bfloat16).pin_memory()
+        saved = dict(h13=step.h13, h_col_codes=step.h_cc, h_col_scales=step.h_cs, x_col_codes=step.x_cc,
+                     x_col_scales=step.x_cs)
+        ws_f = torch.empty(mxk.workspace_bytes(step.M, spec.D, spec.E, spec.F, 1), dtype=torch.uint8, device=dev)
+        ws_b = torch.empty(mxk.workspace_bytes(step.M, spec.D, spec.E, spec.F, 2), dtype=torch.uint8, device=dev)
+
+        def e2e_step():
+            x_d.copy_(x_h, non_blocking=True)
+            dy_d.copy_(dy_h, non_blocking=True)
+            off_d.copy_(off_h, non_blocking=True)
+            mxk.moe_mlp_fwd(x_d, step.w13, step.w2, off_d, spec.pad, y=step.y, saved=saved, workspace=ws_f)
+            mxk.moe_mlp_bwd(dy_d, step.w13, step.w2, off_d, saved, spec.pad, dx=step.dx, dw13=step.dw13,
+                            dw2=step.dw2, workspace=ws_b)
+            out_h[0].copy_(step.y[0], non_blocking=True)
+            out_h[1].copy_(step.dx[0], non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(args.steps):
+            e2e_step()
+        b.record()
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b) / args.steps
+        if world > 1:
+            t = torch.tensor([ms], device=dev)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            ms = float(t.item())
+        h2d = x_h.numel() * 2 + dy_h.numel() * 2 + off_h.numel() * 4
+        e2e = {"value": round(world * useful / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(out_h.numel() * 2),
+               "ms_per_step": round(ms, 3)}
+        if mxk.device_error() != 0:
+            raise RuntimeError("device error during the e2e run")
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu, _ = oracle_sample(inp)
+        cpu["value"] = round(cpu["value"], 6)
+
+    sw = kernels["swiglu_quant_16384x4096"]
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "mxfp8 (e4m3 + e8m0 scales), fp32 accumulate, bf16 io",
+        "data": "synthetic (seeded routing, device-drawn bf16 activations and weights)",
+        "config": config_dict(spec, inp, {"parallelism": f"replicas x{world} (no data-path collective)"}),
+        "fwd_bwd_useful_tflops": round(value, 2),
+        "fwd_bwd_executed_tflops": round(world * executed / (ms_step * 1e-3) / 1e12, 2),
+        "mlp_ms": round(mlp_ms, 3),
+        "mlp_no_weight_cast_tflops": round(useful / ((mlp_ms - cast_w_ms) * 1e-3) / 1e12, 2),
+        "fwd_useful_tflops": round(6.0 * step.R * spec.D * spec.F / (fwd_ms * 1e-3) / 1e12, 2),
+        "swiglu_quant_gbs": sw["GB/s"], "swiglu_quant_frac_hbm": sw["frac"],
+        "kernels": kernels, "roofline": roof, "clocks": clk, "gpu_launches": n_ops * args.steps,
+        "e2e": e2e, "cpu_baseline": cpu, "source_hash": src_hash(),
+    }
+    if rank == 0:
+        print(json.dumps(line))
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())
