@@ -241,6 +241,41 @@ int moe_mlp_bwd(const void* dy, int64_t M, int64_t D,
                 void* dx, void* dw13, void* dw2,
                 void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* -------------------------------------------------------------------------
+ * moe_mlp_fwd_noalloc -- moe_mlp_fwd for callers that cannot allocate.
+ * (No counterpart in the source pages: this is a library-integration entry.)
+ *
+ * Some callers have no way to obtain device memory at call time: code that
+ * runs inside a host framework whose memory is fully owned by its own pool
+ * (an inference-server plugin, a runtime that forbids cudaMalloc after
+ * start-up because it would synchronize the device or fragment the pool), or
+ * a caller with a fixed memory budget that cannot reserve a workspace of
+ * data-dependent size.  This entry point takes the same arguments as
+ * moe_mlp_fwd minus the workspace and uses instead a scratch area compiled
+ * into the library: a file-scope device array of MXMOE_NOALLOC_SCRATCH_BYTES
+ * (32 MiB) that every GPU loading the library holds until the process exits.
+ * It never calls cudaMalloc/cudaFree or any allocating routine.
+ *
+ *  - Layers whose forward workspace (mxmoe_workspace_size(..., 1)) exceeds the
+ *    scratch size are rejected with MXMOE_ERR_WORKSPACE and a message giving
+ *    both sizes; nothing is launched.
+ *  - The first call on a device looks up the device address of the scratch
+ *    array (cudaGetSymbolAddress, with that device current); make that first
+ *    call before any CUDA stream capture begins.
+ *  - All calls on a device share the one scratch area, which keeps whatever
+ *    the previous call left there (every byte a call reads is written by that
+ *    call first).  Calls whose executions overlap on the GPU (different
+ *    streams without ordering, or concurrent host threads) race on it:
+ *    serialize them.
+ *  - Inputs, outputs and `saved` are caller-owned exactly as for moe_mlp_fwd.
+ * ------------------------------------------------------------------------- */
+#define MXMOE_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+
+int moe_mlp_fwd_noalloc(const void* x, int64_t M, int64_t D,
+                        const void* w13, const void* w2, int E, int64_t F,
+                        const int32_t* expert_offsets, int pad_multiple,
+                        void* y, const mxmoe_saved* saved, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

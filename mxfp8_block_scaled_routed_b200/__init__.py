@@ -56,6 +56,7 @@ _SIGS = {
     "mxmoe_workspace_size": ([_L, _L, _I, _L, _I], _S),
     "moe_mlp_fwd": ([_P, _L, _L, _P, _P, _I, _L, _P, _I, _P, ctypes.POINTER(_Saved), _P, _S, _P], _I),
     "moe_mlp_bwd": ([_P, _L, _L, _P, _P, _I, _L, _P, _I, ctypes.POINTER(_Saved), _P, _P, _P, _P, _S, _P], _I),
+    "moe_mlp_fwd_noalloc": ([_P, _L, _L, _P, _P, _I, _L, _P, _I, _P, ctypes.POINTER(_Saved), _P], _I),
 }
 
 _lib = None

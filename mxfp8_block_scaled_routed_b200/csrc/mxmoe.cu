@@ -566,4 +566,38 @@ int moe_mlp_bwd(const void* dy, int64_t M, int64_t D, const void* w13, const voi
                        pad_multiple, dw13, stream);
 }
 
+// Forward composite for callers that cannot allocate (see the header): the
+// workspace is a static device array of this translation unit.  Its device
+// address is looked up once per device and cached.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[MXMOE_NOALLOC_SCRATCH_BYTES];
+
+int moe_mlp_fwd_noalloc(const void* x, int64_t M, int64_t D, const void* w13, const void* w2, int E, int64_t F,
+                        const int32_t* expert_offsets, int pad_multiple, void* y, const mxmoe_saved* saved,
+                        cudaStream_t stream) {
+  static void* scratch_ptr[kMaxDevices] = {};
+  MX_TRY(check_mlp_shapes(M, D, E, F, expert_offsets, pad_multiple));
+  FwdWs w;
+  const size_t need = carve_fwd(nullptr, M, D, E, F, &w);
+  if (need > MXMOE_NOALLOC_SCRATCH_BYTES)
+    return fail(MXMOE_ERR_WORKSPACE,
+                "moe_mlp_fwd_noalloc: this layer needs %zu bytes of scratch, the static scratch holds %zu; "
+                "use moe_mlp_fwd with a caller workspace",
+                need, (size_t)MXMOE_NOALLOC_SCRATCH_BYTES);
+  int dev = 0;
+  MX_CHECK_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(MXMOE_ERR_CUDA, "device index %d out of range", dev);
+  void* ws = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!scratch_ptr[dev]) {
+      void* p = nullptr;
+      MX_CHECK_CUDA(cudaGetSymbolAddress(&p, g_noalloc_scratch), "cudaGetSymbolAddress(scratch)");
+      scratch_ptr[dev] = p;
+    }
+    ws = scratch_ptr[dev];
+  }
+  return moe_mlp_fwd(x, M, D, w13, w2, E, F, expert_offsets, pad_multiple, y, saved, ws,
+                     MXMOE_NOALLOC_SCRATCH_BYTES, stream);
+}
+
 }  // extern "C"
