@@ -134,8 +134,10 @@ class ClockSampler:
 class Step:
     """All buffers of one fwd+bwd step, laid out once; run() issues the kernels.
 
-    The sequence is exactly the one moe_mlp_fwd / moe_mlp_bwd issue, written
-    out call by call so each kernel can be bracketed with CUDA events.
+    The sequence is exactly the one mxmoe_quantize_weights + moe_mlp_fwd_q +
+    moe_mlp_bwd_q issue (a training step: the weights are quantized once, ROW
+    and COL in one pass, and used by both passes), written out call by call so
+    each kernel can be bracketed with CUDA events.
     """
 
     def __init__(self, inp, dev):
@@ -152,14 +154,11 @@ class Step:
         self.x, self.w13, self.w2, self.dy = inp.x, inp.w13, inp.w2, inp.dy
         self.off = torch.from_numpy(inp.routing.offsets).to(dev)
         self.x_rc, self.x_rs, self.x_cc, self.x_cs = u8(M, D), u8(M * D // 32), u8(D, M), u8(M * D // 32)
-        self.w13_c, self.w13_s = u8(E * 2 * F, D), u8(E * 2 * F * D // 32)
-        self.w2_c, self.w2_s = u8(E * D, F), u8(E * D * F // 32)
+        self.qw = self.mxk.make_qweights(E, D, F, dev)
         self.h13 = bf(M, 2 * F)
         self.h_rc, self.h_rs, self.h_cc, self.h_cs = u8(M, F), u8(M * F // 32), u8(F, M), u8(M * F // 32)
         self.y = bf(M, D)
         self.dy_rc, self.dy_rs, self.dy_cc, self.dy_cs = u8(M, D), u8(M * D // 32), u8(D, M), u8(M * D // 32)
-        self.w2t_c, self.w2t_s = u8(E, F, D), u8(E * F * D // 32)
-        self.w13t_c, self.w13t_s = u8(E, D, 2 * F), u8(E * D * 2 * F // 32)
         self.g_rc, self.g_rs, self.g_cc, self.g_cs = u8(M, 2 * F), u8(M * 2 * F // 32), u8(2 * F, M), u8(M * 2 * F // 32)
         self.dx, self.dw13, self.dw2 = bf(M, D), bf(E, 2 * F, D), bf(E, D, F)
         # standalone boundary kernels
@@ -176,35 +175,34 @@ class Step:
         st = self.stream.cuda_stream
         M, D, E, F, pad = self.M, self.D, self.E, self.F, self.pad
         off = p(self.off)
+        q = {k: p(v) for k, v in self.qw.items()}
         self.ops = [
             ("cast_x_dual", "hbm", 4.0625 * M * D,
              lambda: L.mxfp8_quantize(p(self.x), 1, M, D, 3, 1, p(self.x_rc), p(self.x_rs), p(self.x_cc), p(self.x_cs), st)),
-            ("cast_w13_row", "hbm", 3.03125 * E * 2 * F * D,
-             lambda: L.mxfp8_quantize(p(self.w13), 1, E * 2 * F, D, 1, 1, p(self.w13_c), p(self.w13_s), None, None, st)),
-            ("cast_w2_row", "hbm", 3.03125 * E * D * F,
-             lambda: L.mxfp8_quantize(p(self.w2), 1, E * D, F, 1, 1, p(self.w2_c), p(self.w2_s), None, None, st)),
+            ("cast_w13_dual", "hbm", 4.0625 * E * 2 * F * D,
+             lambda: L.mxfp8_quantize(p(self.w13), E, 2 * F, D, 3, 1, q["w13_codes"], q["w13_scales"], q["w13t_codes"],
+                                      q["w13t_scales"], st)),
+            ("cast_w2_dual", "hbm", 4.0625 * E * D * F,
+             lambda: L.mxfp8_quantize(p(self.w2), E, D, F, 3, 1, q["w2_codes"], q["w2_scales"], q["w2t_codes"],
+                                      q["w2t_scales"], st)),
             ("fc1_swiglu_quant", "tensor", 2.0 * M * 2 * F * D,
-             lambda: L.mxfp8_grouped_gemm_swiglu_quant(p(self.x_rc), p(self.x_rs), M, D, p(self.w13_c), p(self.w13_s), E, F,
-                                                       off, pad, p(self.h13), p(self.h_rc), p(self.h_rs), p(self.h_cc),
+             lambda: L.mxfp8_grouped_gemm_swiglu_quant(p(self.x_rc), p(self.x_rs), M, D, q["w13_codes"], q["w13_scales"], E,
+                                                       F, off, pad, p(self.h13), p(self.h_rc), p(self.h_rs), p(self.h_cc),
                                                        p(self.h_cs), st)),
             ("fc2", "tensor", 2.0 * M * D * F,
-             lambda: L.mxfp8_grouped_gemm(p(self.h_rc), p(self.h_rs), M, F, p(self.w2_c), p(self.w2_s), E, D, off, pad,
+             lambda: L.mxfp8_grouped_gemm(p(self.h_rc), p(self.h_rs), M, F, q["w2_codes"], q["w2_scales"], E, D, off, pad,
                                           p(self.y), st)),
             ("cast_dy_dual", "hbm", 4.0625 * M * D,
              lambda: L.mxfp8_quantize(p(self.dy), 1, M, D, 3, 1, p(self.dy_rc), p(self.dy_rs), p(self.dy_cc), p(self.dy_cs), st)),
-            ("cast_w2_col", "hbm", 3.03125 * E * D * F,
-             lambda: L.mxfp8_quantize(p(self.w2), E, D, F, 2, 1, None, None, p(self.w2t_c), p(self.w2t_s), st)),
-            ("cast_w13_col", "hbm", 3.03125 * E * 2 * F * D,
-             lambda: L.mxfp8_quantize(p(self.w13), E, 2 * F, D, 2, 1, None, None, p(self.w13t_c), p(self.w13t_s), st)),
             ("fc2_dgrad_dswiglu_quant", "tensor", 2.0 * M * F * D,
-             lambda: L.mxfp8_grouped_gemm_dswiglu_quant(p(self.dy_rc), p(self.dy_rs), M, D, p(self.w2t_c), p(self.w2t_s), E, F,
-                                                        off, pad, p(self.h13), p(self.g_rc), p(self.g_rs), p(self.g_cc),
-                                                        p(self.g_cs), st)),
+             lambda: L.mxfp8_grouped_gemm_dswiglu_quant(p(self.dy_rc), p(self.dy_rs), M, D, q["w2t_codes"], q["w2t_scales"],
+                                                        E, F, off, pad, p(self.h13), p(self.g_rc), p(self.g_rs),
+                                                        p(self.g_cc), p(self.g_cs), st)),
             ("wgrad_dw2", "tensor", 2.0 * M * D * F,
              lambda: L.mxfp8_grouped_gemm_wgrad(p(self.dy_cc), p(self.dy_cs), D, p(self.h_cc), p(self.h_cs), F, M, off, E, pad,
                                                 p(self.dw2), st)),
             ("dgrad_dx", "tensor", 2.0 * M * 2 * F * D,
-             lambda: L.mxfp8_grouped_gemm(p(self.g_rc), p(self.g_rs), M, 2 * F, p(self.w13t_c), p(self.w13t_s), E, D, off,
+             lambda: L.mxfp8_grouped_gemm(p(self.g_rc), p(self.g_rs), M, 2 * F, q["w13t_codes"], q["w13t_scales"], E, D, off,
                                           pad, p(self.dx), st)),
             ("wgrad_dw13", "tensor", 2.0 * M * 2 * F * D,
              lambda: L.mxfp8_grouped_gemm_wgrad(p(self.g_cc), p(self.g_cs), 2 * F, p(self.x_cc), p(self.x_cs), D, M, off, E,
@@ -215,7 +213,7 @@ class Step:
             ("cast_payload_8192x7168", "hbm", 3.03125 * CAST_ROWS * CAST_COLS,
              lambda: L.mxfp8_quantize(p(self.c_in), 1, CAST_ROWS, CAST_COLS, 1, 0, p(self.c_rc), p(self.c_rs), None, None, st)),
         ]
-        self.mlp_ops = 12
+        self.mlp_ops = 10
 
     def run(self, events=None):
         for i, (name, _, _, fn) in enumerate(self.ops):
@@ -418,7 +416,7 @@ def main():
     useful = step.flops(step.R)
     executed = step.flops(step.M)
     value = world * useful / (ms_step * 1e-3) / 1e12
-    fwd_ms = float(mean_ms[:5].sum())
+    fwd_ms = float(mean_ms[[0, 3, 4]].sum())   # x cast, FC1, FC2 (weights already quantized)
 
     # dominant kernel and its roofline
     imax = int(np.argmax(mean_ms[: step.mlp_ops]))
@@ -446,16 +444,18 @@ def main():
         out_h = torch.empty(2, spec.D, dtype=torch.bfloat16).pin_memory()
         saved = dict(h13=step.h13, h_col_codes=step.h_cc, h_col_scales=step.h_cs, x_col_codes=step.x_cc,
                      x_col_scales=step.x_cs)
-        ws_f = torch.empty(mxk.workspace_bytes(step.M, spec.D, spec.E, spec.F, 1), dtype=torch.uint8, device=dev)
-        ws_b = torch.empty(mxk.workspace_bytes(step.M, spec.D, spec.E, spec.F, 2), dtype=torch.uint8, device=dev)
+
+        ws_f = torch.empty(mxk.workspace_bytes(step.M, spec.D, spec.E, spec.F, 3), dtype=torch.uint8, device=dev)
+        ws_b = torch.empty(mxk.workspace_bytes(step.M, spec.D, spec.E, spec.F, 4), dtype=torch.uint8, device=dev)
 
         def e2e_step():
             x_d.copy_(x_h, non_blocking=True)
             dy_d.copy_(dy_h, non_blocking=True)
             off_d.copy_(off_h, non_blocking=True)
-            mxk.moe_mlp_fwd(x_d, step.w13, step.w2, off_d, spec.pad, y=step.y, saved=saved, workspace=ws_f)
-            mxk.moe_mlp_bwd(dy_d, step.w13, step.w2, off_d, saved, spec.pad, dx=step.dx, dw13=step.dw13,
-                            dw2=step.dw2, workspace=ws_b)
+            mxk.mxmoe_quantize_weights(step.w13, step.w2, qw=step.qw)
+            mxk.moe_mlp_fwd_q(x_d, step.qw, off_d, spec.pad, y=step.y, saved=saved, workspace=ws_f)
+            mxk.moe_mlp_bwd_q(dy_d, step.qw, off_d, saved, spec.pad, dx=step.dx, dw13=step.dw13, dw2=step.dw2,
+                              workspace=ws_b)
             out_h[0].copy_(step.y[0], non_blocking=True)
             out_h[1].copy_(step.dx[0], non_blocking=True)
 
@@ -498,7 +498,7 @@ def main():
         "fwd_bwd_executed_tflops": round(world * executed / (ms_step * 1e-3) / 1e12, 2),
         "mlp_ms": round(mlp_ms, 3),
         "mlp_no_weight_cast_tflops": round(useful / ((mlp_ms - cast_w_ms) * 1e-3) / 1e12, 2),
-        "fwd_useful_tflops": round(6.0 * step.R * spec.D * spec.F / (fwd_ms * 1e-3) / 1e12, 2),
+        "fwd_useful_tflops_prequantized_weights": round(6.0 * step.R * spec.D * spec.F / (fwd_ms * 1e-3) / 1e12, 2),
         "swiglu_quant_gbs": sw["GB/s"], "swiglu_quant_frac_hbm": sw["frac"],
         "kernels": kernels, "roofline": roof, "clocks": clk, "gpu_launches": n_ops * args.steps,
         "e2e": e2e, "cpu_baseline": cpu, "source_hash": src_hash(),

@@ -226,6 +226,8 @@ typedef struct {
   uint8_t* x_col_scales;   /* MMA scales of [D, M]              */
 } mxmoe_saved;
 
+/* Workspace bytes: which = 1 moe_mlp_fwd, 2 moe_mlp_bwd, 3 moe_mlp_fwd_q,
+ * 4 moe_mlp_bwd_q (0 for bad arguments). */
 size_t mxmoe_workspace_size(int64_t M, int64_t D, int E, int64_t F, int which);
 
 int moe_mlp_fwd(const void* x, int64_t M, int64_t D,
@@ -240,6 +242,41 @@ int moe_mlp_bwd(const void* dy, int64_t M, int64_t D,
                 const mxmoe_saved* saved,
                 void* dx, void* dw13, void* dw2,
                 void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* -------------------------------------------------------------------------
+ * Pre-quantized weights.  A training step uses every weight in both passes
+ * (ROW-quantized along D resp. F in the forward, COL-quantized along 2F resp.
+ * D in the backward); mxmoe_quantize_weights produces all four with one dual
+ * (ROW + COL) cast per weight, i.e. one read of each bf16 weight per step, and
+ * the _q composites consume them instead of re-casting the bf16 weights.
+ * All buffers caller-owned device memory; scales in the MMA layout.
+ * ------------------------------------------------------------------------- */
+typedef struct {
+  uint8_t* w13_codes;     /* ROW of W13: [E, 2F, D]            (FC1 operand)  */
+  uint8_t* w13_scales;    /* MMA scales of [E*2F, D]                          */
+  uint8_t* w13t_codes;    /* COL of each W13[e]: [E, D, 2F]    (dx operand)   */
+  uint8_t* w13t_scales;   /* MMA scales of [E*D, 2F]                          */
+  uint8_t* w2_codes;      /* ROW of W2: [E, D, F]              (FC2 operand)  */
+  uint8_t* w2_scales;     /* MMA scales of [E*D, F]                           */
+  uint8_t* w2t_codes;     /* COL of each W2[e]: [E, F, D]      (dh operand)   */
+  uint8_t* w2t_scales;    /* MMA scales of [E*F, D]                           */
+} mxmoe_qweights;
+
+int mxmoe_quantize_weights(const void* w13, const void* w2, int E, int64_t D, int64_t F,
+                           const mxmoe_qweights* qw, cudaStream_t stream);
+
+/* moe_mlp_fwd / moe_mlp_bwd with the weights given pre-quantized (the
+ * forward reads the ROW fields of qw, the backward the COL fields). */
+int moe_mlp_fwd_q(const void* x, int64_t M, int64_t D, const mxmoe_qweights* qw, int E, int64_t F,
+                  const int32_t* expert_offsets, int pad_multiple,
+                  void* y, const mxmoe_saved* saved,
+                  void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+int moe_mlp_bwd_q(const void* dy, int64_t M, int64_t D, const mxmoe_qweights* qw, int E, int64_t F,
+                  const int32_t* expert_offsets, int pad_multiple,
+                  const mxmoe_saved* saved,
+                  void* dx, void* dw13, void* dw2,
+                  void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /* -------------------------------------------------------------------------
  * moe_mlp_fwd_noalloc -- moe_mlp_fwd for callers that cannot allocate.

@@ -20,6 +20,7 @@ __all__ = [
     "mxfp8_grouped_gemm", "mxfp8_grouped_gemm_wgrad",
     "mxfp8_grouped_gemm_swiglu_quant", "mxfp8_grouped_gemm_dswiglu_quant",
     "moe_mlp_fwd", "moe_mlp_bwd", "device_error", "header_functions",
+    "make_qweights", "mxmoe_quantize_weights", "moe_mlp_fwd_q", "moe_mlp_bwd_q",
 ]
 
 ROW, COL = 1, 2
@@ -41,6 +42,11 @@ class _Saved(ctypes.Structure):
                 ("x_col_codes", ctypes.c_void_p), ("x_col_scales", ctypes.c_void_p)]
 
 
+class _QWeights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("w13_codes", "w13_scales", "w13t_codes", "w13t_scales",
+                                                "w2_codes", "w2_scales", "w2t_codes", "w2t_scales")]
+
+
 _P, _I, _L, _S = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
 _SIGS = {
     "mxmoe_last_error": ([], ctypes.c_char_p),
@@ -57,6 +63,11 @@ _SIGS = {
     "moe_mlp_fwd": ([_P, _L, _L, _P, _P, _I, _L, _P, _I, _P, ctypes.POINTER(_Saved), _P, _S, _P], _I),
     "moe_mlp_bwd": ([_P, _L, _L, _P, _P, _I, _L, _P, _I, ctypes.POINTER(_Saved), _P, _P, _P, _P, _S, _P], _I),
     "moe_mlp_fwd_noalloc": ([_P, _L, _L, _P, _P, _I, _L, _P, _I, _P, ctypes.POINTER(_Saved), _P], _I),
+    "mxmoe_quantize_weights": ([_P, _P, _I, _L, _L, ctypes.POINTER(_QWeights), _P], _I),
+    "moe_mlp_fwd_q": ([_P, _L, _L, ctypes.POINTER(_QWeights), _I, _L, _P, _I, _P, ctypes.POINTER(_Saved), _P, _S,
+                       _P], _I),
+    "moe_mlp_bwd_q": ([_P, _L, _L, ctypes.POINTER(_QWeights), _I, _L, _P, _I, ctypes.POINTER(_Saved), _P, _P, _P,
+                       _P, _S, _P], _I),
 }
 
 _lib = None
@@ -294,4 +305,62 @@ def moe_mlp_bwd(dy, w13, w2, offsets, saved, pad_multiple=128, dx=None, dw13=Non
     st = _saved_struct(saved)
     _check(lib().moe_mlp_bwd(_ptr(dy), M, D, _ptr(w13), _ptr(w2), E, F, _ptr(offsets), pad_multiple,
                              ctypes.byref(st), _ptr(dx), _ptr(dw13), _ptr(dw2), _ptr(ws), ws.numel(), _stream(dy)))
+    return dx, dw13, dw2
+
+
+# ----------------------------------------------------------------------------- pre-quantized weights
+def make_qweights(E, D, F, device):
+    """Buffers for the ROW and COL MXFP8 copies of W13 [E, 2F, D] and W2 [E, D, F]."""
+    return dict(w13_codes=_u8((E, 2 * F, D), device), w13_scales=_u8((E * 2 * F * D // 32,), device),
+                w13t_codes=_u8((E, D, 2 * F), device), w13t_scales=_u8((E * 2 * F * D // 32,), device),
+                w2_codes=_u8((E, D, F), device), w2_scales=_u8((E * D * F // 32,), device),
+                w2t_codes=_u8((E, F, D), device), w2t_scales=_u8((E * D * F // 32,), device))
+
+
+def _qw_struct(q):
+    return _QWeights(*(q[n].data_ptr() for n, _ in _QWeights._fields_))
+
+
+def mxmoe_quantize_weights(w13, w2, qw=None):
+    """Dual (ROW + COL) MXFP8 casts of both expert weights, one read of each."""
+    _need(w13, torch.bfloat16, "w13")
+    _need(w2, torch.bfloat16, "w2")
+    E, F2, D = w13.shape
+    F = F2 // 2
+    qw = make_qweights(E, D, F, w13.device) if qw is None else qw
+    st = _qw_struct(qw)
+    _check(lib().mxmoe_quantize_weights(_ptr(w13), _ptr(w2), E, D, F, ctypes.byref(st), _stream(w13)))
+    return qw
+
+
+def moe_mlp_fwd_q(x, qw, offsets, pad_multiple=128, y=None, saved=None, workspace=None):
+    """Forward with pre-quantized weights. Returns (y, saved)."""
+    E = _offs(offsets)
+    _need(x, torch.bfloat16, "x")
+    M, D = x.shape
+    F = qw["w13_codes"].shape[1] // 2
+    dev = x.device
+    y = torch.empty(M, D, dtype=torch.bfloat16, device=dev) if y is None else y
+    saved = make_saved(M, D, F, dev) if saved is None else saved
+    ws = _u8((workspace_bytes(M, D, E, F, 3),), dev) if workspace is None else workspace
+    st, q = _saved_struct(saved), _qw_struct(qw)
+    _check(lib().moe_mlp_fwd_q(_ptr(x), M, D, ctypes.byref(q), E, F, _ptr(offsets), pad_multiple, _ptr(y),
+                               ctypes.byref(st), _ptr(ws), ws.numel(), _stream(x)))
+    return y, saved
+
+
+def moe_mlp_bwd_q(dy, qw, offsets, saved, pad_multiple=128, dx=None, dw13=None, dw2=None, workspace=None):
+    """Backward with pre-quantized weights. Returns (dx, dw13, dw2)."""
+    E = _offs(offsets)
+    _need(dy, torch.bfloat16, "dy")
+    M, D = dy.shape
+    F = qw["w13_codes"].shape[1] // 2
+    dev = dy.device
+    dx = torch.empty(M, D, dtype=torch.bfloat16, device=dev) if dx is None else dx
+    dw13 = torch.empty(E, 2 * F, D, dtype=torch.bfloat16, device=dev) if dw13 is None else dw13
+    dw2 = torch.empty(E, D, F, dtype=torch.bfloat16, device=dev) if dw2 is None else dw2
+    ws = _u8((workspace_bytes(M, D, E, F, 4),), dev) if workspace is None else workspace
+    st, q = _saved_struct(saved), _qw_struct(qw)
+    _check(lib().moe_mlp_bwd_q(_ptr(dy), M, D, ctypes.byref(q), E, F, _ptr(offsets), pad_multiple,
+                               ctypes.byref(st), _ptr(dx), _ptr(dw13), _ptr(dw2), _ptr(ws), ws.numel(), _stream(dy)))
     return dx, dw13, dw2

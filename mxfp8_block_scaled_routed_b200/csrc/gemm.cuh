@@ -77,7 +77,9 @@ struct Cfg {
   static constexpr int OFF_SFA = OFF_B + kStages * B_BYTES;
   static constexpr int OFF_SFB = OFF_SFA + kStages * SFA_BYTES;
   static constexpr int OFF_EPI = OFF_SFB + kStages * SFB_BYTES;
-  static constexpr int EPI_BYTES = 4 * 32 * 17 * 4;        // per-warp 32x32 bf16 transpose buffer
+  static constexpr int EPI_WARPS = 8;
+  static constexpr int EPI_WARP_BYTES = 32 * 17 * 4;       // 32x32 bf16 transpose / staging buffer
+  static constexpr int EPI_BYTES = EPI_WARPS * EPI_WARP_BYTES;
   static constexpr int OFF_BAR = OFF_EPI + EPI_BYTES;
   static constexpr int NUM_BARS = 2 * kStages + 2 * kAcc;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
@@ -155,7 +157,8 @@ __device__ __forceinline__ Tile get_tile(const Params& p, const int32_t* offs, i
 // ---------------------------------------------------------------- epilogue helpers
 // Warp-level 32x32 transpose through shared memory: each lane gives one row
 // of 16 packed bf16 pairs; each lane gets one column as 16 packed pairs.
-__device__ __forceinline__ void warp_transpose32(uint32_t* buf, const uint32_t (&row)[16], uint32_t (&col)[16],
+// Row stride 17 words keeps both phases free of bank conflicts.
+__device__ __forceinline__ void warp_transpose32(uint32_t* buf, const uint32_t* row, uint32_t (&col)[16],
                                                  int lane) {
 #pragma unroll
   for (int j = 0; j < 16; ++j) buf[lane * 17 + j] = row[j];
@@ -170,9 +173,48 @@ __device__ __forceinline__ void warp_transpose32(uint32_t* buf, const uint32_t (
   __syncwarp();
 }
 
+// Store a 32-row x 64-byte block (one row per lane, 4 x 16 B in v) so that
+// each store instruction writes 8 whole 64-byte row segments: the block goes
+// through shared memory (16-byte chunk c of row r at chunk c ^ ((r >> 1) & 3),
+// conflict-free) and comes back out row-contiguous.  dst0 = first row, ld in
+// bytes.
+__device__ __forceinline__ void store_rows64(uint8_t* sbuf, const uint32_t* v, uint8_t* dst0, int64_t ld,
+                                             int lane) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c)
+    *reinterpret_cast<uint4*>(sbuf + lane * 64 + ((c ^ ((lane >> 1) & 3)) << 4)) =
+        make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = 8 * i + (lane >> 2), c = lane & 3;
+    const uint4 t = *reinterpret_cast<const uint4*>(sbuf + r * 64 + ((c ^ ((r >> 1) & 3)) << 4));
+    *reinterpret_cast<uint4*>(dst0 + r * ld + c * 16) = t;
+  }
+  __syncwarp();
+}
+
+// Same for a 32-row x 32-byte block (one row per lane, 2 x 16 B in v):
+// chunk c of row r sits at chunk c ^ ((r >> 2) & 1); each store instruction
+// writes 16 whole 32-byte row segments.
+__device__ __forceinline__ void store_rows32(uint8_t* sbuf, const uint4 (&v)[2], uint8_t* dst0, int64_t ld,
+                                             int lane) {
+#pragma unroll
+  for (int c = 0; c < 2; ++c)
+    *reinterpret_cast<uint4*>(sbuf + lane * 32 + ((c ^ ((lane >> 2) & 1)) << 4)) = v[c];
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const int r = 16 * i + (lane >> 1), c = lane & 1;
+    const uint4 t = *reinterpret_cast<const uint4*>(sbuf + r * 32 + ((c ^ ((r >> 2) & 1)) << 4));
+    *reinterpret_cast<uint4*>(dst0 + r * ld + c * 16) = t;
+  }
+  __syncwarp();
+}
+
 // Quantize 32 packed bf16 (16 words) of one block: returns the scale byte and
-// writes 32 codes to dst (16-byte aligned).
-__device__ __forceinline__ uint32_t quant32_store(const uint32_t (&v)[16], uint8_t* dst) {
+// the 32 codes.
+__device__ __forceinline__ uint32_t quant32(const uint32_t* v, uint4 (&codes)[2]) {
   uint4 q[4];
   uint32_t am = 0;
 #pragma unroll
@@ -183,15 +225,31 @@ __device__ __forceinline__ uint32_t quant32_store(const uint32_t (&v)[16], uint8
   const uint32_t byte = scale_byte_from_bits(am);
   uint2 c0 = encode8(q[0], byte), c1 = encode8(q[1], byte);
   uint2 c2 = encode8(q[2], byte), c3 = encode8(q[3], byte);
-  reinterpret_cast<uint4*>(dst)[0] = make_uint4(c0.x, c0.y, c1.x, c1.y);
-  reinterpret_cast<uint4*>(dst)[1] = make_uint4(c2.x, c2.y, c3.x, c3.y);
+  codes[0] = make_uint4(c0.x, c0.y, c1.x, c1.y);
+  codes[1] = make_uint4(c2.x, c2.y, c3.x, c3.y);
   return byte;
 }
 
-__device__ __forceinline__ void store64(uint16_t* dst, const uint32_t (&v)[16]) {
-  uint4* d = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) d[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+// ROW + COL quantization of a 32x32 bf16 block held one row per lane.
+// ROW: codes of rows row0..row0+31, columns col0..col0+31 of a [*, ld_row]
+// code matrix, scale (row, col0/32) in the MMA layout.  COL: codes of rows
+// col0+lane, columns row0..row0+31 of the transposed [*, M] code matrix,
+// scale (col0 + lane, row0/32).
+__device__ __forceinline__ void dual_quant_block(const uint32_t* v, int lane, uint8_t* sbuf, int64_t row0,
+                                                 int64_t col0, int64_t ld_row, int64_t M, uint8_t* row_codes,
+                                                 uint8_t* row_scales, uint8_t* col_codes, uint8_t* col_scales) {
+  uint4 q[2];
+  const uint32_t rb = quant32(v, q);
+  store_rows32(sbuf, q, row_codes + row0 * ld_row + col0, ld_row, lane);
+  row_scales[mma_scale_offset(row0 + lane, col0 >> 5, ld_row)] = uint8_t(rb);
+  uint32_t c[16];
+  warp_transpose32(reinterpret_cast<uint32_t*>(sbuf), v, c, lane);
+  const int64_t crow = col0 + lane;
+  const uint32_t cb = quant32(c, q);
+  uint4* dst = reinterpret_cast<uint4*>(col_codes + crow * M + row0);
+  dst[0] = q[0];
+  dst[1] = q[1];
+  col_scales[mma_scale_offset(crow, row0 >> 5, M)] = uint8_t(cb);
 }
 
 __device__ __forceinline__ void load64(const uint16_t* src, uint32_t (&v)[16]) {
@@ -203,26 +261,18 @@ __device__ __forceinline__ void load64(const uint16_t* src, uint32_t (&v)[16]) {
   }
 }
 
-// ROW + COL quantization of a 32x32 bf16 block held one row per lane.
-// ROW: codes at row_codes[(row) * ld_row + col0], scale (row, col0/32) of a
-// [*, ld_row] matrix.  COL: codes at col_codes[(col0 + lane) * M + m_blk],
-// scale (col0 + lane, m_blk/32) of a [*, M] matrix.
-__device__ __forceinline__ void dual_quant_block(const uint32_t (&v)[16], int lane, uint32_t* tbuf,
-                                                 int64_t row, int64_t col0, int64_t ld_row, int64_t m_blk,
-                                                 int64_t M, uint8_t* row_codes, uint8_t* row_scales,
-                                                 uint8_t* col_codes, uint8_t* col_scales) {
-  const uint32_t rb = quant32_store(v, row_codes + row * ld_row + col0);
-  row_scales[mma_scale_offset(row, col0 >> 5, ld_row)] = uint8_t(rb);
-  uint32_t c[16];
-  warp_transpose32(tbuf, v, c, lane);
-  const int64_t crow = col0 + lane;
-  const uint32_t cb = quant32_store(c, col_codes + crow * M + m_blk);
-  col_scales[mma_scale_offset(crow, m_blk >> 5, M)] = uint8_t(cb);
+// 32 TMEM columns of this lane's row -> 16 packed bf16 words (round to nearest even).
+__device__ __forceinline__ void drain32_bf16(uint32_t taddr, uint32_t* w) {
+  uint32_t r[32];
+  tmem_ld_32x32b_x32(taddr, r);
+  tmem_wait_ld();
+#pragma unroll
+  for (int j = 0; j < 16; ++j) w[j] = pack_bf16x2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
 }
 
 // ---------------------------------------------------------------- the kernel
 template <int kMode, int kEpi, int BN>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(384, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                     const Params p) {
   using C = Cfg<kMode, kEpi, BN>;
@@ -267,7 +317,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
     }
     for (int a = 0; a < C::kAcc; ++a) {
       mbar_init(tfull_bar(a), 1);
-      mbar_init(tempty_bar(a), 128);
+      mbar_init(tempty_bar(a), 32 * C::EPI_WARPS);
     }
     misc[1] = 0;  // abort flag
     fence_mbar_init();
@@ -357,18 +407,30 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
     }
   } else if (warp >= 4) {
     // ================= epilogue =================
-    const int q = warp - 4;                 // TMEM lane quarter
-    const int r_in = q * 32 + lane;         // row inside the 128-row tile
-    uint32_t* tbuf = reinterpret_cast<uint32_t*>(smem + C::OFF_EPI) + q * 32 * 17;
+    // Warp 4+e (e = 0..7) reads TMEM lane quarter q = warp % 4 (rows 32q..)
+    // and handles column half h = e / 4 of the tile.  The accumulator is
+    // drained into packed bf16 registers and TMEM is released before any
+    // math, so the next tile's MMAs overlap this tile's epilogue.
+    const int q = warp & 3;
+    const int h = (warp - 4) >> 2;
+    uint8_t* sbuf = smem + C::OFF_EPI + (warp - 4) * C::EPI_WARP_BYTES;
+    constexpr int kHalf = (kEpi == kEpiSwiGLU) ? 64 : BN / 2;   // accumulator columns per thread (per operand)
+    constexpr int kChunks = kHalf / 32;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x) {
       const Tile T = get_tile<kMode, kEpi, BN>(p, offs, t);
+      const int64_t row0 = T.out_r0 + q * 32;              // first row of this warp's 32-row slab
       if constexpr (kMode == kRaggedK) {
         if (T.nk == 0) {
           // expert without rows: its weight gradient is exactly zero
-          uint16_t* o = p.out + (int64_t(T.e) * p.rows_a + T.out_r0 + r_in) * p.n_out + T.out_c0;
-          for (int c = 0; c < BN; c += 8) *reinterpret_cast<uint4*>(o + c) = make_uint4(0, 0, 0, 0);
+          uint32_t z[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) z[j] = 0u;
+          uint8_t* o = reinterpret_cast<uint8_t*>(p.out + (int64_t(T.e) * p.rows_a + row0) * p.n_out + T.out_c0 +
+                                                  h * kHalf);
+#pragma unroll 1
+          for (int c = 0; c < kChunks; ++c) store_rows64(sbuf, z, o + c * 64, p.n_out * 2, lane);
           continue;
         }
       }
@@ -379,85 +441,77 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
       }
       tc_fence_after();
       const uint32_t t_row = tmem_base + (uint32_t(q * 32) << 16) + acc * BN;
+      uint32_t va[kChunks * 16];
+      uint32_t vb[(kEpi == kEpiSwiGLU) ? kChunks * 16 : 1];
+#pragma unroll
+      for (int c = 0; c < kChunks; ++c) drain32_bf16(t_row + h * kHalf + 32 * c, va + 16 * c);
+      if constexpr (kEpi == kEpiSwiGLU) {
+#pragma unroll
+        for (int c = 0; c < kChunks; ++c) drain32_bf16(t_row + 128 + h * kHalf + 32 * c, vb + 16 * c);
+      }
+      tc_fence_before();
+      mbar_arrive(tempty_bar(acc));
+      if (++acc == C::kAcc) { acc = 0; acc_phase ^= 1; }
+
       if constexpr (kEpi == kEpiBF16) {
-        uint16_t* o;
+        uint8_t* o;
         if constexpr (kMode == kRaggedK)
-          o = p.out + (int64_t(T.e) * p.rows_a + T.out_r0 + r_in) * p.n_out + T.out_c0;
+          o = reinterpret_cast<uint8_t*>(p.out + (int64_t(T.e) * p.rows_a + row0) * p.n_out + T.out_c0 + h * kHalf);
         else
-          o = p.out + (T.out_r0 + r_in) * p.n_out + T.out_c0;
-#pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(t_row + c, r);
-          tmem_wait_ld();
-          uint32_t w[16];
+          o = reinterpret_cast<uint8_t*>(p.out + row0 * p.n_out + T.out_c0 + h * kHalf);
 #pragma unroll
-          for (int j = 0; j < 16; ++j) w[j] = pack_bf16x2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
-          store64(o + c, w);
-        }
+        for (int c = 0; c < kChunks; ++c) store_rows64(sbuf, va + 16 * c, o + c * 64, p.n_out * 2, lane);
       } else if constexpr (kEpi == kEpiSwiGLU) {
-        const int64_t m = T.out_r0 + r_in;
         const int64_t F = p.F;
-#pragma unroll 1
-        for (int c = 0; c < 128; c += 32) {
-          uint32_t g[32], u[32];
-          tmem_ld_32x32b_x32(t_row + c, g);
-          tmem_ld_32x32b_x32(t_row + 128 + c, u);
-          tmem_wait_ld();
-          uint32_t a2[16], b2[16], h2[16];
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            a2[j] = pack_bf16x2(__uint_as_float(g[2 * j]), __uint_as_float(g[2 * j + 1]));
-            b2[j] = pack_bf16x2(__uint_as_float(u[2 * j]), __uint_as_float(u[2 * j + 1]));
+        for (int c = 0; c < kChunks; ++c) {
+          const int64_t f = T.out_c0 + h * kHalf + 32 * c;
+          const uint32_t* a2 = va + 16 * c;
+          const uint32_t* b2 = vb + 16 * c;
+          if (p.out != nullptr) {
+            uint8_t* o = reinterpret_cast<uint8_t*>(p.out + row0 * 2 * F);
+            store_rows64(sbuf, a2, o + f * 2, 4 * F, lane);
+            store_rows64(sbuf, b2, o + (F + f) * 2, 4 * F, lane);
+          }
+          uint32_t h2[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
             h2[j] = pack_bf16x2(silu_mul(bf16lo_to_f32(a2[j]), bf16lo_to_f32(b2[j])),
                                 silu_mul(bf16hi_to_f32(a2[j]), bf16hi_to_f32(b2[j])));
-          }
-          const int64_t f = T.out_c0 + c;
-          if (p.out != nullptr) {
-            store64(p.out + m * 2 * F + f, a2);
-            store64(p.out + m * 2 * F + F + f, b2);
-          }
-          dual_quant_block(h2, lane, tbuf, m, f, F, T.out_r0 + q * 32, p.M, p.row_codes, p.row_scales,
-                           p.col_codes, p.col_scales);
+          dual_quant_block(h2, lane, sbuf, row0, f, F, p.M, p.row_codes, p.row_scales, p.col_codes, p.col_scales);
         }
       } else {  // kEpiDSwiGLU
-        const int64_t m = T.out_r0 + r_in;
         const int64_t F = p.F;
-#pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
-          const int64_t f = T.out_c0 + c;
+        const int64_t m = row0 + lane;
+#pragma unroll
+        for (int c = 0; c < kChunks; ++c) {
+          const int64_t f = T.out_c0 + h * kHalf + 32 * c;
           uint32_t ha[16], hb[16];
           load64(p.h13 + m * 2 * F + f, ha);
           load64(p.h13 + m * 2 * F + F + f, hb);
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(t_row + c, r);
-          tmem_wait_ld();
           uint32_t dg[16], du[16];
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
+            const uint32_t dw = va[16 * c + j];
             float d[2], a[2], b[2], og[2], ou[2];
-            d[0] = round_bf16(__uint_as_float(r[2 * j]));
-            d[1] = round_bf16(__uint_as_float(r[2 * j + 1]));
+            d[0] = bf16lo_to_f32(dw); d[1] = bf16hi_to_f32(dw);
             a[0] = bf16lo_to_f32(ha[j]); a[1] = bf16hi_to_f32(ha[j]);
             b[0] = bf16lo_to_f32(hb[j]); b[1] = bf16hi_to_f32(hb[j]);
 #pragma unroll
             for (int i = 0; i < 2; ++i) {
-              const float s = 1.0f / (1.0f + expf(-a[i]));
+              const float s = sigmoid_fast(a[i]);
               og[i] = d[i] * b[i] * s * (1.0f + a[i] * (1.0f - s));
               ou[i] = d[i] * a[i] * s;
             }
             dg[j] = pack_bf16x2(og[0], og[1]);
             du[j] = pack_bf16x2(ou[0], ou[1]);
           }
-          dual_quant_block(dg, lane, tbuf, m, f, 2 * F, T.out_r0 + q * 32, p.M, p.row_codes, p.row_scales,
-                           p.col_codes, p.col_scales);
-          dual_quant_block(du, lane, tbuf, m, F + f, 2 * F, T.out_r0 + q * 32, p.M, p.row_codes,
-                           p.row_scales, p.col_codes, p.col_scales);
+          dual_quant_block(dg, lane, sbuf, row0, f, 2 * F, p.M, p.row_codes, p.row_scales, p.col_codes,
+                           p.col_scales);
+          dual_quant_block(du, lane, sbuf, row0, F + f, 2 * F, p.M, p.row_codes, p.row_scales, p.col_codes,
+                           p.col_scales);
         }
       }
-      tc_fence_before();
-      mbar_arrive(tempty_bar(acc));
-      if (++acc == C::kAcc) { acc = 0; acc_phase ^= 1; }
     }
   }
 

@@ -93,6 +93,29 @@ __device__ __forceinline__ uint2 encode8(uint4 v, uint32_t byte) {
   return byte == 0xFFu ? nan8_bf16(v) : quant8_bf16(v, inv_scale_from_byte(byte));
 }
 
+// ---------------------------------------------------------------- float-path helpers
+// max(a, |b|) that propagates NaN (an Inf/NaN anywhere in a block must reach
+// the block maximum).
+__device__ __forceinline__ float absmax_nan(float a, float b) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(fabsf(b)));
+  return r;
+}
+
+// E8M0 byte from the block maximum as fp32 (|amax|, NaN/Inf -> 0xFF); same
+// rule as scale_byte_from_bits: max(expfield - 8, 0).
+__device__ __forceinline__ uint32_t scale_byte_from_f32(float amax) {
+  const uint32_t b = __float_as_uint(amax);
+  if (b >= 0x7F800000u) return 0xFFu;
+  const int e = int(b >> 23) - 8;
+  return uint32_t(e < 0 ? 0 : e);
+}
+
+// Two E4M3 codes of two bf16 held in one 32-bit word, scaled by inv.
+__device__ __forceinline__ uint32_t e4m3x2_of_word(uint32_t w, float inv) {
+  return e4m3x2(bf16lo_to_f32(w) * inv, bf16hi_to_f32(w) * inv);
+}
+
 // ---------------------------------------------------------------- layouts
 // Byte offset of the scale of row r, 32-column block kb in the MMA (tensor
 // core) scale layout of a matrix with `kcols` columns (kcols % 128 == 0).
@@ -102,9 +125,15 @@ __device__ __forceinline__ int64_t mma_scale_offset(int64_t r, int64_t kb, int64
 }
 
 // ---------------------------------------------------------------- SwiGLU
-// h = bf16(silu(a) * b) in fp32 with IEEE division and expf.
+// sigmoid(a) = 1 / (1 + e^-a) with the fast exponential and division
+// intrinsics (relative error a few fp32 ulp, far below the bf16 rounding the
+// results go through; e^-a = inf gives exactly 0).
+__device__ __forceinline__ float sigmoid_fast(float a) {
+  return __fdividef(1.0f, 1.0f + __expf(-a));
+}
+// silu(a) * b in fp32 (rounded to bf16 by the caller).
 __device__ __forceinline__ float silu_mul(float a, float b) {
-  return a / (1.0f + expf(-a)) * b;
+  return a * sigmoid_fast(a) * b;
 }
 
 }  // namespace mxmoe

@@ -18,6 +18,12 @@
 
 using namespace mxmoe;
 
+// Tile width of the wgrad (ragged-K) GEMM when Kx allows both: 256 (one TMEM
+// accumulator) or 128 (two, epilogue overlapped with the next tile's MMAs).
+#ifndef MXMOE_WGRAD_BN
+#define MXMOE_WGRAD_BN 256
+#endif
+
 namespace {
 
 thread_local char g_err[512] = "";
@@ -111,6 +117,60 @@ int make_operand_map(CUtensorMap* map, const uint8_t* base, int64_t rows, int64_
   return MXMOE_OK;
 }
 
+// 3-D bf16 cast input [batch, rows, ld], box 128 x 128 x 1, no swizzle, zero fill
+// past the edges.
+int make_cast_map(CUtensorMap* map, const void* base, int64_t batch, int64_t rows, int64_t ld) {
+  EncodeTiledFn enc;
+  MX_TRY(get_encode(&enc));
+  cuuint64_t dims[3] = {cuuint64_t(ld), cuuint64_t(rows), cuuint64_t(batch)};
+  cuuint64_t strides[2] = {cuuint64_t(ld * 2), cuuint64_t(rows * ld * 2)};
+  cuuint32_t box[3] = {128, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MXMOE_ERR_CUDA, "cuTensorMapEncodeTiled (cast) failed (%d)", int(r));
+  return MXMOE_OK;
+}
+
+template <bool kSwiglu>
+int launch_cast(const void* in, int64_t batch, int64_t rows, int64_t cols, int modes, int layout, uint8_t* rc,
+                uint8_t* rs, uint8_t* cc, uint8_t* cs, const int32_t* dev_rows, cudaStream_t stream) {
+  using C = CastCfg<kSwiglu>;
+  DevInfo* d;
+  MX_TRY(device_info(&d));
+  const int bit = kSwiglu ? 8 : 7;
+  auto kern = mx_cast_kernel<kSwiglu>;
+  if (!(d->attr_set & (1u << bit))) {
+    MX_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem),
+                  "cudaFuncSetAttribute");
+    std::lock_guard<std::mutex> lk(g_mu);
+    d->attr_set |= (1u << bit);
+  }
+  CUtensorMap map;
+  MX_TRY(make_cast_map(&map, in, batch, rows, kSwiglu ? 2 * cols : cols));
+  CastArgs a;
+  a.rows = rows;
+  a.cols = cols;
+  a.batch = batch;
+  a.up_off = kSwiglu ? cols : 0;
+  a.tiles_c = (cols + 127) / 128;
+  a.tiles_r = (rows + 127) / 128;
+  a.modes = modes;
+  a.mma_layout = layout;
+  a.row_codes = rc;
+  a.row_scales = rs;
+  a.col_codes = cc;
+  a.col_scales = cs;
+  a.dev_rows = dev_rows;
+  const int64_t ntiles = batch * a.tiles_r * a.tiles_c;
+  const int64_t per_sm = C::kCtasPerSm;
+  const int grid = int(ntiles < per_sm * d->sms ? ntiles : per_sm * d->sms);
+  kern<<<grid, kCastThreads, C::kSmem, stream>>>(map, a);
+  MX_CHECK_CUDA(cudaGetLastError(), "cast launch");
+  return MXMOE_OK;
+}
+
 // ---------------------------------------------------------------- GEMM launch
 template <int kMode, int kEpi, int BN>
 int launch_gemm(const uint8_t* a, int64_t a_rows, const uint8_t* b, int64_t b_rows, gemm::Params p,
@@ -131,7 +191,7 @@ int launch_gemm(const uint8_t* a, int64_t a_rows, const uint8_t* b, int64_t b_ro
   MX_TRY(make_operand_map(&mb, b, b_rows, p.kext));
   if (max_tiles <= 0) return MXMOE_OK;
   const int grid = int(max_tiles < d->sms ? max_tiles : d->sms);
-  kern<<<grid, 256, C::SMEM_BYTES, stream>>>(ma, mb, p);
+  kern<<<grid, 384, C::SMEM_BYTES, stream>>>(ma, mb, p);
   MX_CHECK_CUDA(cudaGetLastError(), "grouped GEMM launch");
   return MXMOE_OK;
 }
@@ -193,50 +253,17 @@ int quantize_impl(const void* x, int64_t batch, int64_t rows, int64_t cols, int 
     MX_CHECK_CUDA(cudaGetLastError(), "cast launch");
     return MXMOE_OK;
   }
-  TileArgs a;
-  a.in = in;
-  a.rows = rows;
-  a.cols = cols;
-  a.ld_in = swiglu ? 2 * cols : cols;
-  a.up_off = swiglu ? cols : 0;
-  a.modes = modes;
-  a.mma_layout = layout;
-  a.row_codes = rc;
-  a.row_scales = rs;
-  a.col_codes = cc;
-  a.col_scales = cs;
-  a.dev_rows = nullptr;
-  dim3 grid(unsigned((cols + 127) / 128), unsigned((rows + 127) / 128), unsigned(batch));
-  if (grid.y > 65535 || grid.z > 65535) return fail(MXMOE_ERR_SHAPE, "tensor too large for the cast grid");
   if (swiglu)
-    mx_tile_kernel<true><<<grid, kTileThreads, 0, stream>>>(a);
-  else
-    mx_tile_kernel<false><<<grid, kTileThreads, 0, stream>>>(a);
-  MX_CHECK_CUDA(cudaGetLastError(), "cast launch");
-  return MXMOE_OK;
+    return launch_cast<true>(x, 1, rows, cols, modes, layout, rc, rs, cc, cs, nullptr, stream);
+  return launch_cast<false>(x, batch, rows, cols, modes, layout, rc, rs, cc, cs, nullptr, stream);
 }
 
 // Cast of the token buffer used inside the composites: rows at or past
 // offsets[E] (read on the device) are neither read nor written.
 int quantize_tokens(const void* x, int64_t rows, int64_t cols, const int32_t* rows_dev, uint8_t* rc, uint8_t* rs,
                     uint8_t* cc, uint8_t* cs, cudaStream_t stream) {
-  TileArgs a;
-  a.in = static_cast<const uint16_t*>(x);
-  a.rows = rows;
-  a.cols = cols;
-  a.ld_in = cols;
-  a.up_off = 0;
-  a.modes = MXFP8_ROW | MXFP8_COL;
-  a.mma_layout = 1;
-  a.row_codes = rc;
-  a.row_scales = rs;
-  a.col_codes = cc;
-  a.col_scales = cs;
-  a.dev_rows = rows_dev;
-  dim3 grid(unsigned(cols / 128), unsigned(rows / 128), 1);
-  mx_tile_kernel<false><<<grid, kTileThreads, 0, stream>>>(a);
-  MX_CHECK_CUDA(cudaGetLastError(), "cast launch");
-  return MXMOE_OK;
+  return launch_cast<false>(x, 1, rows, cols, MXFP8_ROW | MXFP8_COL, MXFP8_SCALE_MMA, rc, rs, cc, cs, rows_dev,
+                            stream);
 }
 
 int gemm_ragged_m(const uint8_t* a, const uint8_t* as, int64_t M, int64_t K, const uint8_t* w,
@@ -273,7 +300,7 @@ int gemm_ragged_k(const uint8_t* gt, const uint8_t* gs, int64_t N, const uint8_t
   p.a_scales = gs;
   p.b_scales = xs;
   p.out = static_cast<uint16_t*>(dw);
-  if (Kx % 256 == 0)
+  if (Kx % 256 == 0 && MXMOE_WGRAD_BN == 256)
     return launch_gemm<gemm::kRaggedK, gemm::kEpiBF16, 256>(gt, N, xt, Kx, p, int64_t(E) * (N / 128) * (Kx / 256),
                                                             stream, 2);
   return launch_gemm<gemm::kRaggedK, gemm::kEpiBF16, 128>(gt, N, xt, Kx, p, int64_t(E) * (N / 128) * (Kx / 128),
@@ -343,40 +370,97 @@ struct Carver {
 };
 
 struct FwdWs {
-  uint8_t *x_rc, *x_rs, *w13_c, *w13_s, *w2_c, *w2_s, *h_rc, *h_rs;
+  uint8_t *x_rc, *x_rs, *h_rc, *h_rs;
+  mxmoe_qweights qw;   // ROW weight codes when the caller gives bf16 weights
 };
 struct BwdWs {
-  uint8_t *dy_rc, *dy_rs, *dy_cc, *dy_cs, *w2t_c, *w2t_s, *w13t_c, *w13t_s, *g_rc, *g_rs, *g_cc, *g_cs;
+  uint8_t *dy_rc, *dy_rs, *dy_cc, *dy_cs, *g_rc, *g_rs, *g_cc, *g_cs;
+  mxmoe_qweights qw;   // COL weight codes when the caller gives bf16 weights
 };
 
-size_t carve_fwd(uint8_t* base, int64_t M, int64_t D, int E, int64_t F, FwdWs* w) {
+// with_weights: also carve room for the weight codes (bf16-weight composites)
+size_t carve_fwd(uint8_t* base, int64_t M, int64_t D, int E, int64_t F, FwdWs* w, bool with_weights) {
   Carver c{base};
   w->x_rc = c.take<uint8_t>(M * D);
   w->x_rs = c.take<uint8_t>(M * D / 32);
-  w->w13_c = c.take<uint8_t>(int64_t(E) * 2 * F * D);
-  w->w13_s = c.take<uint8_t>(int64_t(E) * 2 * F * D / 32);
-  w->w2_c = c.take<uint8_t>(int64_t(E) * D * F);
-  w->w2_s = c.take<uint8_t>(int64_t(E) * D * F / 32);
   w->h_rc = c.take<uint8_t>(M * F);
   w->h_rs = c.take<uint8_t>(M * F / 32);
+  w->qw = mxmoe_qweights{};
+  if (with_weights) {
+    w->qw.w13_codes = c.take<uint8_t>(int64_t(E) * 2 * F * D);
+    w->qw.w13_scales = c.take<uint8_t>(int64_t(E) * 2 * F * D / 32);
+    w->qw.w2_codes = c.take<uint8_t>(int64_t(E) * D * F);
+    w->qw.w2_scales = c.take<uint8_t>(int64_t(E) * D * F / 32);
+  }
   return c.off + 256;
 }
 
-size_t carve_bwd(uint8_t* base, int64_t M, int64_t D, int E, int64_t F, BwdWs* w) {
+size_t carve_bwd(uint8_t* base, int64_t M, int64_t D, int E, int64_t F, BwdWs* w, bool with_weights) {
   Carver c{base};
   w->dy_rc = c.take<uint8_t>(M * D);
   w->dy_rs = c.take<uint8_t>(M * D / 32);
   w->dy_cc = c.take<uint8_t>(M * D);
   w->dy_cs = c.take<uint8_t>(M * D / 32);
-  w->w2t_c = c.take<uint8_t>(int64_t(E) * D * F);
-  w->w2t_s = c.take<uint8_t>(int64_t(E) * D * F / 32);
-  w->w13t_c = c.take<uint8_t>(int64_t(E) * 2 * F * D);
-  w->w13t_s = c.take<uint8_t>(int64_t(E) * 2 * F * D / 32);
   w->g_rc = c.take<uint8_t>(M * 2 * F);
   w->g_rs = c.take<uint8_t>(M * 2 * F / 32);
   w->g_cc = c.take<uint8_t>(M * 2 * F);
   w->g_cs = c.take<uint8_t>(M * 2 * F / 32);
+  w->qw = mxmoe_qweights{};
+  if (with_weights) {
+    w->qw.w2t_codes = c.take<uint8_t>(int64_t(E) * D * F);
+    w->qw.w2t_scales = c.take<uint8_t>(int64_t(E) * D * F / 32);
+    w->qw.w13t_codes = c.take<uint8_t>(int64_t(E) * 2 * F * D);
+    w->qw.w13t_scales = c.take<uint8_t>(int64_t(E) * 2 * F * D / 32);
+  }
   return c.off + 256;
+}
+
+// forward with ROW-quantized weights in qw (a1, a3, a4)
+int fwd_core(const void* x, int64_t M, int64_t D, const mxmoe_qweights& qw, int E, int64_t F,
+             const int32_t* offsets, int pad, void* y, const mxmoe_saved* saved, const FwdWs& w,
+             cudaStream_t stream) {
+  // a1: x -> ROW (FC1 operand) + COL (dW13 operand, saved)
+  MX_TRY(quantize_tokens(x, M, D, offsets + E, w.x_rc, w.x_rs, saved->x_col_codes, saved->x_col_scales, stream));
+  // a3: FC1 + SwiGLU + dual quantization
+  MX_TRY(gemm_swiglu(w.x_rc, w.x_rs, M, D, qw.w13_codes, qw.w13_scales, E, F, offsets, pad, saved->h13, w.h_rc,
+                     w.h_rs, saved->h_col_codes, saved->h_col_scales, stream));
+  // a4: FC2
+  return gemm_ragged_m(w.h_rc, w.h_rs, M, F, qw.w2_codes, qw.w2_scales, E, D, offsets, pad, y, stream);
+}
+
+// backward with COL-quantized weights in qw (a5 - a9)
+int bwd_core(const void* dy, int64_t M, int64_t D, const mxmoe_qweights& qw, int E, int64_t F,
+             const int32_t* offsets, int pad, const mxmoe_saved* saved, void* dx, void* dw13, void* dw2,
+             const BwdWs& w, cudaStream_t stream) {
+  // a5: dY -> ROW (dh operand) + COL (dW2 operand)
+  MX_TRY(quantize_tokens(dy, M, D, offsets + E, w.dy_rc, w.dy_rs, w.dy_cc, w.dy_cs, stream));
+  // a6: dh = dY . W2[e] with the fused dSwiGLU + dual quantization
+  MX_TRY(gemm_dswiglu(w.dy_rc, w.dy_rs, M, D, qw.w2t_codes, qw.w2t_scales, E, F, offsets, pad, saved->h13, w.g_rc,
+                      w.g_rs, w.g_cc, w.g_cs, stream));
+  // a7: dW2[e] = dY_e^T . h_e
+  MX_TRY(gemm_ragged_k(w.dy_cc, w.dy_cs, D, saved->h_col_codes, saved->h_col_scales, F, M, offsets, E, pad, dw2,
+                       stream));
+  // a8: dx = dh13 . W13[e]
+  MX_TRY(gemm_ragged_m(w.g_rc, w.g_rs, M, 2 * F, qw.w13t_codes, qw.w13t_scales, E, D, offsets, pad, dx, stream));
+  // a9: dW13[e] = dh13_e^T . x_e
+  return gemm_ragged_k(w.g_cc, w.g_cs, 2 * F, saved->x_col_codes, saved->x_col_scales, D, M, offsets, E, pad, dw13,
+                       stream);
+}
+
+int check_qweights(const mxmoe_qweights* qw, bool fwd, bool bwd) {
+  if (!qw) return fail(MXMOE_ERR_NULL, "qweights is NULL");
+  if (fwd) MX_TRY(check_ptrs({{"qw.w13_codes", qw->w13_codes}, {"qw.w13_scales", qw->w13_scales},
+                              {"qw.w2_codes", qw->w2_codes}, {"qw.w2_scales", qw->w2_scales}}));
+  if (bwd) MX_TRY(check_ptrs({{"qw.w13t_codes", qw->w13t_codes}, {"qw.w13t_scales", qw->w13t_scales},
+                              {"qw.w2t_codes", qw->w2t_codes}, {"qw.w2t_scales", qw->w2t_scales}}));
+  return MXMOE_OK;
+}
+
+int check_saved(const mxmoe_saved* saved) {
+  if (!saved) return fail(MXMOE_ERR_NULL, "saved is NULL");
+  return check_ptrs({{"saved.h13", saved->h13}, {"saved.h_col_codes", saved->h_col_codes},
+                     {"saved.h_col_scales", saved->h_col_scales}, {"saved.x_col_codes", saved->x_col_codes},
+                     {"saved.x_col_scales", saved->x_col_scales}});
 }
 
 int check_mlp_shapes(int64_t M, int64_t D, int E, int64_t F, const int32_t* offsets, int pad) {
@@ -500,70 +584,96 @@ size_t mxmoe_workspace_size(int64_t M, int64_t D, int E, int64_t F, int which) {
   if (M <= 0 || D <= 0 || E <= 0 || F <= 0) return 0;
   FwdWs f;
   BwdWs b;
-  if (which == 1) return carve_fwd(nullptr, M, D, E, F, &f);
-  if (which == 2) return carve_bwd(nullptr, M, D, E, F, &b);
-  return 0;
+  switch (which) {
+    case 1: return carve_fwd(nullptr, M, D, E, F, &f, true);
+    case 2: return carve_bwd(nullptr, M, D, E, F, &b, true);
+    case 3: return carve_fwd(nullptr, M, D, E, F, &f, false);
+    case 4: return carve_bwd(nullptr, M, D, E, F, &b, false);
+    default: return 0;
+  }
+}
+
+int mxmoe_quantize_weights(const void* w13, const void* w2, int E, int64_t D, int64_t F, const mxmoe_qweights* qw,
+                           cudaStream_t stream) {
+  if (E <= 0) return fail(MXMOE_ERR_SHAPE, "E=%d must be positive", E);
+  MX_TRY(check_mult("D", D, 128));
+  MX_TRY(check_mult("F", F, 128));
+  MX_TRY(check_ptrs({{"w13", w13}, {"w2", w2}}));
+  MX_TRY(check_qweights(qw, true, true));
+  // W13[e] [2F, D]: ROW along D (FC1) and COL along 2F (dx), one read of W13
+  MX_TRY(quantize_impl(w13, E, 2 * F, D, MXFP8_ROW | MXFP8_COL, MXFP8_SCALE_MMA, qw->w13_codes, qw->w13_scales,
+                       qw->w13t_codes, qw->w13t_scales, stream));
+  // W2[e] [D, F]: ROW along F (FC2) and COL along D (dh), one read of W2
+  return quantize_impl(w2, E, D, F, MXFP8_ROW | MXFP8_COL, MXFP8_SCALE_MMA, qw->w2_codes, qw->w2_scales,
+                       qw->w2t_codes, qw->w2t_scales, stream);
 }
 
 int moe_mlp_fwd(const void* x, int64_t M, int64_t D, const void* w13, const void* w2, int E, int64_t F,
                 const int32_t* expert_offsets, int pad_multiple, void* y, const mxmoe_saved* saved, void* workspace,
                 size_t workspace_bytes, cudaStream_t stream) {
   MX_TRY(check_mlp_shapes(M, D, E, F, expert_offsets, pad_multiple));
-  if (!saved) return fail(MXMOE_ERR_NULL, "saved is NULL");
-  MX_TRY(check_ptrs({{"x", x}, {"w13", w13}, {"w2", w2}, {"y", y}, {"saved.h13", saved->h13},
-                     {"saved.h_col_codes", saved->h_col_codes}, {"saved.h_col_scales", saved->h_col_scales},
-                     {"saved.x_col_codes", saved->x_col_codes}, {"saved.x_col_scales", saved->x_col_scales}}));
+  MX_TRY(check_ptrs({{"x", x}, {"w13", w13}, {"w2", w2}, {"y", y}}));
+  MX_TRY(check_saved(saved));
   FwdWs w;
-  const size_t need = carve_fwd(nullptr, M, D, E, F, &w);
+  const size_t need = carve_fwd(nullptr, M, D, E, F, &w, true);
   if (!workspace || workspace_bytes < need)
     return fail(MXMOE_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed", workspace_bytes, need);
-  carve_fwd(align_ws(workspace), M, D, E, F, &w);
-  // a1: x -> ROW (FC1 operand) + COL (dW13 operand, saved)
-  MX_TRY(quantize_tokens(x, M, D, expert_offsets + E, w.x_rc, w.x_rs, saved->x_col_codes, saved->x_col_scales,
-                         stream));
+  carve_fwd(align_ws(workspace), M, D, E, F, &w, true);
   // a2: weights, ROW along the contraction dimension of each forward GEMM
-  MX_TRY(quantize_impl(w13, 1, int64_t(E) * 2 * F, D, MXFP8_ROW, MXFP8_SCALE_MMA, w.w13_c, w.w13_s, nullptr,
+  MX_TRY(quantize_impl(w13, 1, int64_t(E) * 2 * F, D, MXFP8_ROW, MXFP8_SCALE_MMA, w.qw.w13_codes, w.qw.w13_scales,
+                       nullptr, nullptr, stream));
+  MX_TRY(quantize_impl(w2, 1, int64_t(E) * D, F, MXFP8_ROW, MXFP8_SCALE_MMA, w.qw.w2_codes, w.qw.w2_scales, nullptr,
                        nullptr, stream));
-  MX_TRY(quantize_impl(w2, 1, int64_t(E) * D, F, MXFP8_ROW, MXFP8_SCALE_MMA, w.w2_c, w.w2_s, nullptr, nullptr,
-                       stream));
-  // a3: FC1 + SwiGLU + dual quantization
-  MX_TRY(gemm_swiglu(w.x_rc, w.x_rs, M, D, w.w13_c, w.w13_s, E, F, expert_offsets, pad_multiple, saved->h13,
-                     w.h_rc, w.h_rs, saved->h_col_codes, saved->h_col_scales, stream));
-  // a4: FC2
-  return gemm_ragged_m(w.h_rc, w.h_rs, M, F, w.w2_c, w.w2_s, E, D, expert_offsets, pad_multiple, y, stream);
+  return fwd_core(x, M, D, w.qw, E, F, expert_offsets, pad_multiple, y, saved, w, stream);
 }
 
 int moe_mlp_bwd(const void* dy, int64_t M, int64_t D, const void* w13, const void* w2, int E, int64_t F,
                 const int32_t* expert_offsets, int pad_multiple, const mxmoe_saved* saved, void* dx, void* dw13,
                 void* dw2, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   MX_TRY(check_mlp_shapes(M, D, E, F, expert_offsets, pad_multiple));
-  if (!saved) return fail(MXMOE_ERR_NULL, "saved is NULL");
-  MX_TRY(check_ptrs({{"dy", dy}, {"w13", w13}, {"w2", w2}, {"dx", dx}, {"dw13", dw13}, {"dw2", dw2},
-                     {"saved.h13", saved->h13}, {"saved.h_col_codes", saved->h_col_codes},
-                     {"saved.h_col_scales", saved->h_col_scales}, {"saved.x_col_codes", saved->x_col_codes},
-                     {"saved.x_col_scales", saved->x_col_scales}}));
+  MX_TRY(check_ptrs({{"dy", dy}, {"w13", w13}, {"w2", w2}, {"dx", dx}, {"dw13", dw13}, {"dw2", dw2}}));
+  MX_TRY(check_saved(saved));
   BwdWs w;
-  const size_t need = carve_bwd(nullptr, M, D, E, F, &w);
+  const size_t need = carve_bwd(nullptr, M, D, E, F, &w, true);
   if (!workspace || workspace_bytes < need)
     return fail(MXMOE_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed", workspace_bytes, need);
-  carve_bwd(align_ws(workspace), M, D, E, F, &w);
-  // a5: dY -> ROW (dh operand) + COL (dW2 operand)
-  MX_TRY(quantize_tokens(dy, M, D, expert_offsets + E, w.dy_rc, w.dy_rs, w.dy_cc, w.dy_cs, stream));
+  carve_bwd(align_ws(workspace), M, D, E, F, &w, true);
   // a2 (backward): W2 COL along D, W13 COL along 2F, per expert
-  MX_TRY(quantize_impl(w2, E, D, F, MXFP8_COL, MXFP8_SCALE_MMA, nullptr, nullptr, w.w2t_c, w.w2t_s, stream));
-  MX_TRY(quantize_impl(w13, E, 2 * F, D, MXFP8_COL, MXFP8_SCALE_MMA, nullptr, nullptr, w.w13t_c, w.w13t_s, stream));
-  // a6: dh = dY . W2[e] with the fused dSwiGLU + dual quantization
-  MX_TRY(gemm_dswiglu(w.dy_rc, w.dy_rs, M, D, w.w2t_c, w.w2t_s, E, F, expert_offsets, pad_multiple, saved->h13,
-                      w.g_rc, w.g_rs, w.g_cc, w.g_cs, stream));
-  // a7: dW2[e] = dY_e^T . h_e
-  MX_TRY(gemm_ragged_k(w.dy_cc, w.dy_cs, D, saved->h_col_codes, saved->h_col_scales, F, M, expert_offsets, E,
-                       pad_multiple, dw2, stream));
-  // a8: dx = dh13 . W13[e]
-  MX_TRY(gemm_ragged_m(w.g_rc, w.g_rs, M, 2 * F, w.w13t_c, w.w13t_s, E, D, expert_offsets, pad_multiple, dx,
+  MX_TRY(quantize_impl(w2, E, D, F, MXFP8_COL, MXFP8_SCALE_MMA, nullptr, nullptr, w.qw.w2t_codes, w.qw.w2t_scales,
                        stream));
-  // a9: dW13[e] = dh13_e^T . x_e
-  return gemm_ragged_k(w.g_cc, w.g_cs, 2 * F, saved->x_col_codes, saved->x_col_scales, D, M, expert_offsets, E,
-                       pad_multiple, dw13, stream);
+  MX_TRY(quantize_impl(w13, E, 2 * F, D, MXFP8_COL, MXFP8_SCALE_MMA, nullptr, nullptr, w.qw.w13t_codes,
+                       w.qw.w13t_scales, stream));
+  return bwd_core(dy, M, D, w.qw, E, F, expert_offsets, pad_multiple, saved, dx, dw13, dw2, w, stream);
+}
+
+int moe_mlp_fwd_q(const void* x, int64_t M, int64_t D, const mxmoe_qweights* qw, int E, int64_t F,
+                  const int32_t* expert_offsets, int pad_multiple, void* y, const mxmoe_saved* saved,
+                  void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  MX_TRY(check_mlp_shapes(M, D, E, F, expert_offsets, pad_multiple));
+  MX_TRY(check_ptrs({{"x", x}, {"y", y}}));
+  MX_TRY(check_qweights(qw, true, false));
+  MX_TRY(check_saved(saved));
+  FwdWs w;
+  const size_t need = carve_fwd(nullptr, M, D, E, F, &w, false);
+  if (!workspace || workspace_bytes < need)
+    return fail(MXMOE_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed", workspace_bytes, need);
+  carve_fwd(align_ws(workspace), M, D, E, F, &w, false);
+  return fwd_core(x, M, D, *qw, E, F, expert_offsets, pad_multiple, y, saved, w, stream);
+}
+
+int moe_mlp_bwd_q(const void* dy, int64_t M, int64_t D, const mxmoe_qweights* qw, int E, int64_t F,
+                  const int32_t* expert_offsets, int pad_multiple, const mxmoe_saved* saved, void* dx, void* dw13,
+                  void* dw2, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  MX_TRY(check_mlp_shapes(M, D, E, F, expert_offsets, pad_multiple));
+  MX_TRY(check_ptrs({{"dy", dy}, {"dx", dx}, {"dw13", dw13}, {"dw2", dw2}}));
+  MX_TRY(check_qweights(qw, false, true));
+  MX_TRY(check_saved(saved));
+  BwdWs w;
+  const size_t need = carve_bwd(nullptr, M, D, E, F, &w, false);
+  if (!workspace || workspace_bytes < need)
+    return fail(MXMOE_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed", workspace_bytes, need);
+  carve_bwd(align_ws(workspace), M, D, E, F, &w, false);
+  return bwd_core(dy, M, D, *qw, E, F, expert_offsets, pad_multiple, saved, dx, dw13, dw2, w, stream);
 }
 
 // Forward composite for callers that cannot allocate (see the header): the
@@ -577,7 +687,7 @@ int moe_mlp_fwd_noalloc(const void* x, int64_t M, int64_t D, const void* w13, co
   static void* scratch_ptr[kMaxDevices] = {};
   MX_TRY(check_mlp_shapes(M, D, E, F, expert_offsets, pad_multiple));
   FwdWs w;
-  const size_t need = carve_fwd(nullptr, M, D, E, F, &w);
+  const size_t need = carve_fwd(nullptr, M, D, E, F, &w, true);
   if (need > MXMOE_NOALLOC_SCRATCH_BYTES)
     return fail(MXMOE_ERR_WORKSPACE,
                 "moe_mlp_fwd_noalloc: this layer needs %zu bytes of scratch, the static scratch holds %zu; "

@@ -8,40 +8,50 @@
 // Dequantization: A2E transport page, review "[P2] Handle the two E8M0
 // endpoint encodings before shifting".
 //
-// HBM-bound work: one 128 x 128 tile per CTA, 128-bit loads, the ROW pass in
-// registers straight from the loads (4 lanes per 32-block, shuffle amax), the
-// tile parked in shared memory for the COL pass (one thread per column block
-// of 32 rows, stores of 32 contiguous codes).  With the MMA scale layout the
-// tile's 512 scale bytes of each direction land in one contiguous atom.
+// HBM-bound work: persistent CTAs, a TMA producer warp keeps 128 x 128 tiles
+// streaming into shared memory while eight consumer warps quantize the
+// previous ones (ROW pass: 4 lanes per 32-block, shuffle amax; COL pass: one
+// thread per column pair of a 32-row block, stores of 32 contiguous codes).
+// With the MMA scale layout the tile's 512 scale bytes of each direction land
+// in one contiguous atom.
 #pragma once
+#include <cuda.h>
 #include "mx_common.cuh"
+#include "sm100.cuh"
 
 namespace mxmoe {
 
-struct TileArgs {
-  const uint16_t* in;   // bf16 input
-  int64_t rows;         // rows of the (output) matrix per batch
+struct CastArgs {
+  int64_t rows;         // rows of the quantized matrix per batch
   int64_t cols;         // columns of the quantized matrix (F for SwiGLU)
-  int64_t ld_in;        // elements per input row (cols, or 2F for SwiGLU)
-  int64_t up_off;       // SwiGLU: column offset of the up half (F)
+  int64_t batch;
+  int64_t up_off;       // SwiGLU: column offset of the up half in the input (F)
+  int64_t tiles_c;      // 128-column tiles per row band
+  int64_t tiles_r;      // 128-row tiles per batch
   int modes;            // MXFP8_ROW | MXFP8_COL
   int mma_layout;       // 0 plain, 1 MMA
   uint8_t* row_codes;
   uint8_t* row_scales;
   uint8_t* col_codes;
   uint8_t* col_scales;
-  const int32_t* dev_rows;  // optional: rows at or past *dev_rows are not read or written
+  const int32_t* dev_rows;  // optional: rows at or past *dev_rows are neither read nor written
 };
 
 constexpr int kTile = 128;
-constexpr int kTileThreads = 256;
+constexpr int kCastConsumers = 256;                 // 8 warps
+constexpr int kCastThreads = kCastConsumers + 32;   // + 1 TMA producer warp
+constexpr int kTileBytes = kTile * kTile * 2;       // one bf16 128 x 128 tile
 
-__device__ __forceinline__ uint4 ld_nc_v4(const uint16_t* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
-  return v;
-}
+template <bool kSwiglu>
+struct CastCfg {
+  static constexpr int kStages = 2;
+  static constexpr int kStageBytes = kSwiglu ? 2 * kTileBytes : kTileBytes;
+  static constexpr int kOffColStage = kStages * kStageBytes;         // COL codes of one tile, 128 x 128 B
+  static constexpr int kOffScales = kOffColStage + kTile * kTile;    // ROW then COL scale bytes, 512 B each
+  static constexpr int kOffBars = kOffScales + 1024;
+  static constexpr int kSmem = kOffBars + 2 * kStages * 8 + 128;     // + alignment slack
+  static constexpr int kCtasPerSm = kSwiglu ? 1 : 2;
+};
 
 __device__ __forceinline__ uint32_t swiglu_pair(uint32_t g, uint32_t u) {
   float h0 = silu_mul(bf16lo_to_f32(g), bf16lo_to_f32(u));
@@ -49,105 +59,249 @@ __device__ __forceinline__ uint32_t swiglu_pair(uint32_t g, uint32_t u) {
   return pack_bf16x2(h0, h1);
 }
 
+// ROW quantization of 8 bf16 (one uint4) whose 32-block spans 4 consecutive
+// lanes; returns the 8 codes, *byte_out the block's scale byte.
+__device__ __forceinline__ uint2 row_quant8(uint4 v, uint32_t* byte_out) {
+  float m = 0.0f;
+  m = absmax_nan(m, bf16lo_to_f32(v.x)); m = absmax_nan(m, bf16hi_to_f32(v.x));
+  m = absmax_nan(m, bf16lo_to_f32(v.y)); m = absmax_nan(m, bf16hi_to_f32(v.y));
+  m = absmax_nan(m, bf16lo_to_f32(v.z)); m = absmax_nan(m, bf16hi_to_f32(v.z));
+  m = absmax_nan(m, bf16lo_to_f32(v.w)); m = absmax_nan(m, bf16hi_to_f32(v.w));
+  m = absmax_nan(m, __shfl_xor_sync(0xffffffffu, m, 1));
+  m = absmax_nan(m, __shfl_xor_sync(0xffffffffu, m, 2));
+  const uint32_t byte = scale_byte_from_f32(m);
+  *byte_out = byte;
+  if (byte == 0xFFu) return nan8_bf16(v);
+  const float inv = inv_scale_from_byte(byte);
+  uint2 o;
+  o.x = e4m3x2_of_word(v.x, inv) | (e4m3x2_of_word(v.y, inv) << 16);
+  o.y = e4m3x2_of_word(v.z, inv) | (e4m3x2_of_word(v.w, inv) << 16);
+  return o;
+}
+
+// COL quantization of one column of a 32-row block: the column's values are
+// the low (hi_half = false) or high halves of the 32 words w[j] (word j =
+// row j, two adjacent columns).  Returns the scale byte, codes in q.
+template <bool kHi>
+__device__ __forceinline__ uint32_t col_quant32(const uint32_t (&w)[32], uint4 (&q)[2]) {
+  auto val = [&](int j) { return kHi ? bf16hi_to_f32(w[j]) : bf16lo_to_f32(w[j]); };
+  float m = 0.0f;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) m = absmax_nan(m, val(j));
+  const uint32_t byte = scale_byte_from_f32(m);
+  uint32_t c[8];
+  if (byte == 0xFFu) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      uint32_t r = 0x7F7F7F7Fu;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) r |= ((__float_as_uint(val(4 * k + i)) >> 31) << 7) << (8 * i);
+      c[k] = r;
+    }
+  } else {
+    const float inv = inv_scale_from_byte(byte);
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      c[k] = e4m3x2(val(4 * k) * inv, val(4 * k + 1) * inv) | (e4m3x2(val(4 * k + 2) * inv, val(4 * k + 3) * inv) << 16);
+  }
+  q[0] = make_uint4(c[0], c[1], c[2], c[3]);
+  q[1] = make_uint4(c[4], c[5], c[6], c[7]);
+  return byte;
+}
+
+// Persistent, TMA-fed cast.  Warp 8 streams 128 x 128 bf16 tiles (3-D tensor
+// map [batch, rows, cols], zero fill past the edges) into a ring of shared
+// memory stages; warps 0..7 quantize each tile straight from shared memory:
+//  ROW: lane = 8 consecutive elements, 4 lanes = one 32-block (amax by two
+//       shuffles), codes stored 8 bytes per lane (two 128-byte rows per warp
+//       store);
+//  COL: thread = two adjacent columns of one 32-row block (32 four-byte
+//       shared loads), 32 codes per column stored as two 16-byte stores.
+// SwiGLU: the gate and up tiles arrive together; the ROW pass computes
+// h = bf16(silu(gate) * up), quantizes it and parks it over the gate tile
+// for the COL pass (one barrier among the 256 consumer threads).
 template <bool kSwiglu>
-__global__ void __launch_bounds__(kTileThreads)
-mx_tile_kernel(TileArgs p) {
-  __shared__ __align__(16) uint16_t tile[kTile][kTile];
-  const int tid = threadIdx.x;
-  const int64_t c0 = int64_t(blockIdx.x) * kTile;
-  const int64_t r0 = int64_t(blockIdx.y) * kTile;
-  const int64_t b = blockIdx.z;
+__global__ void __launch_bounds__(kCastThreads, CastCfg<kSwiglu>::kCtasPerSm)
+mx_cast_kernel(const __grid_constant__ CUtensorMap tin, const CastArgs p) {
+  using C = CastCfg<kSwiglu>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBars);
+  uint8_t* cstage = smem + C::kOffColStage;     // COL codes: column c at c*128, 16-byte chunk k at k ^ ((c>>1)&7)
+  uint8_t* rsc = smem + C::kOffScales;          // ROW scales of the tile: [128 rows][4 blocks]
+  uint8_t* csc = rsc + 512;                     // COL scales of the tile: [128 cols][4 blocks]
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t rows = p.rows, cols = p.cols;
-  const bool do_row = p.modes & 1;
-  const bool do_col = p.modes & 2;
-  const uint16_t* in = p.in + b * rows * p.ld_in;
+  const int64_t ntiles = p.batch * p.tiles_r * p.tiles_c;
   int64_t rows_lim = rows;
   if (p.dev_rows != nullptr) rows_lim = min(rows, int64_t(*p.dev_rows));
+  const bool do_row = p.modes & 1, do_col = p.modes & 2;
 
-  // ---- load 8 chunks of 8 elements per thread (all loads first: ILP)
-  uint4 v[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int id = i * kTileThreads + tid;
-    const int64_t row = r0 + (id >> 4);
-    const int64_t col = c0 + (id & 15) * 8;
-    if (row < rows_lim && col < cols) {
-      v[i] = ld_nc_v4(in + row * p.ld_in + col);
-    } else {
-      v[i] = make_uint4(0, 0, 0, 0);
+  if (tid == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      sm100::mbar_init(sm100::smem_u32(&bars[s]), 1);                                  // full
+      sm100::mbar_init(sm100::smem_u32(&bars[C::kStages + s]), kCastConsumers / 32);  // empty
     }
+    sm100::fence_mbar_init();
   }
-  if constexpr (kSwiglu) {
-    uint4 u[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int id = i * kTileThreads + tid;
-      const int64_t row = r0 + (id >> 4);
-      const int64_t col = c0 + (id & 15) * 8;
-      u[i] = (row < rows_lim && col < cols) ? ld_nc_v4(in + row * p.ld_in + p.up_off + col)
-                                        : make_uint4(0, 0, 0, 0);
+  __syncthreads();
+
+  const int64_t per_batch = p.tiles_r * p.tiles_c;
+  if (warp == 8) {
+    // ---------------- producer
+    if (lane == 0) {
+      sm100::prefetch_tmap(&tin);
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x) {
+        const int64_t b = t / per_batch, rem = t - b * per_batch;
+        const int64_t r0 = (rem / p.tiles_c) * kTile, c0 = (rem % p.tiles_c) * kTile;
+        if (r0 >= rows_lim) continue;             // past the valid rows: never read
+        if (!sm100::mbar_wait(sm100::smem_u32(&bars[C::kStages + stage]), phase ^ 1)) {
+          raise_device_error(7);
+          break;
+        }
+        const uint32_t fb = sm100::smem_u32(&bars[stage]);
+        const uint32_t dst = sm100::smem_u32(smem + stage * C::kStageBytes);
+        sm100::mbar_arrive_expect_tx(fb, C::kStageBytes);
+        sm100::tma_load_3d(dst, &tin, fb, int(c0), int(r0), int(b));
+        if constexpr (kSwiglu) sm100::tma_load_3d(dst + kTileBytes, &tin, fb, int(p.up_off + c0), int(r0), int(b));
+        if (++stage == C::kStages) { stage = 0; phase ^= 1; }
+      }
     }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      v[i].x = swiglu_pair(v[i].x, u[i].x);
-      v[i].y = swiglu_pair(v[i].y, u[i].y);
-      v[i].z = swiglu_pair(v[i].z, u[i].z);
-      v[i].w = swiglu_pair(v[i].w, u[i].w);
-    }
+    return;
   }
 
-  // ---- ROW pass (4 consecutive lanes hold one 32-block) + park in smem
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int id = i * kTileThreads + tid;
-    const int rr = id >> 4, ch = id & 15;
-    const int64_t row = r0 + rr;
-    const int64_t col = c0 + ch * 8;
-    if (do_row) {
-      uint32_t am = absmax_bits8(v[i]);
-      am = max(am, __shfl_xor_sync(0xffffffffu, am, 1));
-      am = max(am, __shfl_xor_sync(0xffffffffu, am, 2));
-      const uint32_t byte = scale_byte_from_bits(am);
-      if (row < rows_lim && col < cols) {
-        const int64_t R = b * rows + row;
-        *reinterpret_cast<uint2*>(p.row_codes + R * cols + col) = encode8(v[i], byte);
-        if ((ch & 3) == 0) {
-          const int64_t off = p.mma_layout ? mma_scale_offset(R, col >> 5, cols)
-                                           : R * (cols >> 5) + (col >> 5);
-          p.row_scales[off] = uint8_t(byte);
+  // ---------------- consumers
+  const int ch = tid & 15, rr0 = tid >> 4;      // ROW: chunk i = row i*16 + rr0, columns ch*8..ch*8+7
+  const int cp = tid & 63, rb = tid >> 6;       // COL: columns 2cp, 2cp+1 of 32-row block rb
+  const bool plain = p.mma_layout == 0;
+  int stage = 0;
+  uint32_t phase = 0;
+  for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x) {
+    const int64_t b = t / per_batch, rem = t - b * per_batch;
+    const int64_t r0 = (rem / p.tiles_c) * kTile, c0 = (rem % p.tiles_c) * kTile;
+    if (r0 >= rows_lim) continue;
+    if (!__all_sync(0xffffffffu, sm100::mbar_wait(sm100::smem_u32(&bars[stage]), phase))) {
+      raise_device_error(7);
+      break;
+    }
+    uint8_t* tile = smem + stage * C::kStageBytes;
+    const int vrows = int(min(int64_t(kTile), rows_lim - r0));   // valid rows of the tile (multiple of 32 for COL)
+    const int vcols = int(min(int64_t(kTile), cols - c0));       // valid columns (multiple of 32)
+
+    // ---- ROW pass (and SwiGLU): codes straight to global, scales to shared
+    if (do_row || kSwiglu) {
+      const int64_t col = c0 + ch * 8;
+      const int64_t Rb = b * rows + r0 + rr0;                    // matrix row of chunk 0
+      uint8_t* rcode = p.row_codes + Rb * cols + col;            // advances 16 rows per chunk
+#pragma unroll 2
+      for (int i = 0; i < 8; ++i) {
+        const int rr = i * 16 + rr0;
+        uint8_t* srow = tile + rr * 256 + ch * 16;
+        uint4 v = *reinterpret_cast<const uint4*>(srow);
+        if constexpr (kSwiglu) {
+          const uint4 u = *reinterpret_cast<const uint4*>(srow + kTileBytes);
+          v.x = swiglu_pair(v.x, u.x);
+          v.y = swiglu_pair(v.y, u.y);
+          v.z = swiglu_pair(v.z, u.z);
+          v.w = swiglu_pair(v.w, u.w);
+          *reinterpret_cast<uint4*>(srow) = v;
+        }
+        if (do_row) {
+          uint32_t byte;
+          const uint2 q = row_quant8(v, &byte);
+          if (rr < vrows && ch * 8 < vcols) {
+            *reinterpret_cast<uint2*>(rcode + int64_t(i) * 16 * cols) = q;
+            if ((ch & 3) == 0) rsc[rr * 4 + (ch >> 2)] = uint8_t(byte);
+          }
         }
       }
     }
-    if (do_col) *reinterpret_cast<uint4*>(&tile[rr][ch * 8]) = v[i];
-  }
-  if (!do_col) return;
-  __syncthreads();
+    if (kSwiglu && do_col) sm100::named_bar_sync(1, kCastConsumers);   // h parked for the COL pass
 
-  // ---- COL pass: one thread per (column, 32-row block)
-  const int64_t nrb = rows >> 5;
+    // ---- COL pass: codes into the shared staging tile
+    if (do_col) {
+      if (rb * 32 < vrows && 2 * cp < vcols) {
+        uint32_t w[32];
+        const uint8_t* src = tile + (rb * 32) * 256 + cp * 4;
 #pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    const int task = i * kTileThreads + tid;
-    const int c = task & 127, rb = task >> 7;
-    const int64_t col = c0 + c;
-    const int64_t rowb = r0 + rb * 32;
-    if (col >= cols || rowb >= rows_lim) continue;
-    uint4 w[4];
-    uint32_t* wp = reinterpret_cast<uint32_t*>(w);
+        for (int j = 0; j < 32; ++j) w[j] = *reinterpret_cast<const uint32_t*>(src + j * 256);
 #pragma unroll
-    for (int j = 0; j < 16; ++j)
-      wp[j] = uint32_t(tile[rb * 32 + 2 * j][c]) | (uint32_t(tile[rb * 32 + 2 * j + 1][c]) << 16);
-    uint32_t am = max(max(absmax_bits8(w[0]), absmax_bits8(w[1])),
-                      max(absmax_bits8(w[2]), absmax_bits8(w[3])));
-    const uint32_t byte = scale_byte_from_bits(am);
-    const int64_t R = b * cols + col;
-    uint2 q0 = encode8(w[0], byte), q1 = encode8(w[1], byte);
-    uint2 q2 = encode8(w[2], byte), q3 = encode8(w[3], byte);
-    uint8_t* dst = p.col_codes + R * rows + rowb;
-    reinterpret_cast<uint4*>(dst)[0] = make_uint4(q0.x, q0.y, q1.x, q1.y);
-    reinterpret_cast<uint4*>(dst)[1] = make_uint4(q2.x, q2.y, q3.x, q3.y);
-    const int64_t off = p.mma_layout ? mma_scale_offset(R, rowb >> 5, rows) : R * nrb + (rowb >> 5);
-    p.col_scales[off] = uint8_t(byte);
+        for (int k = 0; k < 2; ++k) {
+          uint4 q[2];
+          const uint32_t byte = k ? col_quant32<true>(w, q) : col_quant32<false>(w, q);
+          const int c = 2 * cp + k;
+          uint8_t* dst = cstage + c * 128;
+          const int swz = cp & 7;
+          *reinterpret_cast<uint4*>(dst + (((2 * rb) ^ swz) << 4)) = q[0];
+          *reinterpret_cast<uint4*>(dst + (((2 * rb + 1) ^ swz) << 4)) = q[1];
+          csc[c * 4 + rb] = uint8_t(byte);
+        }
+      }
+    }
+    // the input tile is no longer read: hand it back to the producer
+    __syncwarp();
+    if (lane == 0) sm100::mbar_arrive(sm100::smem_u32(&bars[C::kStages + stage]));
+    if (++stage == C::kStages) { stage = 0; phase ^= 1; }
+    sm100::named_bar_sync(1, kCastConsumers);                          // COL codes and scales staged
+
+    // ---- write-out: whole 128-byte rows of COL codes, 16-byte scale stores
+    if (do_col) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int qd = u * kCastConsumers + tid;                // 16-byte chunk id of the 16 KB tile
+        const int c = qd >> 3, k = qd & 7;                      // output row (input column) c, chunk k
+        if (c < vcols && k * 16 < vrows) {
+          const uint4 v = *reinterpret_cast<const uint4*>(cstage + c * 128 + ((k ^ ((c >> 1) & 7)) << 4));
+          *reinterpret_cast<uint4*>(p.col_codes + (b * cols + c0 + c) * rows + r0 + k * 16) = v;
+        }
+      }
+    }
+    if (do_row) {
+      if (!plain) {
+        // the tile's 128 rows x 4 blocks are exactly one 512-byte MMA atom:
+        // atom byte (r%32)*16 + (r/32)*4 + kb  <-  staged byte r*4 + kb
+        if (tid < 32 && vrows == kTile && vcols == kTile) {
+          uint32_t wv[4];
+#pragma unroll
+          for (int g = 0; g < 4; ++g) wv[g] = *reinterpret_cast<const uint32_t*>(rsc + (g * 32 + tid) * 4);
+          const int64_t atom = ((b * rows + r0) >> 7) * (cols >> 7) + (c0 >> 7);
+          *reinterpret_cast<uint4*>(p.row_scales + atom * 512 + tid * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+        }
+      } else if (tid < vrows) {
+        const int nb = vcols >> 5;
+        const int64_t R = b * rows + r0 + tid;
+        uint8_t* d = p.row_scales + R * (cols >> 5) + (c0 >> 5);
+        if (nb == 4 && (reinterpret_cast<uintptr_t>(d) & 3) == 0)
+          *reinterpret_cast<uint32_t*>(d) = *reinterpret_cast<const uint32_t*>(rsc + tid * 4);
+        else
+          for (int kb = 0; kb < nb; ++kb) d[kb] = rsc[tid * 4 + kb];
+      }
+    }
+    if (do_col) {
+      if (!plain) {
+        if (tid >= 64 && tid < 96 && vrows == kTile && vcols == kTile) {
+          const int l = tid - 64;
+          uint32_t wv[4];
+#pragma unroll
+          for (int g = 0; g < 4; ++g) wv[g] = *reinterpret_cast<const uint32_t*>(csc + (g * 32 + l) * 4);
+          const int64_t atom = ((b * cols + c0) >> 7) * (rows >> 7) + (r0 >> 7);
+          *reinterpret_cast<uint4*>(p.col_scales + atom * 512 + l * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+        }
+      } else if (tid >= 128 && tid - 128 < vcols) {
+        const int c = tid - 128;
+        const int nb = vrows >> 5;
+        const int64_t R = b * cols + c0 + c;
+        uint8_t* d = p.col_scales + R * (rows >> 5) + (r0 >> 5);
+        if (nb == 4 && (reinterpret_cast<uintptr_t>(d) & 3) == 0)
+          *reinterpret_cast<uint32_t*>(d) = *reinterpret_cast<const uint32_t*>(csc + c * 4);
+        else
+          for (int k = 0; k < nb; ++k) d[k] = csc[c * 4 + k];
+      }
+    }
+    // staging buffers are rewritten by the next tile
+    sm100::named_bar_sync(1, kCastConsumers);
   }
 }
 

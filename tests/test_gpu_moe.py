@@ -123,3 +123,25 @@ def test_dsv3_16b_full_size_sampled_experts():
         _compare_expert(e, lo, hi, rf, rb, y, saved, dx, dw13, dw2, M, F, D)
     for e in zero:
         assert (bf16_np(dw13[e]) == 0).all() and (bf16_np(dw2[e]) == 0).all()
+
+
+def test_prequantized_weights_path_matches_bf16_weight_composites():
+    """mxmoe_quantize_weights + the _q composites give the same bits as the
+    composites that cast the bf16 weights themselves."""
+    inp = synth.make_moe_inputs("tiny", 4)
+    y, saved, dx, dw13, dw2 = _run(inp)
+    off = torch.from_numpy(inp.routing.offsets).to(DEV)
+    pad = inp.spec.pad
+    x, w13, w2, dy = (t.to(DEV) for t in (inp.x, inp.w13, inp.w2, inp.dy))
+    qw = mxk.mxmoe_quantize_weights(w13, w2)
+    yq, sq = mxk.moe_mlp_fwd_q(x, qw, off, pad)
+    dxq, dw13q, dw2q = mxk.moe_mlp_bwd_q(dy, qw, off, sq, pad)
+    torch.cuda.synchronize()
+    for a, b in ((y, yq), (dx, dxq), (dw13, dw13q), (dw2, dw2q), (saved["h13"], sq["h13"])):
+        assert torch.equal(a, b)
+    # the dual weight cast equals the separate ROW and COL casts
+    E, F2, D = w13.shape
+    r = mxk.mxfp8_quantize(w13, mxk.ROW | mxk.COL, mxk.MMA)
+    assert torch.equal(r["row_codes"].reshape(-1), qw["w13_codes"].reshape(-1))
+    assert torch.equal(r["col_codes"].reshape(-1), qw["w13t_codes"].reshape(-1))
+    assert torch.equal(r["row_scales"], qw["w13_scales"]) and torch.equal(r["col_scales"], qw["w13t_scales"])
