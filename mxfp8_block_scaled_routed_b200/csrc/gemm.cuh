@@ -58,19 +58,25 @@ struct Params {
   uint8_t* col_scales;
 };
 
-template <int kMode, int kEpi, int BN>
+// kPair: the CTA pair (cluster of 2, cta_group::2) computes a 256 x BN tile;
+// each CTA holds 128 rows of A, half of the BN rows of B and its own
+// 128 x BN accumulator.
+template <int kMode, int kEpi, int BN, bool kPair>
 struct Cfg {
   static constexpr int BM = 128, BK = 128;
   static constexpr int kAcc = (BN == 256) ? 1 : 2;
-  static constexpr int kStages = (BN == 256) ? 4 : 6;
+  static constexpr int kBBox = kPair ? BN / 256 : BN / 128;   // 128-row B boxes loaded per CTA and stage
   static constexpr int A_BYTES = BM * BK;
-  static constexpr int B_BYTES = BN * BK;
+  static constexpr int B_BYTES = kBBox * 128 * BK;
   static constexpr int SFA_BYTES = 512;
-  static constexpr int SFB_BYTES = (BN / 128) * 512;
+  static constexpr int SFB_BYTES = (BN / 128) * 512;          // scales of all BN rows of B
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+  static constexpr int kStages = kPair ? 6 : ((BN == 256) ? 4 : 6);
   static constexpr int SF_COLS = 4 + BN / 32;           // TMEM columns for one SF buffer
   static constexpr int ACC_COLS = kAcc * BN;
   static constexpr int TMEM_COLS = 512;
   static_assert(ACC_COLS + 2 * SF_COLS <= TMEM_COLS, "TMEM budget");
+  static_assert(!kPair || BN == 256, "CTA pairs use 256-wide tiles");
   // shared memory map (offsets from a 1024-aligned base)
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + kStages * A_BYTES;
@@ -93,31 +99,34 @@ struct Cfg {
 struct Tile {
   int e;
   int nk;           // K blocks of 128
-  int64_t a_row;    // first A row of the tile
-  int64_t b_row0;   // first B row of box 0
-  int64_t b_row1;   // first B row of box 1 (BN == 256)
+  int64_t a_row;    // first A row loaded by this CTA
+  int64_t b_row0;   // first B row of the tile's first 128-row box (scales)
+  int64_t b_row1;   // first B row of the second box (BN == 256)
+  int64_t b_mine;   // CTA pair: the B box this CTA loads
   int64_t k0;       // first K element
-  int64_t out_r0;   // first output row
+  int64_t out_r0;   // first output row of this CTA
   int64_t out_c0;   // first output column (SwiGLU: first f)
 };
 
-template <int kMode, int kEpi, int BN>
+template <int kMode, int kEpi, int BN, bool kPair>
 __device__ __forceinline__ int64_t num_tiles(const Params& p, const int32_t* offs) {
+  constexpr int PM = kPair ? 256 : 128;
   if constexpr (kMode == kRaggedM) {
     const int64_t nt = (kEpi == kEpiSwiGLU) ? p.F / 128 : p.n_out / BN;
-    return (int64_t(offs[p.E]) / 128) * nt;
+    return (int64_t(offs[p.E]) / PM) * nt;
   } else {
-    return int64_t(p.E) * (p.rows_a / 128) * (p.n_out / BN);
+    return int64_t(p.E) * (p.rows_a / PM) * (p.n_out / BN);
   }
 }
 
-template <int kMode, int kEpi, int BN>
-__device__ __forceinline__ Tile get_tile(const Params& p, const int32_t* offs, int64_t t) {
+template <int kMode, int kEpi, int BN, bool kPair>
+__device__ __forceinline__ Tile get_tile(const Params& p, const int32_t* offs, int64_t t, int rank) {
+  constexpr int PM = kPair ? 256 : 128;
   Tile T;
   if constexpr (kMode == kRaggedM) {
     const int64_t nt = (kEpi == kEpiSwiGLU) ? p.F / 128 : p.n_out / BN;
     const int64_t mt = t / nt, ntile = t % nt;
-    const int64_t m0 = mt * 128;
+    const int64_t m0 = mt * PM;
     int lo = 0, hi = p.E;  // last e with offs[e] <= m0
     while (hi - lo > 1) {
       const int mid = (lo + hi) >> 1;
@@ -126,8 +135,8 @@ __device__ __forceinline__ Tile get_tile(const Params& p, const int32_t* offs, i
     T.e = lo;
     T.nk = int(p.kext / 128);
     T.k0 = 0;
-    T.a_row = m0;
-    T.out_r0 = m0;
+    T.a_row = m0 + rank * 128;
+    T.out_r0 = T.a_row;
     if constexpr (kEpi == kEpiSwiGLU) {
       const int64_t f0 = ntile * 128;
       T.b_row0 = int64_t(T.e) * 2 * p.F + f0;          // gate rows
@@ -139,18 +148,19 @@ __device__ __forceinline__ Tile get_tile(const Params& p, const int32_t* offs, i
       T.out_c0 = ntile * BN;
     }
   } else {
-    const int64_t nn = p.rows_a / 128, nj = p.n_out / BN;
+    const int64_t nn = p.rows_a / PM, nj = p.n_out / BN;
     const int64_t e = t / (nn * nj), rem = t % (nn * nj);
     const int64_t nt = rem / nj, jt = rem % nj;
     T.e = int(e);
     T.k0 = offs[e];
     T.nk = int((offs[e + 1] - offs[e]) / 128);
-    T.a_row = nt * 128;
+    T.a_row = nt * PM + rank * 128;
     T.b_row0 = jt * BN;
     T.b_row1 = jt * BN + 128;
-    T.out_r0 = nt * 128;
+    T.out_r0 = T.a_row;
     T.out_c0 = jt * BN;
   }
+  T.b_mine = rank ? T.b_row1 : T.b_row0;
   return T;
 }
 
@@ -271,15 +281,20 @@ __device__ __forceinline__ void drain32_bf16(uint32_t taddr, uint32_t* w) {
 }
 
 // ---------------------------------------------------------------- the kernel
-template <int kMode, int kEpi, int BN>
+template <int kMode, int kEpi, int BN, bool kPair>
 __global__ void __launch_bounds__(384, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                    const __grid_constant__ CUtensorMap tmap_sa, const __grid_constant__ CUtensorMap tmap_sb,
                     const Params p) {
-  using C = Cfg<kMode, kEpi, BN>;
+  using C = Cfg<kMode, kEpi, BN, kPair>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // CTA pairs: the cluster is (2,1,1), so the rank in the pair is blockIdx.x & 1
+  const int rank = kPair ? int(cluster_ctarank()) : 0;
+  const int64_t unit = kPair ? (blockIdx.x >> 1) : blockIdx.x;       // tile-walker index of this CTA / pair
+  const int64_t nunits = kPair ? (gridDim.x >> 1) : gridDim.x;
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   auto full_bar = [&](int s) { return smem_u32(&bars[s]); };
@@ -289,7 +304,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
   volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(smem + C::OFF_MISC);
   int32_t* offs = reinterpret_cast<int32_t*>(smem + C::OFF_OFFS);
 
-  // ---- offsets into shared memory + validation (every CTA checks)
+  // ---- offsets into shared memory + validation (every CTA checks; both
+  // CTAs of a pair see the same table, so they take the same decision)
   bool bad = p.E > C::MAX_E;
   if (!bad) {
     for (int i = threadIdx.x; i <= p.E; i += blockDim.x) offs[i] = p.offsets[i];
@@ -311,96 +327,138 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmap_a);
     prefetch_tmap(&tmap_b);
+    if constexpr (kPair) {
+      prefetch_tmap(&tmap_sa);
+      prefetch_tmap(&tmap_sb);
+    }
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(full_bar(s), 1);
       mbar_init(empty_bar(s), 1);
     }
     for (int a = 0; a < C::kAcc; ++a) {
       mbar_init(tfull_bar(a), 1);
-      mbar_init(tempty_bar(a), 32 * C::EPI_WARPS);
+      mbar_init(tempty_bar(a), (kPair ? 2 : 1) * C::EPI_WARPS); // one arrival per epilogue warp
     }
     misc[1] = 0;  // abort flag
     fence_mbar_init();
   }
   if (warp == 2) {
-    tmem_alloc(smem_u32(const_cast<uint32_t*>(misc)), C::TMEM_COLS);
-    tmem_relinquish();
+    if constexpr (kPair) {
+      tmem_alloc_pair(smem_u32(const_cast<uint32_t*>(misc)), C::TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(const_cast<uint32_t*>(misc)), C::TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if constexpr (kPair) cluster_sync_all(); else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = misc[0];
-  const int64_t ntiles = num_tiles<kMode, kEpi, BN>(p, offs);
+  const int64_t ntiles = num_tiles<kMode, kEpi, BN, kPair>(p, offs);
 
   if (warp == 0) {
-    // ================= producer =================
+    // ================= producer (every CTA loads its own operand halves)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-        const Tile T = get_tile<kMode, kEpi, BN>(p, offs, t);
+      for (int64_t t = unit; t < ntiles && ok; t += nunits) {
+        const Tile T = get_tile<kMode, kEpi, BN, kPair>(p, offs, t, rank);
         for (int kb = 0; kb < T.nk; ++kb) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1)) { ok = false; break; }
-          const uint32_t fb = full_bar(stage);
-          mbar_arrive_expect_tx(fb, C::A_BYTES + C::B_BYTES + C::SFA_BYTES + C::SFB_BYTES);
           const int64_t k = T.k0 + int64_t(kb) * 128;
-          tma_load_2d(sbase + C::OFF_A + stage * C::A_BYTES, &tmap_a, fb, int(k), int(T.a_row));
-          tma_load_2d(sbase + C::OFF_B + stage * C::B_BYTES, &tmap_b, fb, int(k), int(T.b_row0));
-          if constexpr (BN == 256)
-            tma_load_2d(sbase + C::OFF_B + stage * C::B_BYTES + 16384, &tmap_b, fb, int(k), int(T.b_row1));
           const int64_t katoms = p.kext / 128, kat = k / 128;
-          bulk_load(sbase + C::OFF_SFA + stage * C::SFA_BYTES,
-                    p.a_scales + ((T.a_row / 128) * katoms + kat) * 512, 512, fb);
-          bulk_load(sbase + C::OFF_SFB + stage * C::SFB_BYTES,
-                    p.b_scales + ((T.b_row0 / 128) * katoms + kat) * 512, 512, fb);
-          if constexpr (BN == 256)
-            bulk_load(sbase + C::OFF_SFB + stage * C::SFB_BYTES + 512,
-                      p.b_scales + ((T.b_row1 / 128) * katoms + kat) * 512, 512, fb);
+          if constexpr (kPair) {
+            // both CTAs' loads are credited to the even CTA's full barrier,
+            // which expects the bytes of the whole pair
+            const uint32_t fb = mapa_cluster(full_bar(stage), 0);
+            if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), 2 * C::STAGE_BYTES);
+            tma_load_2d_pair(sbase + C::OFF_A + stage * C::A_BYTES, &tmap_a, fb, int(k), int(T.a_row));
+            tma_load_2d_pair(sbase + C::OFF_B + stage * C::B_BYTES, &tmap_b, fb, int(k), int(T.b_mine));
+            // scale atoms: a 512-byte atom is two 256-byte rows of the scale map
+            tma_load_2d_pair(sbase + C::OFF_SFA + stage * C::SFA_BYTES, &tmap_sa, fb, 0,
+                             int(((T.a_row / 128) * katoms + kat) * 2));
+            tma_load_2d_pair(sbase + C::OFF_SFB + stage * C::SFB_BYTES, &tmap_sb, fb, 0,
+                             int(((T.b_row0 / 128) * katoms + kat) * 2));
+            tma_load_2d_pair(sbase + C::OFF_SFB + stage * C::SFB_BYTES + 512, &tmap_sb, fb, 0,
+                             int(((T.b_row1 / 128) * katoms + kat) * 2));
+          } else {
+            const uint32_t fb = full_bar(stage);
+            mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
+            tma_load_2d(sbase + C::OFF_A + stage * C::A_BYTES, &tmap_a, fb, int(k), int(T.a_row));
+            tma_load_2d(sbase + C::OFF_B + stage * C::B_BYTES, &tmap_b, fb, int(k), int(T.b_row0));
+            if constexpr (BN == 256)
+              tma_load_2d(sbase + C::OFF_B + stage * C::B_BYTES + 16384, &tmap_b, fb, int(k), int(T.b_row1));
+            bulk_load(sbase + C::OFF_SFA + stage * C::SFA_BYTES,
+                      p.a_scales + ((T.a_row / 128) * katoms + kat) * 512, 512, fb);
+            bulk_load(sbase + C::OFF_SFB + stage * C::SFB_BYTES,
+                      p.b_scales + ((T.b_row0 / 128) * katoms + kat) * 512, 512, fb);
+            if constexpr (BN == 256)
+              bulk_load(sbase + C::OFF_SFB + stage * C::SFB_BYTES + 512,
+                        p.b_scales + ((T.b_row1 / 128) * katoms + kat) * 512, 512, fb);
+          }
           if (++stage == C::kStages) { stage = 0; phase ^= 1; }
         }
       }
       if (!ok) { misc[1] = 1; raise_device_error(kErrTimeout); }
     }
   } else if (warp == 1) {
-    // ================= MMA issuer =================
-    if (lane == 0) {
+    // ================= MMA issuer (the even CTA of a pair issues for both)
+    if (lane == 0 && rank == 0) {
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
       uint32_t sfbuf = 0;
       bool ok = true;
       const uint32_t sf_col0 = C::ACC_COLS;
-      for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-        const Tile T = get_tile<kMode, kEpi, BN>(p, offs, t);
+      constexpr uint32_t kMmaM = kPair ? 256 : 128;
+      for (int64_t t = unit; t < ntiles && ok; t += nunits) {
+        const Tile T = get_tile<kMode, kEpi, BN, kPair>(p, offs, t, 0);
         if (T.nk == 0) continue;
-        if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1)) { ok = false; break; }
+        if (!(kPair ? mbar_wait_cluster(tempty_bar(acc), acc_phase ^ 1) : mbar_wait(tempty_bar(acc), acc_phase ^ 1))) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
         for (int kb = 0; kb < T.nk; ++kb) {
-          if (!mbar_wait(full_bar(stage), phase)) { ok = false; break; }
+          if (!(kPair ? mbar_wait_cluster(full_bar(stage), phase) : mbar_wait(full_bar(stage), phase))) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
           const uint32_t sfa_t = tmem_base + sf_col0 + sfbuf * C::SF_COLS;
           const uint32_t sfb_t = sfa_t + 4;
           const uint32_t sfa_s = sbase + C::OFF_SFA + stage * C::SFA_BYTES;
           const uint32_t sfb_s = sbase + C::OFF_SFB + stage * C::SFB_BYTES;
-          utccp_32x128b_warpx4(sfa_t, smem_desc(sfa_s, 0, 128, 0));
+          if constexpr (kPair) {
+            utccp_32x128b_warpx4_pair(sfa_t, smem_desc(sfa_s, 0, 128, 0));
 #pragma unroll
-          for (int j = 0; j < BN / 128; ++j)
-            utccp_32x128b_warpx4(sfb_t + 4 * j, smem_desc(sfb_s + 512 * j, 0, 128, 0));
+            for (int j = 0; j < BN / 128; ++j)
+              utccp_32x128b_warpx4_pair(sfb_t + 4 * j, smem_desc(sfb_s + 512 * j, 0, 128, 0));
+          } else {
+            utccp_32x128b_warpx4(sfa_t, smem_desc(sfa_s, 0, 128, 0));
+#pragma unroll
+            for (int j = 0; j < BN / 128; ++j)
+              utccp_32x128b_warpx4(sfb_t + 4 * j, smem_desc(sfb_s + 512 * j, 0, 128, 0));
+          }
           const uint32_t a_s = sbase + C::OFF_A + stage * C::A_BYTES;
           const uint32_t b_s = sbase + C::OFF_B + stage * C::B_BYTES;
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
             const uint64_t ad = smem_desc(a_s + k * 32, 0, 1024, 2);
             const uint64_t bd = smem_desc(b_s + k * 32, 0, 1024, 2);
-            mma_mxf8(d_tmem, ad, bd, mxf8_idesc(128, BN, k), sfa_t, sfb_t, (kb | k) != 0);
+            if constexpr (kPair)
+              mma_mxf8_pair(d_tmem, ad, bd, mxf8_idesc(kMmaM, BN, k), sfa_t, sfb_t, (kb | k) != 0);
+            else
+              mma_mxf8(d_tmem, ad, bd, mxf8_idesc(kMmaM, BN, k), sfa_t, sfb_t, (kb | k) != 0);
           }
-          mma_commit(empty_bar(stage));
+          if constexpr (kPair) mma_commit_pair(empty_bar(stage)); else mma_commit(empty_bar(stage));
           sfbuf ^= 1;
           if (++stage == C::kStages) { stage = 0; phase ^= 1; }
         }
         if (!ok) break;
-        mma_commit(tfull_bar(acc));
+        if constexpr (kPair) mma_commit_pair(tfull_bar(acc)); else mma_commit(tfull_bar(acc));
         if (++acc == C::kAcc) { acc = 0; acc_phase ^= 1; }
       }
       if (!ok) { misc[1] = 1; raise_device_error(kErrTimeout); }
@@ -418,8 +476,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
     constexpr int kChunks = kHalf / 32;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x) {
-      const Tile T = get_tile<kMode, kEpi, BN>(p, offs, t);
+    for (int64_t t = unit; t < ntiles; t += nunits) {
+      const Tile T = get_tile<kMode, kEpi, BN, kPair>(p, offs, t, rank);
       const int64_t row0 = T.out_r0 + q * 32;              // first row of this warp's 32-row slab
       if constexpr (kMode == kRaggedK) {
         if (T.nk == 0) {
@@ -450,7 +508,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
         for (int c = 0; c < kChunks; ++c) drain32_bf16(t_row + 128 + h * kHalf + 32 * c, vb + 16 * c);
       }
       tc_fence_before();
-      mbar_arrive(tempty_bar(acc));
+      __syncwarp();
+      if (lane == 0) {
+        if constexpr (kPair) mbar_arrive_remote(tempty_bar(acc), 0); else mbar_arrive(tempty_bar(acc));
+      }
       if (++acc == C::kAcc) { acc = 0; acc_phase ^= 1; }
 
       if constexpr (kEpi == kEpiBF16) {
@@ -515,12 +576,14 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
     }
   }
 
-  // ---- teardown: every role has left its loop (all waits are bounded)
+  // ---- teardown: every role has left its loop (all waits are bounded); in a
+  // pair, neither CTA frees its TMEM or exits while the other may still
+  // arrive on its barriers or run MMAs into its TMEM
   tc_fence_before();
-  __syncthreads();
+  if constexpr (kPair) cluster_sync_all(); else __syncthreads();
   if (warp == 2) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, C::TMEM_COLS);
+    if constexpr (kPair) tmem_dealloc_pair(tmem_base, C::TMEM_COLS); else tmem_dealloc(tmem_base, C::TMEM_COLS);
   }
 }
 

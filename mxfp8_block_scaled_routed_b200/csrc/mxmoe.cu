@@ -23,6 +23,13 @@ using namespace mxmoe;
 #ifndef MXMOE_WGRAD_BN
 #define MXMOE_WGRAD_BN 256
 #endif
+// 256 x 256 tiles on CTA pairs (cta_group::2) wherever the shapes allow.
+#ifndef MXMOE_USE_PAIRS
+#define MXMOE_USE_PAIRS 1
+#endif
+#ifndef MXMOE_WGRAD_PAIRS
+#define MXMOE_WGRAD_PAIRS 0
+#endif
 
 namespace {
 
@@ -171,14 +178,30 @@ int launch_cast(const void* in, int64_t batch, int64_t rows, int64_t cols, int m
   return MXMOE_OK;
 }
 
+// Scale atoms of an MMA-layout scale buffer of `bytes` bytes as a 2-D uint8
+// map [bytes/256, 256] with 256 x 2 boxes (one 512-byte atom per box).
+int make_scale_map(CUtensorMap* map, const uint8_t* base, int64_t bytes) {
+  EncodeTiledFn enc;
+  MX_TRY(get_encode(&enc));
+  cuuint64_t dims[2] = {256, cuuint64_t(bytes / 256)};
+  cuuint64_t strides[1] = {256};
+  cuuint32_t box[2] = {256, 2};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MXMOE_ERR_CUDA, "cuTensorMapEncodeTiled (scales) failed (%d)", int(r));
+  return MXMOE_OK;
+}
+
 // ---------------------------------------------------------------- GEMM launch
-template <int kMode, int kEpi, int BN>
+template <int kMode, int kEpi, int BN, bool kPair>
 int launch_gemm(const uint8_t* a, int64_t a_rows, const uint8_t* b, int64_t b_rows, gemm::Params p,
                 int64_t max_tiles, cudaStream_t stream, int attr_bit) {
-  using C = gemm::Cfg<kMode, kEpi, BN>;
+  using C = gemm::Cfg<kMode, kEpi, BN, kPair>;
   DevInfo* d;
   MX_TRY(device_info(&d));
-  auto kern = gemm::grouped_gemm_kernel<kMode, kEpi, BN>;
+  auto kern = gemm::grouped_gemm_kernel<kMode, kEpi, BN, kPair>;
   if (!(d->attr_set & (1u << attr_bit))) {
     MX_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES),
                   "cudaFuncSetAttribute");
@@ -186,12 +209,43 @@ int launch_gemm(const uint8_t* a, int64_t a_rows, const uint8_t* b, int64_t b_ro
     d->attr_set |= (1u << attr_bit);
   }
   if (p.E > C::MAX_E) return fail(MXMOE_ERR_SHAPE, "E=%d exceeds the supported maximum %d", p.E, C::MAX_E);
-  CUtensorMap ma, mb;
+  CUtensorMap ma, mb, msa, msb;
   MX_TRY(make_operand_map(&ma, a, a_rows, p.kext));
   MX_TRY(make_operand_map(&mb, b, b_rows, p.kext));
+  if constexpr (kPair) {
+    MX_TRY(make_scale_map(&msa, p.a_scales, a_rows * p.kext / 32));
+    MX_TRY(make_scale_map(&msb, p.b_scales, b_rows * p.kext / 32));
+  } else {
+    msa = ma;   // unused by the single-CTA kernel
+    msb = mb;
+  }
   if (max_tiles <= 0) return MXMOE_OK;
-  const int grid = int(max_tiles < d->sms ? max_tiles : d->sms);
-  kern<<<grid, 384, C::SMEM_BYTES, stream>>>(ma, mb, p);
+  if constexpr (!kPair) {
+    const int grid = int(max_tiles < d->sms ? max_tiles : d->sms);
+    kern<<<grid, 384, C::SMEM_BYTES, stream>>>(ma, mb, msa, msb, p);
+  } else {
+    // clusters of two CTAs, one pair per two SMs (as many as can be resident)
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.blockDim = dim3(384, 1, 1);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int pairs = d->sms / 2;
+    cfg.gridDim = dim3(unsigned(2 * pairs), 1, 1);
+    int active = 0;
+    if (cudaOccupancyMaxActiveClusters(&active, kern, &cfg) == cudaSuccess && active > 0 && active < pairs)
+      pairs = active;
+    cudaGetLastError();
+    if (max_tiles < pairs) pairs = int(max_tiles);
+    cfg.gridDim = dim3(unsigned(2 * pairs), 1, 1);
+    MX_CHECK_CUDA(cudaLaunchKernelEx(&cfg, kern, ma, mb, msa, msb, p), "grouped GEMM (CTA pair) launch");
+  }
   MX_CHECK_CUDA(cudaGetLastError(), "grouped GEMM launch");
   return MXMOE_OK;
 }
@@ -280,11 +334,14 @@ int gemm_ragged_m(const uint8_t* a, const uint8_t* as, int64_t M, int64_t K, con
   p.a_scales = as;
   p.b_scales = ws;
   p.out = static_cast<uint16_t*>(out);
+  if (MXMOE_USE_PAIRS && N % 256 == 0 && pad % 256 == 0)
+    return launch_gemm<gemm::kRaggedM, gemm::kEpiBF16, 256, true>(a, M, w, int64_t(E) * N, p,
+                                                                  (M / 256) * (N / 256), stream, 9);
   if (N % 256 == 0)
-    return launch_gemm<gemm::kRaggedM, gemm::kEpiBF16, 256>(a, M, w, int64_t(E) * N, p, (M / 128) * (N / 256),
-                                                            stream, 0);
-  return launch_gemm<gemm::kRaggedM, gemm::kEpiBF16, 128>(a, M, w, int64_t(E) * N, p, (M / 128) * (N / 128),
-                                                          stream, 1);
+    return launch_gemm<gemm::kRaggedM, gemm::kEpiBF16, 256, false>(a, M, w, int64_t(E) * N, p,
+                                                                   (M / 128) * (N / 256), stream, 0);
+  return launch_gemm<gemm::kRaggedM, gemm::kEpiBF16, 128, false>(a, M, w, int64_t(E) * N, p, (M / 128) * (N / 128),
+                                                                 stream, 1);
 }
 
 int gemm_ragged_k(const uint8_t* gt, const uint8_t* gs, int64_t N, const uint8_t* xt, const uint8_t* xs,
@@ -300,11 +357,16 @@ int gemm_ragged_k(const uint8_t* gt, const uint8_t* gs, int64_t N, const uint8_t
   p.a_scales = gs;
   p.b_scales = xs;
   p.out = static_cast<uint16_t*>(dw);
+  // (CTA pairs measured slower here: experts' short K leave little mainloop
+  // to hide the pair's per-tile accumulator hand-off)
+  if (MXMOE_WGRAD_PAIRS && Kx % 256 == 0 && N % 256 == 0)
+    return launch_gemm<gemm::kRaggedK, gemm::kEpiBF16, 256, true>(gt, N, xt, Kx, p,
+                                                                  int64_t(E) * (N / 256) * (Kx / 256), stream, 10);
   if (Kx % 256 == 0 && MXMOE_WGRAD_BN == 256)
-    return launch_gemm<gemm::kRaggedK, gemm::kEpiBF16, 256>(gt, N, xt, Kx, p, int64_t(E) * (N / 128) * (Kx / 256),
-                                                            stream, 2);
-  return launch_gemm<gemm::kRaggedK, gemm::kEpiBF16, 128>(gt, N, xt, Kx, p, int64_t(E) * (N / 128) * (Kx / 128),
-                                                          stream, 3);
+    return launch_gemm<gemm::kRaggedK, gemm::kEpiBF16, 256, false>(gt, N, xt, Kx, p,
+                                                                   int64_t(E) * (N / 128) * (Kx / 256), stream, 2);
+  return launch_gemm<gemm::kRaggedK, gemm::kEpiBF16, 128, false>(gt, N, xt, Kx, p,
+                                                                 int64_t(E) * (N / 128) * (Kx / 128), stream, 3);
 }
 
 int gemm_swiglu(const uint8_t* a, const uint8_t* as, int64_t M, int64_t K, const uint8_t* w13, const uint8_t* ws,
@@ -326,8 +388,11 @@ int gemm_swiglu(const uint8_t* a, const uint8_t* as, int64_t M, int64_t K, const
   p.row_scales = hrs;
   p.col_codes = hcc;
   p.col_scales = hcs;
-  return launch_gemm<gemm::kRaggedM, gemm::kEpiSwiGLU, 256>(a, M, w13, int64_t(E) * 2 * F, p, (M / 128) * (F / 128),
-                                                            stream, 4);
+  if (MXMOE_USE_PAIRS && pad % 256 == 0)
+    return launch_gemm<gemm::kRaggedM, gemm::kEpiSwiGLU, 256, true>(a, M, w13, int64_t(E) * 2 * F, p,
+                                                                    (M / 256) * (F / 128), stream, 11);
+  return launch_gemm<gemm::kRaggedM, gemm::kEpiSwiGLU, 256, false>(a, M, w13, int64_t(E) * 2 * F, p,
+                                                                   (M / 128) * (F / 128), stream, 4);
 }
 
 int gemm_dswiglu(const uint8_t* dy, const uint8_t* ds, int64_t M, int64_t D, const uint8_t* w2t,
@@ -349,11 +414,14 @@ int gemm_dswiglu(const uint8_t* dy, const uint8_t* ds, int64_t M, int64_t D, con
   p.row_scales = grs;
   p.col_codes = gcc;
   p.col_scales = gcs;
+  if (MXMOE_USE_PAIRS && F % 256 == 0 && pad % 256 == 0)
+    return launch_gemm<gemm::kRaggedM, gemm::kEpiDSwiGLU, 256, true>(dy, M, w2t, int64_t(E) * F, p,
+                                                                     (M / 256) * (F / 256), stream, 12);
   if (F % 256 == 0)
-    return launch_gemm<gemm::kRaggedM, gemm::kEpiDSwiGLU, 256>(dy, M, w2t, int64_t(E) * F, p, (M / 128) * (F / 256),
-                                                               stream, 5);
-  return launch_gemm<gemm::kRaggedM, gemm::kEpiDSwiGLU, 128>(dy, M, w2t, int64_t(E) * F, p, (M / 128) * (F / 128),
-                                                             stream, 6);
+    return launch_gemm<gemm::kRaggedM, gemm::kEpiDSwiGLU, 256, false>(dy, M, w2t, int64_t(E) * F, p,
+                                                                      (M / 128) * (F / 256), stream, 5);
+  return launch_gemm<gemm::kRaggedM, gemm::kEpiDSwiGLU, 128, false>(dy, M, w2t, int64_t(E) * F, p,
+                                                                    (M / 128) * (F / 128), stream, 6);
 }
 
 // ---------------------------------------------------------------- workspace

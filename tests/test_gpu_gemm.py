@@ -45,20 +45,21 @@ def _exact_pow2_ternary(g, shape, spread=3):
 
 
 # ------------------------------------------------------------------ ragged M
-@pytest.mark.parametrize("N", [256, 384])
-def test_grouped_gemm_exact_closed_form(N):
+@pytest.mark.parametrize("N,pad", [(256, 128), (384, 128), (512, 256), (256, 256)])
+def test_grouped_gemm_exact_closed_form(N, pad):
     """Exactly representable operands: fp32 accumulation is exact, so the bf16
-    output must equal round_to_bf16 of the exact product bit for bit."""
+    output must equal round_to_bf16 of the exact product bit for bit.
+    pad 256 with N % 256 == 0 runs the CTA-pair (256 x 256 tile) kernel."""
     g = np.random.default_rng(1)
     E, K = 3, 512
-    off = _offsets([200, 0, 300], 128)
+    off = _offsets([200, 0, 300], pad)
     M = int(off[-1]) + 128
     a = _exact_pow2_ternary(g, (M, K))
     w = _exact_pow2_ternary(g, (E, N, K))
     ac, as_ = _mx_rows_dev(_bf16(a))
     wc, ws = _mx_rows_dev(_bf16(w.reshape(E * N, K)))
     out = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device=DEV)
-    mxk.mxfp8_grouped_gemm(ac, as_, wc.reshape(E, N, K), ws, _dev(off), 128, out=out)
+    mxk.mxfp8_grouped_gemm(ac, as_, wc.reshape(E, N, K), ws, _dev(off), pad, out=out)
     got = bf16_np(out)
     for e in range(E):
         lo, hi = off[e], off[e + 1]
@@ -67,7 +68,7 @@ def test_grouped_gemm_exact_closed_form(N):
     assert mxk.device_error() == 0
 
 
-@pytest.mark.parametrize("pad,N,K", [(128, 512, 256), (256, 384, 640), (128, 256, 1408)])
+@pytest.mark.parametrize("pad,N,K", [(128, 512, 256), (256, 384, 640), (128, 256, 1408), (256, 512, 768)])
 def test_grouped_gemm_random_vs_oracle(pad, N, K):
     g = synth.rng(2)
     E = 4
@@ -122,9 +123,11 @@ def _mx_cols_dev(x_bf16: torch.Tensor):
     return o["col_codes"], o["col_scales"]
 
 
-def test_wgrad_exact_closed_form_and_empty_expert():
+@pytest.mark.parametrize("N,Kx", [(256, 384), (512, 512)])
+def test_wgrad_exact_closed_form_and_empty_expert(N, Kx):
+    """N = 256 / Kx = 384 takes the 128-wide tile, 512 / 512 the 256-wide one."""
     g = np.random.default_rng(4)
-    E, N, Kx = 3, 256, 384
+    E = 3
     off = _offsets([256, 0, 300], 128)
     M = int(off[-1])
     # COL quantization of G and X is exact when each 32-row block of a column
@@ -142,7 +145,7 @@ def test_wgrad_exact_closed_form_and_empty_expert():
     assert (got[1] == 0).all() and not np.signbit(got[1]).any()
 
 
-@pytest.mark.parametrize("pad,N,Kx", [(128, 256, 256), (256, 384, 512)])
+@pytest.mark.parametrize("pad,N,Kx", [(128, 256, 256), (256, 384, 512), (256, 512, 768)])
 def test_wgrad_random_vs_oracle(pad, N, Kx):
     g = synth.rng(5)
     E = 4
@@ -161,16 +164,17 @@ def test_wgrad_random_vs_oracle(pad, N, Kx):
 
 
 # ------------------------------------------------------------------ fused epilogues
-def test_fc1_swiglu_dual_quant_vs_oracle_and_standalone():
+@pytest.mark.parametrize("pad", [128, 256])
+def test_fc1_swiglu_dual_quant_vs_oracle_and_standalone(pad):
     g = synth.rng(6)
     E, D, F = 3, 256, 384
-    off = _offsets([200, 0, 140], 128)
+    off = _offsets([200, 0, 140], pad)
     M = int(off[-1])
     x = _bf16(synth.normal(g, (M, D)))
     w13 = _bf16(synth.normal(g, (E, 2 * F, D), 0.05))
     xc, xs = _mx_rows_dev(x)
     wc, ws = _mx_rows_dev(w13.reshape(E * 2 * F, D))
-    o = mxk.mxfp8_grouped_gemm_swiglu_quant(xc, xs, wc.reshape(E, 2 * F, D), ws, _dev(off), 128)
+    o = mxk.mxfp8_grouped_gemm_swiglu_quant(xc, xs, wc.reshape(E, 2 * F, D), ws, _dev(off), pad)
     # oracle: h13 per expert, then SwiGLU + dual quantization
     xr = mx.quantize_rows(bf16_np(x))
     wr = mx.quantize_weights_rows(bf16_np(w13))
@@ -188,10 +192,11 @@ def test_fc1_swiglu_dual_quant_vs_oracle_and_standalone():
         assert torch.equal(s[k].reshape(-1), o["h_" + k].reshape(-1)), k
 
 
-def test_fc2_dgrad_dswiglu_dual_quant_vs_oracle():
+@pytest.mark.parametrize("pad", [128, 256])
+def test_fc2_dgrad_dswiglu_dual_quant_vs_oracle(pad):
     g = synth.rng(7)
     E, D, F = 3, 384, 256
-    off = _offsets([150, 0, 250], 128)
+    off = _offsets([150, 0, 250], pad)
     M = int(off[-1])
     dy = _bf16(synth.normal(g, (M, D), 1e-2))
     w2 = _bf16(synth.normal(g, (E, D, F), 0.05))
@@ -199,7 +204,7 @@ def test_fc2_dgrad_dswiglu_dual_quant_vs_oracle():
     dr, ds = _mx_rows_dev(dy)
     w2t = mxk.mxfp8_quantize(w2.to(DEV), mxk.COL, mxk.MMA)        # [E, F, D]
     o = mxk.mxfp8_grouped_gemm_dswiglu_quant(dr, ds, w2t["col_codes"], w2t["col_scales"], _dev(off),
-                                             h13.to(DEV), 128)
+                                             h13.to(DEV), pad)
     dyr = mx.quantize_rows(bf16_np(dy))
     w2c = mx.quantize_weights_cols(bf16_np(w2))
     dh = mx.round_to_bf16(np.nan_to_num(mx.grouped_gemm(*dyr, *w2c, off)))
