@@ -290,6 +290,22 @@ def dist_setup(args):
     return world, rank, local
 
 
+def max_over_ranks(x: float, device=None) -> float:
+    """Max of a per-rank scalar over all ranks (identity without a process group)."""
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return float(x)
+    dev = device if device is not None else "cpu"
+    t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(flops_per_rank: float, world: int, ms_max: float) -> float:
+    """Replicas: every rank processes its own batch; the job's throughput is
+    all ranks' work over the slowest rank's time."""
+    return world * flops_per_rank / (ms_max * 1e-3) / 1e12
+
+
 def config_dict(spec, inp, extra=None):
     d = {"workload": f"{spec.name}: E={spec.E} D={spec.D} F={spec.F} tokens={spec.tokens} top{spec.top_k} "
                      f"Zipf({spec.zipf_s}) pad {spec.pad}, fwd+bwd; + SwiGLU quant 16384x2x4096 + cast 8192x7168",
@@ -394,11 +410,7 @@ def main():
         raise RuntimeError("device error during the timed region")
     per = np.array([[evs[k][i].elapsed_time(evs[k][i + 1]) for i in range(n_ops)] for k in range(args.steps)])
     mean_ms = per.mean(axis=0)
-    ms_step = ms_total / args.steps
-    if world > 1:
-        t = torch.tensor([ms_step], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_step = float(t.item())
+    ms_step = max_over_ranks(ms_total / args.steps, dev)
 
     peaks, peak_src = load_peaks()
     fp8_sus = 2.0 * peaks["bf16_tflops_sustained"]     # MXFP8 dense = 2 x bf16 (nominal 4.5 / 2.25 PF)
@@ -415,7 +427,7 @@ def main():
     cast_w_ms = float(sum(mean_ms[i] for i, (n, *_r) in enumerate(step.ops) if n.startswith("cast_w")))
     useful = step.flops(step.R)
     executed = step.flops(step.M)
-    value = world * useful / (ms_step * 1e-3) / 1e12
+    value = whole_job_tflops(useful, world, ms_step)
     fwd_ms = float(mean_ms[[0, 3, 4]].sum())   # x cast, FC1, FC2 (weights already quantized)
 
     # dominant kernel and its roofline
@@ -470,13 +482,9 @@ def main():
             e2e_step()
         b.record()
         torch.cuda.synchronize()
-        ms = a.elapsed_time(b) / args.steps
-        if world > 1:
-            t = torch.tensor([ms], device=dev)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            ms = float(t.item())
+        ms = max_over_ranks(a.elapsed_time(b) / args.steps, dev)
         h2d = x_h.numel() * 2 + dy_h.numel() * 2 + off_h.numel() * 4
-        e2e = {"value": round(world * useful / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+        e2e = {"value": round(whole_job_tflops(useful, world, ms), 2), "unit": "TFLOP/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(out_h.numel() * 2),
                "ms_per_step": round(ms, 3)}
         if mxk.device_error() != 0:
@@ -495,7 +503,7 @@ def main():
         "data": "synthetic (seeded routing, device-drawn bf16 activations and weights)",
         "config": config_dict(spec, inp, {"parallelism": f"replicas x{world} (no data-path collective)"}),
         "fwd_bwd_useful_tflops": round(value, 2),
-        "fwd_bwd_executed_tflops": round(world * executed / (ms_step * 1e-3) / 1e12, 2),
+        "fwd_bwd_executed_tflops": round(whole_job_tflops(executed, world, ms_step), 2),
         "mlp_ms": round(mlp_ms, 3),
         "mlp_no_weight_cast_tflops": round(useful / ((mlp_ms - cast_w_ms) * 1e-3) / 1e12, 2),
         "fwd_useful_tflops_prequantized_weights": round(6.0 * step.R * spec.D * spec.F / (fwd_ms * 1e-3) / 1e12, 2),

@@ -65,18 +65,18 @@ template <int kMode, int kEpi, int BN, bool kPair>
 struct Cfg {
   static constexpr int BM = 128, BK = 128;
   static constexpr int kAcc = (BN == 256) ? 1 : 2;
-  static constexpr int kBBox = kPair ? BN / 256 : BN / 128;   // 128-row B boxes loaded per CTA and stage
+  static constexpr int B_ROWS = kPair ? BN / 2 : BN;           // B rows loaded per CTA and stage
   static constexpr int A_BYTES = BM * BK;
-  static constexpr int B_BYTES = kBBox * 128 * BK;
+  static constexpr int B_BYTES = B_ROWS * BK;
   static constexpr int SFA_BYTES = 512;
   static constexpr int SFB_BYTES = (BN / 128) * 512;          // scales of all BN rows of B
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
-  static constexpr int kStages = kPair ? 6 : ((BN == 256) ? 4 : 6);
+  static constexpr int kStages = kPair ? ((BN == 256) ? 6 : 7) : ((BN == 256) ? 4 : 6);
   static constexpr int SF_COLS = 4 + BN / 32;           // TMEM columns for one SF buffer
   static constexpr int ACC_COLS = kAcc * BN;
   static constexpr int TMEM_COLS = 512;
   static_assert(ACC_COLS + 2 * SF_COLS <= TMEM_COLS, "TMEM budget");
-  static_assert(!kPair || BN == 256, "CTA pairs use 256-wide tiles");
+  static_assert(!kPair || BN == 256 || BN == 128, "CTA pair tile widths");
   // shared memory map (offsets from a 1024-aligned base)
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + kStages * A_BYTES;
@@ -84,7 +84,7 @@ struct Cfg {
   static constexpr int OFF_SFB = OFF_SFA + kStages * SFA_BYTES;
   static constexpr int OFF_EPI = OFF_SFB + kStages * SFB_BYTES;
   static constexpr int EPI_WARPS = 8;
-  static constexpr int EPI_WARP_BYTES = 32 * 17 * 4;       // 32x32 bf16 transpose / staging buffer
+  static constexpr int EPI_WARP_BYTES = 2560;               // 32x32 bf16 transpose / staging buffer (512-aligned)
   static constexpr int EPI_BYTES = EPI_WARPS * EPI_WARP_BYTES;
   static constexpr int OFF_BAR = OFF_EPI + EPI_BYTES;
   static constexpr int NUM_BARS = 2 * kStages + 2 * kAcc;
@@ -160,7 +160,10 @@ __device__ __forceinline__ Tile get_tile(const Params& p, const int32_t* offs, i
     T.out_r0 = T.a_row;
     T.out_c0 = jt * BN;
   }
-  T.b_mine = rank ? T.b_row1 : T.b_row0;
+  if constexpr (kEpi == kEpiSwiGLU)
+    T.b_mine = rank ? T.b_row1 : T.b_row0;          // gate rows on the even CTA, up rows on the odd one
+  else
+    T.b_mine = T.b_row0 + rank * (BN / 2);
   return T;
 }
 
@@ -183,25 +186,31 @@ __device__ __forceinline__ void warp_transpose32(uint32_t* buf, const uint32_t* 
   __syncwarp();
 }
 
-// Store a 32-row x 64-byte block (one row per lane, 4 x 16 B in v) so that
-// each store instruction writes 8 whole 64-byte row segments: the block goes
-// through shared memory (16-byte chunk c of row r at chunk c ^ ((r >> 1) & 3),
-// conflict-free) and comes back out row-contiguous.  dst0 = first row, ld in
-// bytes.
-__device__ __forceinline__ void store_rows64(uint8_t* sbuf, const uint32_t* v, uint8_t* dst0, int64_t ld,
-                                             int lane) {
+// The warp's staging buffer may still be read by this warp's last TMA store:
+// wait for that read before rewriting it.
+__device__ __forceinline__ void sbuf_acquire(int lane) {
+  if (lane == 0) bulk_wait_read_all();
+  __syncwarp();
+}
+
+// Store a 32-row x 32-column bf16 block (one row per lane, 4 x 16 B in v) with
+// one asynchronous TMA store: the block is written to the warp's staging
+// buffer in the tensor map's 64-byte swizzle (16-byte chunk c of row r at
+// chunk c ^ ((r >> 1) & 3), conflict-free) and lane 0 hands it to the TMA
+// engine; the warp continues without waiting for the global write.
+__device__ __forceinline__ void store_block_tma(uint8_t* sbuf, const uint32_t* v, const void* tmap, int x, int y,
+                                                int lane) {
+  sbuf_acquire(lane);
 #pragma unroll
   for (int c = 0; c < 4; ++c)
     *reinterpret_cast<uint4*>(sbuf + lane * 64 + ((c ^ ((lane >> 1) & 3)) << 4)) =
         make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+  fence_proxy_async();
   __syncwarp();
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int r = 8 * i + (lane >> 2), c = lane & 3;
-    const uint4 t = *reinterpret_cast<const uint4*>(sbuf + r * 64 + ((c ^ ((r >> 1) & 3)) << 4));
-    *reinterpret_cast<uint4*>(dst0 + r * ld + c * 16) = t;
+  if (lane == 0) {
+    tma_store_2d(tmap, smem_u32(sbuf), x, y);
+    bulk_commit();
   }
-  __syncwarp();
 }
 
 // Same for a 32-row x 32-byte block (one row per lane, 2 x 16 B in v):
@@ -209,6 +218,7 @@ __device__ __forceinline__ void store_rows64(uint8_t* sbuf, const uint32_t* v, u
 // writes 16 whole 32-byte row segments.
 __device__ __forceinline__ void store_rows32(uint8_t* sbuf, const uint4 (&v)[2], uint8_t* dst0, int64_t ld,
                                              int lane) {
+  sbuf_acquire(lane);
 #pragma unroll
   for (int c = 0; c < 2; ++c)
     *reinterpret_cast<uint4*>(sbuf + lane * 32 + ((c ^ ((lane >> 2) & 1)) << 4)) = v[c];
@@ -253,6 +263,7 @@ __device__ __forceinline__ void dual_quant_block(const uint32_t* v, int lane, ui
   store_rows32(sbuf, q, row_codes + row0 * ld_row + col0, ld_row, lane);
   row_scales[mma_scale_offset(row0 + lane, col0 >> 5, ld_row)] = uint8_t(rb);
   uint32_t c[16];
+  sbuf_acquire(lane);
   warp_transpose32(reinterpret_cast<uint32_t*>(sbuf), v, c, lane);
   const int64_t crow = col0 + lane;
   const uint32_t cb = quant32(c, q);
@@ -285,7 +296,7 @@ template <int kMode, int kEpi, int BN, bool kPair>
 __global__ void __launch_bounds__(384, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                     const __grid_constant__ CUtensorMap tmap_sa, const __grid_constant__ CUtensorMap tmap_sb,
-                    const Params p) {
+                    const __grid_constant__ CUtensorMap tmap_o, const Params p) {
   using C = Cfg<kMode, kEpi, BN, kPair>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -381,8 +392,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
                              int(((T.a_row / 128) * katoms + kat) * 2));
             tma_load_2d_pair(sbase + C::OFF_SFB + stage * C::SFB_BYTES, &tmap_sb, fb, 0,
                              int(((T.b_row0 / 128) * katoms + kat) * 2));
-            tma_load_2d_pair(sbase + C::OFF_SFB + stage * C::SFB_BYTES + 512, &tmap_sb, fb, 0,
-                             int(((T.b_row1 / 128) * katoms + kat) * 2));
+            if constexpr (BN == 256)
+              tma_load_2d_pair(sbase + C::OFF_SFB + stage * C::SFB_BYTES + 512, &tmap_sb, fb, 0,
+                               int(((T.b_row1 / 128) * katoms + kat) * 2));
           } else {
             const uint32_t fb = full_bar(stage);
             mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
@@ -485,10 +497,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
           uint32_t z[16];
 #pragma unroll
           for (int j = 0; j < 16; ++j) z[j] = 0u;
-          uint8_t* o = reinterpret_cast<uint8_t*>(p.out + (int64_t(T.e) * p.rows_a + row0) * p.n_out + T.out_c0 +
-                                                  h * kHalf);
 #pragma unroll 1
-          for (int c = 0; c < kChunks; ++c) store_rows64(sbuf, z, o + c * 64, p.n_out * 2, lane);
+          for (int c = 0; c < kChunks; ++c)
+            store_block_tma(sbuf, z, &tmap_o, int(T.out_c0 + h * kHalf + 32 * c), int(int64_t(T.e) * p.rows_a + row0),
+                            lane);
           continue;
         }
       }
@@ -515,13 +527,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
       if (++acc == C::kAcc) { acc = 0; acc_phase ^= 1; }
 
       if constexpr (kEpi == kEpiBF16) {
-        uint8_t* o;
-        if constexpr (kMode == kRaggedK)
-          o = reinterpret_cast<uint8_t*>(p.out + (int64_t(T.e) * p.rows_a + row0) * p.n_out + T.out_c0 + h * kHalf);
-        else
-          o = reinterpret_cast<uint8_t*>(p.out + row0 * p.n_out + T.out_c0 + h * kHalf);
+        const int64_t orow = (kMode == kRaggedK) ? int64_t(T.e) * p.rows_a + row0 : row0;
 #pragma unroll
-        for (int c = 0; c < kChunks; ++c) store_rows64(sbuf, va + 16 * c, o + c * 64, p.n_out * 2, lane);
+        for (int c = 0; c < kChunks; ++c)
+          store_block_tma(sbuf, va + 16 * c, &tmap_o, int(T.out_c0 + h * kHalf + 32 * c), int(orow), lane);
       } else if constexpr (kEpi == kEpiSwiGLU) {
         const int64_t F = p.F;
 #pragma unroll
@@ -530,9 +539,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
           const uint32_t* a2 = va + 16 * c;
           const uint32_t* b2 = vb + 16 * c;
           if (p.out != nullptr) {
-            uint8_t* o = reinterpret_cast<uint8_t*>(p.out + row0 * 2 * F);
-            store_rows64(sbuf, a2, o + f * 2, 4 * F, lane);
-            store_rows64(sbuf, b2, o + (F + f) * 2, 4 * F, lane);
+            store_block_tma(sbuf, a2, &tmap_o, int(f), int(row0), lane);
+            store_block_tma(sbuf, b2, &tmap_o, int(F + f), int(row0), lane);
           }
           uint32_t h2[16];
 #pragma unroll
@@ -575,6 +583,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
       }
     }
   }
+
+  // outstanding TMA stores of the epilogue warps complete before the CTA exits
+  if (warp >= 4 && lane == 0) bulk_wait_all();
 
   // ---- teardown: every role has left its loop (all waits are bounded); in a
   // pair, neither CTA frees its TMEM or exits while the other may still

@@ -109,13 +109,13 @@ int get_encode(EncodeTiledFn* fn) {
   return MXMOE_OK;
 }
 
-// 2-D uint8 K-major operand [rows, kext], box 128 x 128 bytes, 128-byte swizzle.
-int make_operand_map(CUtensorMap* map, const uint8_t* base, int64_t rows, int64_t kext) {
+// 2-D uint8 K-major operand [rows, kext], box 128 bytes x box_rows, 128-byte swizzle.
+int make_operand_map(CUtensorMap* map, const uint8_t* base, int64_t rows, int64_t kext, uint32_t box_rows = 128) {
   EncodeTiledFn enc;
   MX_TRY(get_encode(&enc));
   cuuint64_t dims[2] = {cuuint64_t(kext), cuuint64_t(rows)};
   cuuint64_t strides[1] = {cuuint64_t(kext)};
-  cuuint32_t box[2] = {128, 128};
+  cuuint32_t box[2] = {128, box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -178,6 +178,21 @@ int launch_cast(const void* in, int64_t batch, int64_t rows, int64_t cols, int m
   return MXMOE_OK;
 }
 
+// bf16 output [rows, cols] stored in 32 x 32 boxes with the 64-byte swizzle.
+int make_out_map(CUtensorMap* map, const void* base, int64_t rows, int64_t cols) {
+  EncodeTiledFn enc;
+  MX_TRY(get_encode(&enc));
+  cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
+  cuuint64_t strides[1] = {cuuint64_t(cols * 2)};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MXMOE_ERR_CUDA, "cuTensorMapEncodeTiled (output) failed (%d)", int(r));
+  return MXMOE_OK;
+}
+
 // Scale atoms of an MMA-layout scale buffer of `bytes` bytes as a 2-D uint8
 // map [bytes/256, 256] with 256 x 2 boxes (one 512-byte atom per box).
 int make_scale_map(CUtensorMap* map, const uint8_t* base, int64_t bytes) {
@@ -211,7 +226,7 @@ int launch_gemm(const uint8_t* a, int64_t a_rows, const uint8_t* b, int64_t b_ro
   if (p.E > C::MAX_E) return fail(MXMOE_ERR_SHAPE, "E=%d exceeds the supported maximum %d", p.E, C::MAX_E);
   CUtensorMap ma, mb, msa, msb;
   MX_TRY(make_operand_map(&ma, a, a_rows, p.kext));
-  MX_TRY(make_operand_map(&mb, b, b_rows, p.kext));
+  MX_TRY(make_operand_map(&mb, b, b_rows, p.kext, kPair ? BN / 2 : 128));
   if constexpr (kPair) {
     MX_TRY(make_scale_map(&msa, p.a_scales, a_rows * p.kext / 32));
     MX_TRY(make_scale_map(&msb, p.b_scales, b_rows * p.kext / 32));
@@ -219,10 +234,22 @@ int launch_gemm(const uint8_t* a, int64_t a_rows, const uint8_t* b, int64_t b_ro
     msa = ma;   // unused by the single-CTA kernel
     msb = mb;
   }
+  // bf16 output written by TMA stores: [M, N] (ragged M), [E*N, Kx] (ragged K), h13 [M, 2F] (SwiGLU)
+  CUtensorMap mo = ma;
+  if (p.out != nullptr) {
+    if constexpr (kEpi == gemm::kEpiBF16) {
+      if constexpr (kMode == gemm::kRaggedK)
+        MX_TRY(make_out_map(&mo, p.out, int64_t(p.E) * p.rows_a, p.n_out));
+      else
+        MX_TRY(make_out_map(&mo, p.out, p.M, p.n_out));
+    } else if constexpr (kEpi == gemm::kEpiSwiGLU) {
+      MX_TRY(make_out_map(&mo, p.out, p.M, 2 * p.F));
+    }
+  }
   if (max_tiles <= 0) return MXMOE_OK;
   if constexpr (!kPair) {
     const int grid = int(max_tiles < d->sms ? max_tiles : d->sms);
-    kern<<<grid, 384, C::SMEM_BYTES, stream>>>(ma, mb, msa, msb, p);
+    kern<<<grid, 384, C::SMEM_BYTES, stream>>>(ma, mb, msa, msb, mo, p);
   } else {
     // clusters of two CTAs, one pair per two SMs (as many as can be resident)
     cudaLaunchConfig_t cfg = {};
@@ -244,7 +271,7 @@ int launch_gemm(const uint8_t* a, int64_t a_rows, const uint8_t* b, int64_t b_ro
     cudaGetLastError();
     if (max_tiles < pairs) pairs = int(max_tiles);
     cfg.gridDim = dim3(unsigned(2 * pairs), 1, 1);
-    MX_CHECK_CUDA(cudaLaunchKernelEx(&cfg, kern, ma, mb, msa, msb, p), "grouped GEMM (CTA pair) launch");
+    MX_CHECK_CUDA(cudaLaunchKernelEx(&cfg, kern, ma, mb, msa, msb, mo, p), "grouped GEMM (CTA pair) launch");
   }
   MX_CHECK_CUDA(cudaGetLastError(), "grouped GEMM launch");
   return MXMOE_OK;
