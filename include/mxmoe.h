@@ -80,8 +80,16 @@ const char* mxmoe_last_error(void);
  * the read itself failed. */
 int mxmoe_device_error(cudaStream_t stream, int reset, int* code);
 
-/* Library version string and number of SMs the kernels size grids for. */
+/* Library version string. */
 const char* mxmoe_version(void);
+
+/* Self-test of the failure path: launches one thread that waits, with the
+ * same bounded mbarrier wait the GEMM and cast kernels use, on a barrier that
+ * nothing ever arrives on.  After the wait limit (about 2^32 SM cycles, ~2 s)
+ * the kernel records MXMOE_ERR_DEVICE_TIMEOUT in the device error word and
+ * returns normally, leaving the context usable; read it with
+ * mxmoe_device_error(). */
+int mxmoe_selftest_wait_timeout(cudaStream_t stream);
 
 /* -------------------------------------------------------------------------
  * mxfp8_quantize -- bf16 -> MXFP8 cast, row-wise and/or column-wise.

@@ -64,6 +64,7 @@ _SIGS = {
     "moe_mlp_bwd": ([_P, _L, _L, _P, _P, _I, _L, _P, _I, ctypes.POINTER(_Saved), _P, _P, _P, _P, _S, _P], _I),
     "moe_mlp_fwd_noalloc": ([_P, _L, _L, _P, _P, _I, _L, _P, _I, _P, ctypes.POINTER(_Saved), _P], _I),
     "mxmoe_quantize_weights": ([_P, _P, _I, _L, _L, ctypes.POINTER(_QWeights), _P], _I),
+    "mxmoe_selftest_wait_timeout": ([_P], _I),
     "moe_mlp_fwd_q": ([_P, _L, _L, ctypes.POINTER(_QWeights), _I, _L, _P, _I, _P, ctypes.POINTER(_Saved), _P, _S,
                        _P], _I),
     "moe_mlp_bwd_q": ([_P, _L, _L, ctypes.POINTER(_QWeights), _I, _L, _P, _I, ctypes.POINTER(_Saved), _P, _P, _P,

@@ -572,8 +572,27 @@ uint8_t* align_ws(void* ws) {
 
 }  // namespace
 
+// One thread waits on a barrier nothing arrives on: the bounded wait gives up
+// and the kernel records the timeout (exercises the failure path).
+__global__ void selftest_wait_kernel() {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mxmoe::sm100::mbar_init(mxmoe::sm100::smem_u32(&bar), 1);
+    mxmoe::sm100::fence_mbar_init();
+    if (!mxmoe::sm100::mbar_wait(mxmoe::sm100::smem_u32(&bar), 0)) raise_device_error(MXMOE_ERR_DEVICE_TIMEOUT);
+  }
+}
+
 // =====================================================================================
 extern "C" {
+
+int mxmoe_selftest_wait_timeout(cudaStream_t stream) {
+  DevInfo* d;
+  MX_TRY(device_info(&d));
+  selftest_wait_kernel<<<1, 32, 0, stream>>>();
+  MX_CHECK_CUDA(cudaGetLastError(), "self-test launch");
+  return MXMOE_OK;
+}
 
 const char* mxmoe_last_error(void) { return g_err; }
 

@@ -44,13 +44,13 @@ constexpr int kTileBytes = kTile * kTile * 2;       // one bf16 128 x 128 tile
 
 template <bool kSwiglu>
 struct CastCfg {
-  static constexpr int kStages = 2;
+  static constexpr int kStages = kSwiglu ? 1 : 2;       // SwiGLU: two CTAs per SM take turns instead
   static constexpr int kStageBytes = kSwiglu ? 2 * kTileBytes : kTileBytes;
   static constexpr int kOffColStage = kStages * kStageBytes;         // COL codes of one tile, 128 x 128 B
   static constexpr int kOffScales = kOffColStage + kTile * kTile;    // ROW then COL scale bytes, 512 B each
   static constexpr int kOffBars = kOffScales + 1024;
   static constexpr int kSmem = kOffBars + 2 * kStages * 8 + 128;     // + alignment slack
-  static constexpr int kCtasPerSm = kSwiglu ? 1 : 2;
+  static constexpr int kCtasPerSm = 2;
 };
 
 __device__ __forceinline__ uint32_t swiglu_pair(uint32_t g, uint32_t u) {

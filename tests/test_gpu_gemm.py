@@ -216,3 +216,19 @@ def test_fc2_dgrad_dswiglu_dual_quant_vs_oracle(pad):
     got_cs = mma_to_plain(u8(o["g_col_scales"]), 2 * F, M)
     assert_codes_close(u8(o["g_row_codes"]), rc, got_rs, rs, "dh13 ROW")
     assert_codes_close(u8(o["g_col_codes"]), cc, got_cs, cs, "dh13 COL")
+
+
+def test_bounded_wait_times_out_and_reports():
+    """A wait on a barrier nothing arrives on gives up (about 2 s), records
+    MXMOE_ERR_DEVICE_TIMEOUT and leaves the context usable."""
+    import ctypes
+    L = mxk.lib()
+    assert mxk.device_error() == 0
+    st = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    assert L.mxmoe_selftest_wait_timeout(st) == 0
+    assert mxk.device_error(reset=True) == 7
+    # the context still works
+    x = torch.ones(128, 128, dtype=torch.bfloat16, device=DEV)
+    o = mxk.mxfp8_quantize(x, mxk.ROW)
+    assert (o["row_codes"] == 0x78).all()           # 1.0 under scale 2^-8 is 256 = E4M3 0x78
+    assert mxk.device_error() == 0

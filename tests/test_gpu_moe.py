@@ -145,3 +145,141 @@ def test_prequantized_weights_path_matches_bf16_weight_composites():
     assert torch.equal(r["row_codes"].reshape(-1), qw["w13_codes"].reshape(-1))
     assert torch.equal(r["col_codes"].reshape(-1), qw["w13t_codes"].reshape(-1))
     assert torch.equal(r["row_scales"], qw["w13_scales"]) and torch.equal(r["col_scales"], qw["w13t_scales"])
+
+
+def _assert_chained_close(got, ref, what):
+    """Chained composite outputs: every GEMM of the chain is held to the GEMM
+    bar on identical operands (test_dsv3_full_size_step_gemms_on_oracle_operands);
+    end to end the two sides also differ by the allowed one-code differences of
+    the fused epilogues (h, dh13: fp32 vs float64 accumulation moves a bf16
+    rounding in ~1e-3 of the elements), which outlier activations (x50)
+    amplify in the weight gradients.  Bar: relative Frobenius 2e-3, max-abs
+    5e-2 * max|ref|."""
+    assert_gemm_close(got, ref, what, rel=2e-3, absf=5e-2)
+
+
+def test_dsv3_full_size_prequantized_path_sampled_experts():
+    """The configuration bench.py times: E=256, D=7168, F=2048, 16384 tokens
+    top-8, Zipf(1.0), pad 256, inputs drawn on the device, one training step
+    through mxmoe_quantize_weights + moe_mlp_fwd_q + moe_mlp_bwd_q.  The
+    median-sized and the largest expert are checked against the oracle chain."""
+    inp = synth.device_moe_inputs("dsv3", 0, device=DEV)
+    r = inp.routing
+    off = torch.from_numpy(r.offsets).to(DEV)
+    qw = mxk.mxmoe_quantize_weights(inp.w13, inp.w2)
+    y, saved = mxk.moe_mlp_fwd_q(inp.x, qw, off, inp.spec.pad)
+    dx, dw13, dw2 = mxk.moe_mlp_bwd_q(inp.dy, qw, off, saved, inp.spec.pad)
+    torch.cuda.synchronize()
+    assert mxk.device_error() == 0
+    counts = r.counts
+    order = [int(e) for e in np.argsort(counts) if counts[e] > 0]
+    M, D, F = r.M, inp.spec.D, inp.spec.F
+    for e in (order[len(order) // 2], order[-1]):
+        lo, hi = int(r.offsets[e]), int(r.offsets[e + 1])
+        x_e, dy_e = bf16_np(inp.x[lo:hi]), bf16_np(inp.dy[lo:hi])
+        w13_e, w2_e = bf16_np(inp.w13[e]), bf16_np(inp.w2[e])
+        rf = mx.expert_fwd(x_e, w13_e, w2_e)
+        rb = mx.expert_bwd(dy_e, rf, x_e, w13_e, w2_e)
+        assert_gemm_close(bf16_np(saved["h13"][lo:hi]), rf["h13"], f"h13[e={e}]")
+        assert_gemm_close(bf16_np(y[lo:hi]), rf["y"], f"y[e={e}]")
+        _assert_chained_close(bf16_np(dx[lo:hi]), rb["dx"], f"dx[e={e}]")
+        _assert_chained_close(bf16_np(dw13[e]), rb["dw13"], f"dw13[e={e}]")
+        _assert_chained_close(bf16_np(dw2[e]), rb["dw2"], f"dw2[e={e}]")
+        xcc = u8(saved["x_col_codes"])[:, lo:hi]
+        np.testing.assert_array_equal(xcc, rf["x_col"][0])           # the cast is exact
+        hcc = u8(saved["h_col_codes"])[:, lo:hi]
+        hcs = mma_to_plain(u8(saved["h_col_scales"]), F, M)[:, lo // 32:hi // 32]
+        assert_codes_close(hcc, rf["h_col"][0], hcs, rf["h_col"][1], f"h COL[e={e}]")
+
+
+def _full_mma(plain_full):
+    """Plain [R, C/32] scales -> flat MMA-layout bytes on the device."""
+    from mxtest import plain_to_mma
+    return torch.from_numpy(plain_to_mma(plain_full)).to(DEV)
+
+
+def test_dsv3_full_size_step_gemms_on_oracle_operands():
+    """Each grouped GEMM of the step at the DSv3-scale launch configuration
+    (full routing, M = 162,560 padded rows, E = 256) on operands the oracle
+    quantized: one expert's rows/columns hold the oracle's codes and scales,
+    every other expert's are zero.  The GPU result for that expert must meet
+    the GEMM bar against the oracle's float64 product of the same codes."""
+    spec = synth.SPECS["dsv3"]
+    r = synth.make_routing(spec, 0)
+    M, E, D, F = r.M, spec.E, spec.D, spec.F
+    order = [int(e) for e in np.argsort(r.counts) if r.counts[e] > 0]
+    e = order[len(order) // 2]
+    lo, hi = int(r.offsets[e]), int(r.offsets[e + 1])
+    n = hi - lo
+    g = synth.rng(11)
+    f = lambda a: synth.to_bf16(a).float().double().numpy()
+    x_e = f(synth.normal(g, (n, D), 1.0, 1e-3, 50.0))
+    x_e[int(r.counts[e]):] = 0.0                                   # pad rows
+    dy_e = f(synth.normal(g, (n, D), 1e-2))
+    dy_e[int(r.counts[e]):] = 0.0
+    w13_e = f(synth.normal(g, (2 * F, D), spec.w_std))
+    w2_e = f(synth.normal(g, (D, F), spec.w_std))
+    rf = mx.expert_fwd(x_e, w13_e, w2_e)
+    rb = mx.expert_bwd(dy_e, rf, x_e, w13_e, w2_e)
+    off = torch.from_numpy(r.offsets).to(DEV)
+    u8z = lambda *sh: np.zeros(sh, dtype=np.uint8)
+
+    def rows_operand(codes_e, scales_e, K):           # [M, K] with rows lo:hi filled
+        c, s_ = u8z(M, K), u8z(M, K // 32)
+        c[lo:hi], s_[lo:hi] = codes_e, scales_e
+        return torch.from_numpy(c).to(DEV), _full_mma(s_)
+
+    def cols_operand(codes_e, scales_e, N):           # [N, M] with columns lo:hi filled
+        c, s_ = u8z(N, M), u8z(N, M // 32)
+        c[:, lo:hi], s_[:, lo // 32:hi // 32] = codes_e, scales_e
+        return torch.from_numpy(c).to(DEV), _full_mma(s_)
+
+    def weight_operand(codes_e, scales_e, N, K):      # [E, N, K] with expert e filled
+        c, s_ = u8z(E, N, K), u8z(E * N, K // 32)
+        c[e] = codes_e
+        s_[e * N:(e + 1) * N] = scales_e
+        return torch.from_numpy(c).to(DEV), _full_mma(s_)
+
+    # a3: h13 = x_ROW . W13_ROW^T, SwiGLU + dual quant
+    a, sa = rows_operand(*rf["x_row"], D)
+    w, sw = weight_operand(*mx.quantize_rows(w13_e), 2 * F, D)
+    o = mxk.mxfp8_grouped_gemm_swiglu_quant(a, sa, w, sw, off, spec.pad)
+    assert_gemm_close(bf16_np(o["h13"][lo:hi]), rf["h13"], "h13 (a3)")
+    rs = mma_to_plain(u8(o["h_row_scales"]), M, F)[lo:hi]
+    assert_codes_close(u8(o["h_row_codes"])[lo:hi], rf["h_row"][0], rs, rf["h_row"][1], "h ROW (a3)")
+    del a, sa, w, sw, o
+    # a6: dh = dY_ROW . W2_COL, dSwiGLU with the oracle's h13, dual quant
+    a, sa = rows_operand(*rb["dy_row"], D)
+    w, sw = weight_operand(*mx.quantize_cols(w2_e), F, D)
+    h13 = np.zeros((M, 2 * F), dtype=np.float32)
+    h13[lo:hi] = rf["h13"]
+    o = mxk.mxfp8_grouped_gemm_dswiglu_quant(a, sa, w, sw, off, synth.to_bf16(h13).to(DEV), spec.pad)
+    gs_ = mma_to_plain(u8(o["g_row_scales"]), M, 2 * F)[lo:hi]
+    assert_codes_close(u8(o["g_row_codes"])[lo:hi], rb["dh13_row"][0], gs_, rb["dh13_row"][1], "dh13 ROW (a6)")
+    del a, sa, w, sw, o, h13
+    torch.cuda.empty_cache()
+    # a4: y = h_ROW . W2_ROW^T
+    a, sa = rows_operand(*rf["h_row"], F)
+    w, sw = weight_operand(*mx.quantize_rows(w2_e), D, F)
+    y = mxk.mxfp8_grouped_gemm(a, sa, w, sw, off, spec.pad)
+    assert_gemm_close(bf16_np(y[lo:hi]), rf["y"], "y (a4)")
+    del a, sa, w, sw, y
+    # a8: dx = dh13_ROW . W13_COL (W13 COL codes stored [E, D, 2F])
+    a, sa = rows_operand(*rb["dh13_row"], 2 * F)
+    w, sw = weight_operand(*mx.quantize_cols(w13_e), D, 2 * F)
+    dx = mxk.mxfp8_grouped_gemm(a, sa, w, sw, off, spec.pad)
+    assert_gemm_close(bf16_np(dx[lo:hi]), rb["dx"], "dx (a8)")
+    del a, sa, w, sw, dx
+    torch.cuda.empty_cache()
+    # a7: dW2 = dY_COL^T . h_COL ; a9: dW13 = dh13_COL^T . x_COL
+    gt, gs = cols_operand(*rb["dy_col"], D)
+    xt, xs = cols_operand(*rf["h_col"], F)
+    dw2 = mxk.mxfp8_grouped_gemm_wgrad(gt, gs, xt, xs, off, spec.pad)
+    assert_gemm_close(bf16_np(dw2[e]), rb["dw2"], "dW2 (a7)")
+    del gt, gs, xt, xs, dw2
+    torch.cuda.empty_cache()
+    gt, gs = cols_operand(*rb["dh13_col"], 2 * F)
+    xt, xs = cols_operand(*rf["x_col"], D)
+    dw13 = mxk.mxfp8_grouped_gemm_wgrad(gt, gs, xt, xs, off, spec.pad)
+    assert_gemm_close(bf16_np(dw13[e]), rb["dw13"], "dW13 (a9)")
+    assert mxk.device_error() == 0
