@@ -6,8 +6,9 @@ tokens: the DSv3-scale expert layer (E=256, D=7168, F=2048, 16384 tokens
 top-8, Zipf(1.0) routing padded to 256) forward and backward -- token and
 weight casts, FC1 + SwiGLU + dual quant, FC2, dY casts, FC2 dgrad + dSwiGLU +
 dual quant, dW2, dx, dW13 -- plus the standalone SwiGLU + dual quant of
-h13 [16384, 2x4096] and the bf16 -> MXFP8 cast of the [8192, 7168] transport
-payload.
+h13 [16384, 2x4096], the bf16 -> MXFP8 cast of the [8192, 7168] transport
+payload and its dequantization back to bf16.  After the timed steps the fused
+forward is timed against the unfused ("swiglu" plan) forward.
 
 Prints one JSON line.  `value` is the useful (real routed rows) fwd+bwd
 TFLOP/s of the expert MLP with inputs resident in HBM; every input is larger
@@ -167,6 +168,7 @@ class Step:
         self.sw_cc, self.sw_cs = u8(SWIGLU_F, SWIGLU_ROWS), u8(SWIGLU_ROWS * SWIGLU_F // 32)
         self.c_in = inp.cast_x
         self.c_rc, self.c_rs = u8(CAST_ROWS, CAST_COLS), u8(CAST_ROWS, CAST_COLS // 32)
+        self.c_deq = bf(CAST_ROWS, CAST_COLS)
         self.stream = torch.cuda.current_stream(dev)
         self._build()
 
@@ -212,6 +214,8 @@ class Step:
                                           p(self.sw_cc), p(self.sw_cs), st)),
             ("cast_payload_8192x7168", "hbm", 3.03125 * CAST_ROWS * CAST_COLS,
              lambda: L.mxfp8_quantize(p(self.c_in), 1, CAST_ROWS, CAST_COLS, 1, 0, p(self.c_rc), p(self.c_rs), None, None, st)),
+            ("dequant_payload_8192x7168", "hbm", 3.03125 * CAST_ROWS * CAST_COLS,
+             lambda: L.mxfp8_dequantize(p(self.c_rc), p(self.c_rs), CAST_ROWS, CAST_COLS, p(self.c_deq), st)),
         ]
         self.mlp_ops = 10
 
@@ -430,6 +434,39 @@ def main():
     value = whole_job_tflops(useful, world, ms_step)
     fwd_ms = float(mean_ms[[0, 3, 4]].sum())   # x cast, FC1, FC2 (weights already quantized)
 
+    # fused vs unfused forward (the pages' comparison), same inputs and weights
+    def fwd_fused():
+        step.ops[0][3]()
+        step.ops[3][3]()
+        step.ops[4][3]()
+
+    def fwd_unfused():
+        L, p, st = step.L, (lambda t: t.data_ptr()), step.stream.cuda_stream
+        q = {k: p(v) for k, v in step.qw.items()}
+        M, D, E, F, pad, off = step.M, step.D, step.E, step.F, step.pad, p(step.off)
+        step.ops[0][3]()
+        L.mxfp8_grouped_gemm(p(step.x_rc), p(step.x_rs), M, D, q["w13_codes"], q["w13_scales"], E, 2 * F, off, pad,
+                             p(step.h13), st)
+        L.mxfp8_swiglu_quant(p(step.h13), M, F, 3, 1, p(step.h_rc), p(step.h_rs), p(step.h_cc), p(step.h_cs), st)
+        step.ops[4][3]()
+
+    def time_it(fn, n=5):
+        for _ in range(2):
+            fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(step.stream)
+        for _ in range(n):
+            fn()
+        e1.record(step.stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / n
+
+    ms_fused, ms_unfused = time_it(fwd_fused), time_it(fwd_unfused)
+    fused_vs_unfused = {"fused_fwd_ms": round(ms_fused, 3), "unfused_fwd_ms": round(ms_unfused, 3),
+                        "fused_speedup": round(ms_unfused / ms_fused, 4),
+                        "what": "x cast + FC1 (+SwiGLU + dual quant fused in the epilogue) + FC2, vs x cast + FC1 "
+                                "to bf16 h13 + standalone SwiGLU + dual quant + FC2; same padding (pad-matched)"}
+
     # dominant kernel and its roofline
     imax = int(np.argmax(mean_ms[: step.mlp_ops]))
     dname, dbound, dwork, _ = step.ops[imax]
@@ -536,7 +573,8 @@ def main():
         "mlp_no_weight_cast_tflops": round(useful / ((mlp_ms - cast_w_ms) * 1e-3) / 1e12, 2),
         "fwd_useful_tflops_prequantized_weights": round(6.0 * step.R * spec.D * spec.F / (fwd_ms * 1e-3) / 1e12, 2),
         "swiglu_quant_gbs": sw["GB/s"], "swiglu_quant_frac_hbm": sw["frac"],
-        "kernels": kernels, "roofline": roof, "clocks": clk, "gpu_launches": n_ops * args.steps,
+        "kernels": kernels, "fused_vs_unfused": fused_vs_unfused, "roofline": roof, "clocks": clk,
+        "gpu_launches": n_ops * args.steps,
         "e2e": e2e, "cpu_baseline": cpu, "source_hash": src_hash(),
     }
     if rank == 0:

@@ -280,6 +280,16 @@ int moe_mlp_fwd_q(const void* x, int64_t M, int64_t D, const mxmoe_qweights* qw,
                   void* y, const mxmoe_saved* saved,
                   void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* moe_mlp_fwd_unfused_q -- the unfused ("swiglu" plan) forward, the baseline
+ * of the fully-fused plan page ("Performance": +2.3 % / +5.0 % tokens/s over
+ * the pad-matched unfused MXFP8 baseline): FC1 grouped GEMM to a bf16 h13 in
+ * HBM, the standalone SwiGLU + dual quantization kernel, FC2.  Same arguments,
+ * outputs and workspace (which = 3) as moe_mlp_fwd_q; bitwise equal results. */
+int moe_mlp_fwd_unfused_q(const void* x, int64_t M, int64_t D, const mxmoe_qweights* qw, int E, int64_t F,
+                          const int32_t* expert_offsets, int pad_multiple,
+                          void* y, const mxmoe_saved* saved,
+                          void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
 int moe_mlp_bwd_q(const void* dy, int64_t M, int64_t D, const mxmoe_qweights* qw, int E, int64_t F,
                   const int32_t* expert_offsets, int pad_multiple,
                   const mxmoe_saved* saved,

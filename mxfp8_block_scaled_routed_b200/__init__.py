@@ -20,7 +20,7 @@ __all__ = [
     "mxfp8_grouped_gemm", "mxfp8_grouped_gemm_wgrad",
     "mxfp8_grouped_gemm_swiglu_quant", "mxfp8_grouped_gemm_dswiglu_quant",
     "moe_mlp_fwd", "moe_mlp_bwd", "device_error", "header_functions",
-    "make_qweights", "mxmoe_quantize_weights", "moe_mlp_fwd_q", "moe_mlp_bwd_q",
+    "make_qweights", "mxmoe_quantize_weights", "moe_mlp_fwd_q", "moe_mlp_bwd_q", "moe_mlp_fwd_unfused_q",
 ]
 
 ROW, COL = 1, 2
@@ -65,6 +65,8 @@ _SIGS = {
     "moe_mlp_fwd_noalloc": ([_P, _L, _L, _P, _P, _I, _L, _P, _I, _P, ctypes.POINTER(_Saved), _P], _I),
     "mxmoe_quantize_weights": ([_P, _P, _I, _L, _L, ctypes.POINTER(_QWeights), _P], _I),
     "mxmoe_selftest_wait_timeout": ([_P], _I),
+    "moe_mlp_fwd_unfused_q": ([_P, _L, _L, ctypes.POINTER(_QWeights), _I, _L, _P, _I, _P, ctypes.POINTER(_Saved),
+                               _P, _S, _P], _I),
     "moe_mlp_fwd_q": ([_P, _L, _L, ctypes.POINTER(_QWeights), _I, _L, _P, _I, _P, ctypes.POINTER(_Saved), _P, _S,
                        _P], _I),
     "moe_mlp_bwd_q": ([_P, _L, _L, ctypes.POINTER(_QWeights), _I, _L, _P, _I, ctypes.POINTER(_Saved), _P, _P, _P,
@@ -347,6 +349,22 @@ def moe_mlp_fwd_q(x, qw, offsets, pad_multiple=128, y=None, saved=None, workspac
     st, q = _saved_struct(saved), _qw_struct(qw)
     _check(lib().moe_mlp_fwd_q(_ptr(x), M, D, ctypes.byref(q), E, F, _ptr(offsets), pad_multiple, _ptr(y),
                                ctypes.byref(st), _ptr(ws), ws.numel(), _stream(x)))
+    return y, saved
+
+
+def moe_mlp_fwd_unfused_q(x, qw, offsets, pad_multiple=128, y=None, saved=None, workspace=None):
+    """Unfused forward (FC1 -> bf16 h13 -> standalone SwiGLU cast -> FC2). Returns (y, saved)."""
+    E = _offs(offsets)
+    _need(x, torch.bfloat16, "x")
+    M, D = x.shape
+    F = qw["w13_codes"].shape[1] // 2
+    dev = x.device
+    y = torch.empty(M, D, dtype=torch.bfloat16, device=dev) if y is None else y
+    saved = make_saved(M, D, F, dev) if saved is None else saved
+    ws = _u8((workspace_bytes(M, D, E, F, 3),), dev) if workspace is None else workspace
+    st, q = _saved_struct(saved), _qw_struct(qw)
+    _check(lib().moe_mlp_fwd_unfused_q(_ptr(x), M, D, ctypes.byref(q), E, F, _ptr(offsets), pad_multiple, _ptr(y),
+                                       ctypes.byref(st), _ptr(ws), ws.numel(), _stream(x)))
     return y, saved
 
 

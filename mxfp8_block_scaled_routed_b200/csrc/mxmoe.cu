@@ -775,6 +775,30 @@ int moe_mlp_fwd_q(const void* x, int64_t M, int64_t D, const mxmoe_qweights* qw,
   return fwd_core(x, M, D, *qw, E, F, expert_offsets, pad_multiple, y, saved, w, stream);
 }
 
+int moe_mlp_fwd_unfused_q(const void* x, int64_t M, int64_t D, const mxmoe_qweights* qw, int E, int64_t F,
+                          const int32_t* expert_offsets, int pad_multiple, void* y, const mxmoe_saved* saved,
+                          void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  MX_TRY(check_mlp_shapes(M, D, E, F, expert_offsets, pad_multiple));
+  MX_TRY(check_ptrs({{"x", x}, {"y", y}}));
+  MX_TRY(check_qweights(qw, true, false));
+  MX_TRY(check_saved(saved));
+  FwdWs w;
+  const size_t need = carve_fwd(nullptr, M, D, E, F, &w, false);
+  if (!workspace || workspace_bytes < need)
+    return fail(MXMOE_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed", workspace_bytes, need);
+  carve_fwd(align_ws(workspace), M, D, E, F, &w, false);
+  MX_TRY(quantize_tokens(x, M, D, expert_offsets + E, w.x_rc, w.x_rs, saved->x_col_codes, saved->x_col_scales,
+                         stream));
+  // FC1 to a bf16 h13 in HBM ([gate | up] columns of the plain W13 rows)
+  MX_TRY(gemm_ragged_m(w.x_rc, w.x_rs, M, D, qw->w13_codes, qw->w13_scales, E, 2 * F, expert_offsets, pad_multiple,
+                       saved->h13, stream));
+  // standalone SwiGLU + dual quantization of the rows below offsets[E]
+  MX_TRY(launch_cast<true>(saved->h13, 1, M, F, MXFP8_ROW | MXFP8_COL, MXFP8_SCALE_MMA, w.h_rc, w.h_rs,
+                           saved->h_col_codes, saved->h_col_scales, expert_offsets + E, stream));
+  return gemm_ragged_m(w.h_rc, w.h_rs, M, F, qw->w2_codes, qw->w2_scales, E, D, expert_offsets, pad_multiple, y,
+                       stream);
+}
+
 int moe_mlp_bwd_q(const void* dy, int64_t M, int64_t D, const mxmoe_qweights* qw, int E, int64_t F,
                   const int32_t* expert_offsets, int pad_multiple, const mxmoe_saved* saved, void* dx, void* dw13,
                   void* dw2, void* workspace, size_t workspace_bytes, cudaStream_t stream) {

@@ -283,3 +283,38 @@ def test_dsv3_full_size_step_gemms_on_oracle_operands():
     dw13 = mxk.mxfp8_grouped_gemm_wgrad(gt, gs, xt, xs, off, spec.pad)
     assert_gemm_close(bf16_np(dw13[e]), rb["dw13"], "dW13 (a9)")
     assert mxk.device_error() == 0
+
+
+@pytest.mark.parametrize("name", ["tiny", "dsv3_16b"])
+def test_unfused_plan_forward_equals_fused_bitwise(name):
+    """The unfused "swiglu" plan (FC1 -> bf16 h13 in HBM -> standalone SwiGLU +
+    dual quant -> FC2) and the fused FC1 epilogue give the same bits
+    (SwiGLU-boundary page: fused forward bitwise equal to the standalone cast)."""
+    inp = synth.make_moe_inputs(name, 5)
+    off = torch.from_numpy(inp.routing.offsets).to(DEV)
+    pad = inp.spec.pad
+    x, w13, w2 = inp.x.to(DEV), inp.w13.to(DEV), inp.w2.to(DEV)
+    qw = mxk.mxmoe_quantize_weights(w13, w2)
+    yf, sf = mxk.moe_mlp_fwd_q(x, qw, off, pad)
+    yu, su = mxk.moe_mlp_fwd_unfused_q(x, qw, off, pad)
+    torch.cuda.synchronize()
+    M = int(inp.routing.offsets[-1])
+    assert torch.equal(yf[:M], yu[:M])
+    assert torch.equal(sf["h13"][:M], su["h13"][:M])
+    for k in ("h_col_codes", "h_col_scales", "x_col_codes", "x_col_scales"):
+        assert torch.equal(sf[k], su[k]), k
+
+
+def test_dense_feedforward_is_the_one_expert_case():
+    """E = 1 (a dense SwiGLU FeedForward in MXFP8) against the oracle."""
+    spec = synth.Spec("dense", 1, 256, 384, 300, 1, 128, None, 0, 0.05)
+    inp = synth.make_moe_inputs(spec, 6)
+    y, saved, dx, dw13, dw2 = _run(inp)
+    x, w13, w2, dy = _np(inp)
+    off = inp.routing.offsets
+    rf = mx.moe_mlp_fwd(x, w13, w2, off)
+    rb = mx.moe_mlp_bwd(dy, rf, x, w13, w2, off)
+    assert_gemm_close(bf16_np(y), rf["y"], "y")
+    assert_gemm_close(bf16_np(dx), rb["dx"], "dx")
+    assert_gemm_close(bf16_np(dw13), rb["dw13"], "dw13")
+    assert_gemm_close(bf16_np(dw2), rb["dw2"], "dw2")
