@@ -6,3 +6,4 @@ the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 no code.
 """
 from . import mx  # noqa: F401
+from . import routing  # noqa: F401

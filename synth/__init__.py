@@ -40,6 +40,7 @@ class Routing:
     src_token: np.ndarray     # [M] source token of each row, -1 for pad rows
     M: int                    # rows of the buffer (= offsets[-1])
     R: int                    # real rows (tokens * top_k)
+    topk: np.ndarray | None = None   # [T, k] drawn expert ids (None for explicit counts)
 
 
 @dataclasses.dataclass
@@ -99,6 +100,7 @@ def make_routing(spec: Spec, seed: int = 0, counts_override=None) -> Routing:
         # explicit per-expert real counts (tests of edge cases); tokens are
         # assigned round-robin so that every row has a source token.
         counts = np.asarray(counts_override, dtype=np.int64)
+        choice = None
         lists = []
         t = 0
         for e in range(E):
@@ -129,7 +131,8 @@ def make_routing(spec: Spec, seed: int = 0, counts_override=None) -> Routing:
         o = offsets[e]
         src[o:o + counts[e]] = lists[e]
     return Routing(counts=counts, padded=padded, offsets=offsets, src_token=src,
-                   M=M, R=int(counts.sum()))
+                   M=M, R=int(counts.sum()),
+                   topk=None if choice is None else choice.astype(np.int32))
 
 
 def normal(g: np.random.Generator, shape, std=1.0, outlier_frac=0.0, outlier_mul=1.0):
@@ -171,6 +174,24 @@ def make_moe_inputs(spec: Spec | str, seed: int = 0, counts_override=None,
     if with_dy:
         dy[real] = normal(g, (int(real.sum()), spec.D), spec.dy_std)
     return MoEInputs(spec, routing, to_bf16(x), to_bf16(w13), to_bf16(w2), to_bf16(dy))
+
+
+def router_weights(T: int, k: int, seed: int = 0) -> np.ndarray:
+    """[T, k] float32 combine weights: a softmax over k N(0,1) logits per token."""
+    g = rng(seed + 7)
+    z = g.standard_normal(size=(T, k))
+    w = np.exp(z - z.max(axis=1, keepdims=True))
+    return (w / w.sum(axis=1, keepdims=True)).astype(np.float32)
+
+
+def topk_ids(T: int, k: int, E: int, seed: int = 0, zipf_s: float | None = None) -> np.ndarray:
+    """[T, k] int32 distinct expert ids per token (uniform or Zipf popularity)."""
+    spec = Spec("route", E, 32, 32, T, k, 32, zipf_s, 0, 1.0)
+    g = rng(seed)
+    p = popularity(spec, g)
+    with np.errstate(divide="ignore"):
+        keys = np.log(p)[None, :] + g.gumbel(size=(T, E))
+    return np.argsort(-keys, axis=1)[:, :k].astype(np.int32)
 
 
 def make_swiglu_input(rows: int = 16384, F: int = 4096, seed: int = 0) -> torch.Tensor:
