@@ -169,6 +169,18 @@ class Step:
         self.c_in = inp.cast_x
         self.c_rc, self.c_rs = u8(CAST_ROWS, CAST_COLS), u8(CAST_ROWS, CAST_COLS // 32)
         self.c_deq = bf(CAST_ROWS, CAST_COLS)
+        # dispatcher: routing of the same draw, token rows, router weights, upstream token gradient
+        self.T, self.k = s.tokens, s.top_k
+        self.topk = torch.from_numpy(inp.routing.topk).to(dev)
+        self.x_tok = inp.x_tok
+        self.dout = inp.dout_tok
+        self.wr = inp.router_w
+        self.r_off = torch.empty(E + 1, dtype=torch.int32, device=dev)
+        self.r_row_slot = torch.empty(M, dtype=torch.int32, device=dev)
+        self.r_slot_row = torch.empty(self.T * self.k, dtype=torch.int32, device=dev)
+        self.r_ws = u8(max(16, int(self.L.mxmoe_route_workspace_size(self.T, self.k, E))))
+        self.comb = bf(self.T, D)
+        self.dwr = torch.empty(self.T, self.k, dtype=torch.float32, device=dev)
         self.stream = torch.cuda.current_stream(dev)
         self._build()
 
@@ -176,6 +188,7 @@ class Step:
         L, p = self.L, (lambda t: torch.Tensor.data_ptr(t))
         st = self.stream.cuda_stream
         M, D, E, F, pad = self.M, self.D, self.E, self.F, self.pad
+        T, k, R = self.T, self.k, self.R
         off = p(self.off)
         q = {k: p(v) for k, v in self.qw.items()}
         self.ops = [
@@ -218,6 +231,25 @@ class Step:
              lambda: L.mxfp8_dequantize(p(self.c_rc), p(self.c_rs), CAST_ROWS, CAST_COLS, p(self.c_deq), st)),
         ]
         self.mlp_ops = 10
+        # dispatcher around the MLP (same routing; m_cap = the padded rows), timed
+        # after the step, outside the step's own clock
+        self.disp_ops = [
+            ("route", "hbm", 4.0 * (3 * T * k + M + 2 * E),
+             lambda: L.mxmoe_route(p(self.topk), T, k, E, pad, M, p(self.r_off), p(self.r_row_slot),
+                                   p(self.r_slot_row), p(self.r_ws), self.r_ws.numel(), st)),
+            ("permute_quant_x_dual", "hbm", 2.0 * R * D + 2.0625 * M * D,
+             lambda: L.mxmoe_permute_quant(p(self.x_tok), T, D, p(self.r_row_slot), k, None, M, p(self.r_off) + 4 * E,
+                                           3, 1, p(self.x_rc), p(self.x_rs), p(self.x_cc), p(self.x_cs), st)),
+            ("permute_quant_dy_weighted", "hbm", 2.0 * R * D + 2.0625 * M * D,
+             lambda: L.mxmoe_permute_quant(p(self.dout), T, D, p(self.r_row_slot), k, p(self.wr), M,
+                                           p(self.r_off) + 4 * E, 3, 1, p(self.dy_rc), p(self.dy_rs), p(self.dy_cc),
+                                           p(self.dy_cs), st)),
+            ("combine_y", "hbm", 2.0 * R * D + 2.0 * T * D,
+             lambda: L.mxmoe_unpermute_combine(p(self.y), M, D, p(self.r_slot_row), p(self.wr), T, k, p(self.comb), st)),
+            ("combine_weight_grad", "hbm", 2.0 * R * D + 2.0 * T * D,
+             lambda: L.mxmoe_combine_weight_grad(p(self.dout), p(self.y), M, D, p(self.r_slot_row), T, k, p(self.dwr),
+                                                 st)),
+        ]
 
     def run(self, events=None):
         for i, (name, _, _, fn) in enumerate(self.ops):
@@ -244,6 +276,9 @@ def make_inputs(workload: str, seed: int, dev):
     inp.swiglu_h13 = h.to(torch.bfloat16)
     del h, idx
     inp.cast_x = torch.randn(CAST_ROWS, CAST_COLS, generator=gen, device=dev).to(torch.bfloat16)
+    s = inp.spec
+    inp.dout_tok = (torch.randn(s.tokens, s.D, generator=gen, device=dev) * s.dy_std).to(torch.bfloat16)
+    inp.router_w = torch.from_numpy(synth.router_weights(s.tokens, s.top_k, seed)).to(dev)
     return inp
 
 
@@ -467,6 +502,17 @@ def main():
                         "what": "x cast + FC1 (+SwiGLU + dual quant fused in the epilogue) + FC2, vs x cast + FC1 "
                                 "to bf16 h13 + standalone SwiGLU + dual quant + FC2; same padding (pad-matched)"}
 
+    # dispatcher kernels (not part of the step): each timed alone, n launches
+    dispatcher = {}
+    for name, bound, work, fn in step.disp_ops:
+        if fn() != 0:
+            raise RuntimeError(f"{name}: {step.L.mxmoe_last_error().decode()}")
+        ms = time_it(fn, n=10)
+        ach = work / (ms * 1e-3) / 1e9
+        dispatcher[name] = {"ms": round(ms, 4), "GB/s": round(ach, 1), "frac": round(ach / hbm, 3)}
+    if mxk.device_error() != 0:
+        raise RuntimeError("device error in the dispatcher kernels")
+
     # dominant kernel and its roofline
     imax = int(np.argmax(mean_ms[: step.mlp_ops]))
     dname, dbound, dwork, _ = step.ops[imax]
@@ -573,7 +619,7 @@ def main():
         "mlp_no_weight_cast_tflops": round(useful / ((mlp_ms - cast_w_ms) * 1e-3) / 1e12, 2),
         "fwd_useful_tflops_prequantized_weights": round(6.0 * step.R * spec.D * spec.F / (fwd_ms * 1e-3) / 1e12, 2),
         "swiglu_quant_gbs": sw["GB/s"], "swiglu_quant_frac_hbm": sw["frac"],
-        "kernels": kernels, "fused_vs_unfused": fused_vs_unfused, "roofline": roof, "clocks": clk,
+        "kernels": kernels, "fused_vs_unfused": fused_vs_unfused, "dispatcher": dispatcher, "roofline": roof, "clocks": clk,
         "gpu_launches": n_ops * args.steps,
         "e2e": e2e, "cpu_baseline": cpu, "source_hash": src_hash(),
     }

@@ -331,6 +331,84 @@ int moe_mlp_fwd_noalloc(const void* x, int64_t M, int64_t D,
                         const int32_t* expert_offsets, int pad_multiple,
                         void* y, const mxmoe_saved* saved, cudaStream_t stream);
 
+/* -------------------------------------------------------------------------
+ * Token dispatcher around the MLP.
+ *
+ * The fully-fused plan page ("What it adds") installs a dispatcher that pads
+ * each expert's token rows to a multiple of pad_multiple, and the
+ * SwiGLU-boundary page ("Usage") has it produce the padded expert-major
+ * layout the kernels consume.  Slot s = t*top_k + j is token t's j-th routed
+ * copy, sent to expert topk_ids[s].  Expert e's segment
+ * [offsets[e], offsets[e+1]) lists its slots in ascending slot order
+ * (ascending token order), then pad rows up to the next multiple of
+ * pad_multiple; an expert with no slot has an empty segment.
+ *
+ *   forward   rows   = permute(x)               row m <- x[row_slot[m] / top_k]
+ *             out[t] = sum_j w[t,j] * y[slot_row[t*top_k + j]]    (combine)
+ *   backward  dy[row(t,j)] = bf16(w[t,j] * dout[t])               (permute, weighted)
+ *             dw[t,j]      = <dout[t], y[row(t,j)]>              (combine_weight_grad)
+ *             dx_tok[t]    = sum_j dx[row(t,j)]                  (combine, no weights)
+ * ------------------------------------------------------------------------- */
+
+/* Rows a layout can need: T*top_k real rows plus at most pad_multiple-1 pad
+ * rows for each expert that receives a slot, rounded up to a multiple of 128
+ * (the grouped GEMMs' row tile).  Host-only arithmetic; returns -1 for
+ * non-positive or overflowing arguments. */
+int64_t mxmoe_route_capacity(int64_t T, int top_k, int E, int pad_multiple);
+
+/* Bytes of device workspace mxmoe_route needs: 4 * E * ceil(T*top_k / 4096). */
+size_t mxmoe_route_workspace_size(int64_t T, int top_k, int E);
+
+/* Build the padded expert-major layout from a top-k routing (three kernels:
+ * per-chunk histogram, padded scan, stable ranking).
+ *   topk_ids  DEVICE int32 [T, top_k], ids in [0, E) (ids outside raise
+ *             MXMOE_ERR_ARG in mxmoe_device_error and their slot gets row -1)
+ *   E <= 1024, pad_multiple >= 1, T*top_k < 2^31
+ *   m_cap     rows of row_slot (use mxmoe_route_capacity); a routing that
+ *             needs more raises MXMOE_ERR_SHAPE on the device and rows past
+ *             m_cap are not written
+ *   offsets   DEVICE int32 [E+1] out: offsets[0] = 0, offsets[E] = M
+ *   row_slot  DEVICE int32 [m_cap] out: slot of each row, -1 for pad rows and
+ *             for rows [M, m_cap)
+ *   slot_row  DEVICE int32 [T*top_k] out: row of each slot
+ * The result is deterministic (a stable counting sort). */
+int mxmoe_route(const int32_t* topk_ids, int64_t T, int top_k, int E, int pad_multiple, int64_t m_cap,
+                int32_t* offsets, int32_t* row_slot, int32_t* slot_row,
+                void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Gather token rows into the layout and MXFP8-quantize them in the same pass
+ * (the x cast of the forward, and with slot_weights the dY cast of the
+ * backward): row m is x_tokens[row_slot[m] / top_k] ([T, D] bf16), zero when
+ * row_slot[m] < 0; with slot_weights (DEVICE fp32 [T*top_k], may be NULL)
+ * it is bf16(slot_weights[s] * x) with one fp32 product per element.
+ *   m_cap % 128 == 0 and D % 128 == 0 with MXFP8_SCALE_MMA, D % 32 == 0 and
+ *   m_cap % 32 == 0 otherwise; x_tokens 16-byte aligned.
+ *   rows_dev  DEVICE int32* (may be NULL), e.g. offsets + E: rows at or past
+ *             *rows_dev are neither read nor written
+ *   outputs   as mxfp8_quantize for a [m_cap, D] matrix (COL codes [D, m_cap]).
+ * A slot >= T*top_k in row_slot raises MXMOE_ERR_OFFSETS and that row reads as
+ * zero. */
+int mxmoe_permute_quant(const void* x_tokens, int64_t T, int64_t D, const int32_t* row_slot, int top_k,
+                        const float* slot_weights, int64_t m_cap, const int32_t* rows_dev,
+                        int modes, int scale_layout,
+                        uint8_t* row_codes, uint8_t* row_scales,
+                        uint8_t* col_codes, uint8_t* col_scales, cudaStream_t stream);
+
+/* out[t] = bf16( sum_j w[t*top_k+j] * y[slot_row[t*top_k+j]] ), fp32
+ * accumulation in j order; w = 1 when slot_weights is NULL.  y [m_rows, D]
+ * bf16, out [T, D] bf16, D % 8 == 0, top_k <= 64, 16-byte aligned y/out.
+ * slot_row entries of -1 contribute nothing; entries >= m_rows raise
+ * MXMOE_ERR_OFFSETS and contribute nothing. */
+int mxmoe_unpermute_combine(const void* y, int64_t m_rows, int64_t D, const int32_t* slot_row,
+                            const float* slot_weights, int64_t T, int top_k, void* out, cudaStream_t stream);
+
+/* dweights[t*top_k+j] = <dout[t], y[slot_row[t*top_k+j]]> in fp32 (0 for a
+ * slot whose row is -1).  dout [T, D] bf16, y [m_rows, D] bf16, D % 8 == 0,
+ * 16-byte aligned. */
+int mxmoe_combine_weight_grad(const void* dout, const void* y, int64_t m_rows, int64_t D,
+                              const int32_t* slot_row, int64_t T, int top_k, float* dweights,
+                              cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

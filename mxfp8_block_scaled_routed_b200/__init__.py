@@ -21,6 +21,8 @@ __all__ = [
     "mxfp8_grouped_gemm_swiglu_quant", "mxfp8_grouped_gemm_dswiglu_quant",
     "moe_mlp_fwd", "moe_mlp_bwd", "device_error", "header_functions",
     "make_qweights", "mxmoe_quantize_weights", "moe_mlp_fwd_q", "moe_mlp_bwd_q", "moe_mlp_fwd_unfused_q",
+    "mxmoe_route_capacity", "mxmoe_route", "mxmoe_permute_quant", "mxmoe_unpermute_combine",
+    "mxmoe_combine_weight_grad",
 ]
 
 ROW, COL = 1, 2
@@ -71,6 +73,12 @@ _SIGS = {
                        _P], _I),
     "moe_mlp_bwd_q": ([_P, _L, _L, ctypes.POINTER(_QWeights), _I, _L, _P, _I, ctypes.POINTER(_Saved), _P, _P, _P,
                        _P, _S, _P], _I),
+    "mxmoe_route_capacity": ([_L, _I, _I, _I], _L),
+    "mxmoe_route_workspace_size": ([_L, _I, _I], _S),
+    "mxmoe_route": ([_P, _L, _I, _I, _I, _L, _P, _P, _P, _P, _S, _P], _I),
+    "mxmoe_permute_quant": ([_P, _L, _L, _P, _I, _P, _L, _P, _I, _I, _P, _P, _P, _P, _P], _I),
+    "mxmoe_unpermute_combine": ([_P, _L, _L, _P, _P, _L, _I, _P, _P], _I),
+    "mxmoe_combine_weight_grad": ([_P, _P, _L, _L, _P, _L, _I, _P, _P], _I),
 }
 
 _lib = None
@@ -383,3 +391,81 @@ def moe_mlp_bwd_q(dy, qw, offsets, saved, pad_multiple=128, dx=None, dw13=None, 
     _check(lib().moe_mlp_bwd_q(_ptr(dy), M, D, ctypes.byref(q), E, F, _ptr(offsets), pad_multiple,
                                ctypes.byref(st), _ptr(dx), _ptr(dw13), _ptr(dw2), _ptr(ws), ws.numel(), _stream(dy)))
     return dx, dw13, dw2
+
+
+# ----------------------------------------------------------------------------- dispatcher
+def mxmoe_route_capacity(T: int, top_k: int, E: int, pad_multiple: int) -> int:
+    """Rows a padded expert-major layout of T tokens x top_k can need (multiple of 128)."""
+    cap = lib().mxmoe_route_capacity(T, top_k, E, pad_multiple)
+    if cap < 0:
+        raise ValueError("invalid routing sizes")
+    return int(cap)
+
+
+def mxmoe_route(topk_ids: torch.Tensor, E: int, pad_multiple: int, m_cap: int | None = None):
+    """int32 [T, top_k] expert ids -> dict(offsets [E+1], row_slot [m_cap], slot_row [T*top_k])."""
+    _need(topk_ids, torch.int32, "topk_ids")
+    T, k = topk_ids.shape
+    if m_cap is None:
+        m_cap = mxmoe_route_capacity(T, k, E, pad_multiple)
+    dev = topk_ids.device
+    out = {"offsets": torch.empty(E + 1, dtype=torch.int32, device=dev),
+           "row_slot": torch.empty(m_cap, dtype=torch.int32, device=dev),
+           "slot_row": torch.empty(T * k, dtype=torch.int32, device=dev)}
+    nws = lib().mxmoe_route_workspace_size(T, k, E)
+    ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=dev)
+    _check(lib().mxmoe_route(_ptr(topk_ids), T, k, E, pad_multiple, m_cap, _ptr(out["offsets"]),
+                             _ptr(out["row_slot"]), _ptr(out["slot_row"]), _ptr(ws), ws.numel(), _stream(topk_ids)))
+    return out
+
+
+def mxmoe_permute_quant(x_tokens: torch.Tensor, row_slot: torch.Tensor, top_k: int, weights=None,
+                        rows_dev=None, modes: int = ROW | COL, scale_layout: int = MMA):
+    """Gather token rows into the padded layout and MXFP8-quantize them (optionally weighted)."""
+    _need(x_tokens, torch.bfloat16, "x_tokens")
+    _need(row_slot, torch.int32, "row_slot")
+    if weights is not None:
+        _need(weights, torch.float32, "weights")
+    if rows_dev is not None:
+        _need(rows_dev, torch.int32, "rows_dev")
+    T, D = x_tokens.shape
+    m = row_slot.numel()
+    dev = x_tokens.device
+    out = {}
+    if modes & ROW:
+        out["row_codes"] = _u8((m, D), dev)
+        out["row_scales"] = _u8((m, D // 32), dev) if scale_layout == PLAIN else _u8((m * D // 32,), dev)
+    if modes & COL:
+        out["col_codes"] = _u8((D, m), dev)
+        out["col_scales"] = _u8((D, m // 32), dev) if scale_layout == PLAIN else _u8((m * D // 32,), dev)
+    _check(lib().mxmoe_permute_quant(_ptr(x_tokens), T, D, _ptr(row_slot), top_k, _ptr(weights), m,
+                                     _ptr(rows_dev), modes, scale_layout,
+                                     _ptr(out.get("row_codes")), _ptr(out.get("row_scales")),
+                                     _ptr(out.get("col_codes")), _ptr(out.get("col_scales")), _stream(x_tokens)))
+    return out
+
+
+def mxmoe_unpermute_combine(y: torch.Tensor, slot_row: torch.Tensor, top_k: int, weights=None, out=None):
+    """out[t] = sum_j w[t, j] * y[slot_row[t*top_k + j]] (bf16 [T, D])."""
+    _need(y, torch.bfloat16, "y")
+    _need(slot_row, torch.int32, "slot_row")
+    if weights is not None:
+        _need(weights, torch.float32, "weights")
+    T = slot_row.numel() // top_k
+    if out is None:
+        out = torch.empty(T, y.shape[1], dtype=torch.bfloat16, device=y.device)
+    _check(lib().mxmoe_unpermute_combine(_ptr(y), y.shape[0], y.shape[1], _ptr(slot_row), _ptr(weights), T, top_k,
+                                         _ptr(out), _stream(y)))
+    return out
+
+
+def mxmoe_combine_weight_grad(dout: torch.Tensor, y: torch.Tensor, slot_row: torch.Tensor, top_k: int):
+    """d w[t, j] = <dout[t], y[slot_row[t*top_k + j]]> as fp32 [T, top_k]."""
+    _need(dout, torch.bfloat16, "dout")
+    _need(y, torch.bfloat16, "y")
+    _need(slot_row, torch.int32, "slot_row")
+    T, D = dout.shape
+    dw = torch.empty(T, top_k, dtype=torch.float32, device=dout.device)
+    _check(lib().mxmoe_combine_weight_grad(_ptr(dout), _ptr(y), y.shape[0], D, _ptr(slot_row), T, top_k,
+                                           _ptr(dw), _stream(dout)))
+    return dw

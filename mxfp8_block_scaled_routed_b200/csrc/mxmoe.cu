@@ -15,6 +15,7 @@
 #include "../../include/mxmoe.h"
 #include "gemm.cuh"
 #include "quant.cuh"
+#include "route.cuh"
 
 using namespace mxmoe;
 
@@ -124,6 +125,13 @@ int make_operand_map(CUtensorMap* map, const uint8_t* base, int64_t rows, int64_
   return MXMOE_OK;
 }
 
+struct GatherArgs {
+  const int32_t* row_slot;
+  const float* slot_weight;
+  int64_t n_slots;
+  int top_k;
+};
+
 // 3-D bf16 cast input [batch, rows, ld], box 128 x 128 x 1, no swizzle, zero fill
 // past the edges.
 int make_cast_map(CUtensorMap* map, const void* base, int64_t batch, int64_t rows, int64_t ld) {
@@ -140,14 +148,32 @@ int make_cast_map(CUtensorMap* map, const void* base, int64_t batch, int64_t row
   return MXMOE_OK;
 }
 
-template <bool kSwiglu>
+// 2-D bf16 token matrix [tokens, ld] for four-row gathers: box 128 x 1, no
+// swizzle, zero fill past the column edge.
+int make_gather_map(CUtensorMap* map, const void* base, int64_t tokens, int64_t ld) {
+  EncodeTiledFn enc;
+  MX_TRY(get_encode(&enc));
+  cuuint64_t dims[2] = {cuuint64_t(ld), cuuint64_t(tokens > 0 ? tokens : 1)};
+  cuuint64_t strides[1] = {cuuint64_t(ld * 2)};
+  cuuint32_t box[2] = {128, 1};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MXMOE_ERR_CUDA, "cuTensorMapEncodeTiled (gather) failed (%d)", int(r));
+  return MXMOE_OK;
+}
+
+template <int kMode>
 int launch_cast(const void* in, int64_t batch, int64_t rows, int64_t cols, int modes, int layout, uint8_t* rc,
-                uint8_t* rs, uint8_t* cc, uint8_t* cs, const int32_t* dev_rows, cudaStream_t stream) {
-  using C = CastCfg<kSwiglu>;
+                uint8_t* rs, uint8_t* cc, uint8_t* cs, const int32_t* dev_rows, cudaStream_t stream,
+                const GatherArgs* g = nullptr) {
+  using C = CastCfg<kMode>;
+  constexpr bool kSwiglu = kMode == kCastSwiglu;
   DevInfo* d;
   MX_TRY(device_info(&d));
-  const int bit = kSwiglu ? 8 : 7;
-  auto kern = mx_cast_kernel<kSwiglu>;
+  const int bit = kMode == kCastPlain ? 7 : kMode == kCastSwiglu ? 8 : 13;   // distinct from the GEMM bits
+  auto kern = mx_cast_kernel<kMode>;
   if (!(d->attr_set & (1u << bit))) {
     MX_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem),
                   "cudaFuncSetAttribute");
@@ -155,8 +181,20 @@ int launch_cast(const void* in, int64_t batch, int64_t rows, int64_t cols, int m
     d->attr_set |= (1u << bit);
   }
   CUtensorMap map;
-  MX_TRY(make_cast_map(&map, in, batch, rows, kSwiglu ? 2 * cols : cols));
+  if constexpr (kMode == kCastGather) {
+    if (!g) return fail(MXMOE_ERR_ARG, "gather cast without a slot table");
+    MX_TRY(make_gather_map(&map, in, g->n_slots / g->top_k, cols));
+  } else
+    MX_TRY(make_cast_map(&map, in, batch, rows, kSwiglu ? 2 * cols : cols));
   CastArgs a;
+  memset(&a, 0, sizeof(a));
+  if (g) {
+    a.src = static_cast<const uint16_t*>(in);
+    a.row_slot = g->row_slot;
+    a.slot_weight = g->slot_weight;
+    a.n_slots = g->n_slots;
+    a.top_k = g->top_k;
+  }
   a.rows = rows;
   a.cols = cols;
   a.batch = batch;
@@ -335,15 +373,15 @@ int quantize_impl(const void* x, int64_t batch, int64_t rows, int64_t cols, int 
     return MXMOE_OK;
   }
   if (swiglu)
-    return launch_cast<true>(x, 1, rows, cols, modes, layout, rc, rs, cc, cs, nullptr, stream);
-  return launch_cast<false>(x, batch, rows, cols, modes, layout, rc, rs, cc, cs, nullptr, stream);
+    return launch_cast<kCastSwiglu>(x, 1, rows, cols, modes, layout, rc, rs, cc, cs, nullptr, stream);
+  return launch_cast<kCastPlain>(x, batch, rows, cols, modes, layout, rc, rs, cc, cs, nullptr, stream);
 }
 
 // Cast of the token buffer used inside the composites: rows at or past
 // offsets[E] (read on the device) are neither read nor written.
 int quantize_tokens(const void* x, int64_t rows, int64_t cols, const int32_t* rows_dev, uint8_t* rc, uint8_t* rs,
                     uint8_t* cc, uint8_t* cs, cudaStream_t stream) {
-  return launch_cast<false>(x, 1, rows, cols, MXFP8_ROW | MXFP8_COL, MXFP8_SCALE_MMA, rc, rs, cc, cs, rows_dev,
+  return launch_cast<kCastPlain>(x, 1, rows, cols, MXFP8_ROW | MXFP8_COL, MXFP8_SCALE_MMA, rc, rs, cc, cs, rows_dev,
                             stream);
 }
 
@@ -632,6 +670,22 @@ int mxfp8_dequantize(const uint8_t* codes, const uint8_t* scales, int64_t rows, 
   DevInfo* d;
   MX_TRY(device_info(&d));
   const int64_t n = rows * cols;
+  const bool vec = cols % 16 == 0 && reinterpret_cast<uintptr_t>(codes) % 16 == 0 &&
+                   reinterpret_cast<uintptr_t>(out) % 16 == 0;
+  if (vec) {
+    const int64_t n16 = n / 16, cpr = cols / 16, ncb = (cols + 31) / 32;
+    const int64_t blocks = std::min<int64_t>((n16 + 255) / 256, int64_t(d->sms) * 8);
+    const auto* c4 = reinterpret_cast<const uint4*>(codes);
+    auto* o4 = static_cast<uint4*>(out);
+    if (n16 < (int64_t(1) << 31))
+      mx_dequant16_kernel<uint32_t><<<unsigned(blocks), 256, 0, stream>>>(c4, scales, uint32_t(n16), uint32_t(cpr),
+                                                                          uint32_t(ncb), o4);
+    else
+      mx_dequant16_kernel<uint64_t><<<unsigned(blocks), 256, 0, stream>>>(c4, scales, uint64_t(n16), uint64_t(cpr),
+                                                                          uint64_t(ncb), o4);
+    MX_CHECK_CUDA(cudaGetLastError(), "dequant launch");
+    return MXMOE_OK;
+  }
   const int64_t blocks = (n + 255) / 256;
   if (blocks > 0x7FFFFFFF) return fail(MXMOE_ERR_SHAPE, "tensor too large");
   mx_dequant_kernel<<<unsigned(blocks), 256, 0, stream>>>(codes, scales, rows, cols, static_cast<uint16_t*>(out));
@@ -793,7 +847,7 @@ int moe_mlp_fwd_unfused_q(const void* x, int64_t M, int64_t D, const mxmoe_qweig
   MX_TRY(gemm_ragged_m(w.x_rc, w.x_rs, M, D, qw->w13_codes, qw->w13_scales, E, 2 * F, expert_offsets, pad_multiple,
                        saved->h13, stream));
   // standalone SwiGLU + dual quantization of the rows below offsets[E]
-  MX_TRY(launch_cast<true>(saved->h13, 1, M, F, MXFP8_ROW | MXFP8_COL, MXFP8_SCALE_MMA, w.h_rc, w.h_rs,
+  MX_TRY(launch_cast<kCastSwiglu>(saved->h13, 1, M, F, MXFP8_ROW | MXFP8_COL, MXFP8_SCALE_MMA, w.h_rc, w.h_rs,
                            saved->h_col_codes, saved->h_col_scales, expert_offsets + E, stream));
   return gemm_ragged_m(w.h_rc, w.h_rs, M, F, qw->w2_codes, qw->w2_scales, E, D, expert_offsets, pad_multiple, y,
                        stream);
@@ -846,6 +900,126 @@ int moe_mlp_fwd_noalloc(const void* x, int64_t M, int64_t D, const void* w13, co
   }
   return moe_mlp_fwd(x, M, D, w13, w2, E, F, expert_offsets, pad_multiple, y, saved, ws,
                      MXMOE_NOALLOC_SCRATCH_BYTES, stream);
+}
+
+// ---------------------------------------------------------------- dispatcher
+int64_t mxmoe_route_capacity(int64_t T, int top_k, int E, int pad_multiple) {
+  if (T < 0 || top_k <= 0 || E <= 0 || pad_multiple <= 0) return -1;
+  if (T > (int64_t(1) << 40) / top_k) return -1;
+  const int64_t n = T * top_k;
+  const int64_t busy = n < E ? n : E;
+  const int64_t cap = n + busy * (pad_multiple - 1);
+  return (cap + 127) / 128 * 128;
+}
+
+size_t mxmoe_route_workspace_size(int64_t T, int top_k, int E) {
+  if (T <= 0 || top_k <= 0 || E <= 0) return 0;
+  const int64_t chunks = (T * top_k + kRouteChunk - 1) / kRouteChunk;
+  return size_t(chunks) * size_t(E) * 4;
+}
+
+int mxmoe_route(const int32_t* topk_ids, int64_t T, int top_k, int E, int pad_multiple, int64_t m_cap,
+                int32_t* offsets, int32_t* row_slot, int32_t* slot_row, void* workspace, size_t workspace_bytes,
+                cudaStream_t stream) {
+  if (!offsets) return fail(MXMOE_ERR_NULL, "offsets is NULL");
+  if (T < 0 || top_k <= 0) return fail(MXMOE_ERR_SHAPE, "T=%lld top_k=%d", (long long)T, top_k);
+  if (E <= 0 || E > kRouteMaxE) return fail(MXMOE_ERR_SHAPE, "E=%d must be in [1, %d]", E, kRouteMaxE);
+  if (pad_multiple <= 0) return fail(MXMOE_ERR_ARG, "pad_multiple=%d must be positive", pad_multiple);
+  if (m_cap < 0 || m_cap >= (int64_t(1) << 31)) return fail(MXMOE_ERR_SHAPE, "m_cap=%lld", (long long)m_cap);
+  if (T > ((int64_t(1) << 31) - 1) / top_k) return fail(MXMOE_ERR_SHAPE, "T*top_k must be below 2^31");
+  const int64_t n = T * top_k;
+  if (n + int64_t(E) * (pad_multiple - 1) >= (int64_t(1) << 31))
+    return fail(MXMOE_ERR_SHAPE, "T*top_k + E*(pad_multiple-1) must be below 2^31");
+  if (n > 0 && (!topk_ids || !slot_row)) return fail(MXMOE_ERR_NULL, "topk_ids/slot_row is NULL");
+  if (m_cap > 0 && !row_slot) return fail(MXMOE_ERR_NULL, "row_slot is NULL");
+  const size_t need = mxmoe_route_workspace_size(T, top_k, E);
+  if (need > 0 && (!workspace || workspace_bytes < need))
+    return fail(MXMOE_ERR_WORKSPACE, "mxmoe_route needs %zu workspace bytes, got %zu", need, workspace_bytes);
+  if (need > 0 && reinterpret_cast<uintptr_t>(workspace) % 4 != 0)
+    return fail(MXMOE_ERR_ALIGN, "workspace is not 4-byte aligned");
+  DevInfo* d;
+  MX_TRY(device_info(&d));
+  const int chunks = int((n + kRouteChunk - 1) / kRouteChunk);
+  auto* counts = static_cast<int32_t*>(workspace);
+  if (chunks > 0) {
+    route_count_kernel<<<chunks, kRouteThreads, 0, stream>>>(topk_ids, n, E, counts);
+    MX_CHECK_CUDA(cudaGetLastError(), "route count launch");
+  }
+  route_scan_kernel<<<1, kRouteThreads, 0, stream>>>(counts, chunks, E, pad_multiple, m_cap, offsets, row_slot);
+  MX_CHECK_CUDA(cudaGetLastError(), "route scan launch");
+  if (chunks > 0) {
+    const int smem = E * 4 + 32 * E * 2;
+    if (smem > 48 * 1024 && !(d->attr_set & (1u << 14))) {
+      MX_CHECK_CUDA(cudaFuncSetAttribute(route_assign_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
+                    "cudaFuncSetAttribute(route)");
+      std::lock_guard<std::mutex> lk(g_mu);
+      d->attr_set |= (1u << 14);
+    }
+    route_assign_kernel<<<chunks, kRouteThreads, smem, stream>>>(topk_ids, n, E, counts, m_cap, row_slot, slot_row);
+    MX_CHECK_CUDA(cudaGetLastError(), "route assign launch");
+  }
+  return MXMOE_OK;
+}
+
+int mxmoe_permute_quant(const void* x_tokens, int64_t T, int64_t D, const int32_t* row_slot, int top_k,
+                        const float* slot_weights, int64_t m_cap, const int32_t* rows_dev, int modes,
+                        int scale_layout, uint8_t* row_codes, uint8_t* row_scales, uint8_t* col_codes,
+                        uint8_t* col_scales, cudaStream_t stream) {
+  if (!x_tokens || !row_slot) return fail(MXMOE_ERR_NULL, "x_tokens/row_slot is NULL");
+  if (T < 0 || top_k <= 0 || D <= 0 || m_cap <= 0)
+    return fail(MXMOE_ERR_SHAPE, "T=%lld top_k=%d D=%lld m_cap=%lld", (long long)T, top_k, (long long)D,
+                (long long)m_cap);
+  if (modes < 1 || modes > 3) return fail(MXMOE_ERR_ARG, "modes=%d must be MXFP8_ROW, MXFP8_COL or both", modes);
+  if (scale_layout != MXFP8_SCALE_PLAIN && scale_layout != MXFP8_SCALE_MMA)
+    return fail(MXMOE_ERR_ARG, "scale_layout=%d invalid", scale_layout);
+  const bool row = modes & MXFP8_ROW, col = modes & MXFP8_COL;
+  if (row && (!row_codes || !row_scales)) return fail(MXMOE_ERR_NULL, "row_codes/row_scales NULL with MXFP8_ROW");
+  if (col && (!col_codes || !col_scales)) return fail(MXMOE_ERR_NULL, "col_codes/col_scales NULL with MXFP8_COL");
+  if (D % 32 != 0 || m_cap % 32 != 0)
+    return fail(MXMOE_ERR_SHAPE, "D=%lld and m_cap=%lld must be multiples of 32", (long long)D, (long long)m_cap);
+  if (scale_layout == MXFP8_SCALE_MMA && (D % 128 != 0 || m_cap % 128 != 0))
+    return fail(MXMOE_ERR_SHAPE, "MMA scale layout needs D and m_cap multiples of 128");
+  if (!aligned16(x_tokens) || (row && !aligned16(row_codes)) || (col && !aligned16(col_codes)))
+    return fail(MXMOE_ERR_ALIGN, "x_tokens and code buffers must be 16-byte aligned");
+  GatherArgs g{row_slot, slot_weights, T * top_k, top_k};
+  return launch_cast<kCastGather>(x_tokens, 1, m_cap, D, modes, scale_layout, row_codes, row_scales, col_codes,
+                                  col_scales, rows_dev, stream, &g);
+}
+
+static int check_combine_args(const void* a, const void* y, const int32_t* slot_row, const void* out, int64_t m_rows,
+                              int64_t D, int64_t T, int top_k) {
+  if (!a || !y || !slot_row || !out) return fail(MXMOE_ERR_NULL, "a required pointer is NULL");
+  if (m_rows < 0 || D <= 0 || D % 8 != 0 || T < 0 || top_k <= 0 || top_k > 64)
+    return fail(MXMOE_ERR_SHAPE, "m_rows=%lld D=%lld (multiple of 8) T=%lld top_k=%d (1..64)", (long long)m_rows,
+                (long long)D, (long long)T, top_k);
+  if (T > 0x7FFFFFFF) return fail(MXMOE_ERR_SHAPE, "T=%lld too large", (long long)T);
+  if (!aligned16(a) || !aligned16(y)) return fail(MXMOE_ERR_ALIGN, "bf16 tensors must be 16-byte aligned");
+  return MXMOE_OK;
+}
+
+int mxmoe_unpermute_combine(const void* y, int64_t m_rows, int64_t D, const int32_t* slot_row,
+                            const float* slot_weights, int64_t T, int top_k, void* out, cudaStream_t stream) {
+  MX_TRY(check_combine_args(out, y, slot_row, out, m_rows, D, T, top_k));
+  DevInfo* d;
+  MX_TRY(device_info(&d));
+  if (T == 0) return MXMOE_OK;
+  combine_kernel<<<unsigned(T), 256, 0, stream>>>(static_cast<const uint16_t*>(y), m_rows, slot_row, slot_weights,
+                                                 top_k, D, static_cast<uint16_t*>(out));
+  MX_CHECK_CUDA(cudaGetLastError(), "combine launch");
+  return MXMOE_OK;
+}
+
+int mxmoe_combine_weight_grad(const void* dout, const void* y, int64_t m_rows, int64_t D, const int32_t* slot_row,
+                              int64_t T, int top_k, float* dweights, cudaStream_t stream) {
+  MX_TRY(check_combine_args(dout, y, slot_row, dweights, m_rows, D, T, top_k));
+  DevInfo* d;
+  MX_TRY(device_info(&d));
+  if (T == 0) return MXMOE_OK;
+  combine_weight_grad_kernel<<<unsigned(T), 256, 0, stream>>>(static_cast<const uint16_t*>(dout),
+                                                             static_cast<const uint16_t*>(y), m_rows, slot_row,
+                                                             top_k, D, dweights);
+  MX_CHECK_CUDA(cudaGetLastError(), "combine weight-grad launch");
+  return MXMOE_OK;
 }
 
 }  // extern "C"

@@ -35,23 +35,43 @@ struct CastArgs {
   uint8_t* col_codes;
   uint8_t* col_scales;
   const int32_t* dev_rows;  // optional: rows at or past *dev_rows are neither read nor written
+  // gather mode: row m of the quantized matrix is token row_slot[m] / top_k
+  // of src ([*, cols] bf16, row stride cols), zero where row_slot[m] < 0;
+  // with slot_weight, that row times slot_weight[row_slot[m]] rounded to bf16
+  const uint16_t* src;
+  const int32_t* row_slot;
+  const float* slot_weight;
+  int64_t n_slots;
+  int top_k;
 };
+
+constexpr int kCastPlain = 0;    // TMA tiles of a [batch, rows, cols] tensor
+constexpr int kCastSwiglu = 1;   // TMA gate + up tiles, h = silu(gate) * up
+constexpr int kCastGather = 2;   // rows gathered by bulk copies through a slot table
 
 constexpr int kTile = 128;
 constexpr int kCastConsumers = 256;                 // 8 warps
 constexpr int kCastThreads = kCastConsumers + 32;   // + 1 TMA producer warp
 constexpr int kTileBytes = kTile * kTile * 2;       // one bf16 128 x 128 tile
 
-template <bool kSwiglu>
+template <int kMode>
 struct CastCfg {
+  static constexpr bool kSwiglu = kMode == kCastSwiglu;
   static constexpr int kStages = kSwiglu ? 1 : 2;       // SwiGLU: two CTAs per SM take turns instead
   static constexpr int kStageBytes = kSwiglu ? 2 * kTileBytes : kTileBytes;
   static constexpr int kOffColStage = kStages * kStageBytes;         // COL codes of one tile, 128 x 128 B
   static constexpr int kOffScales = kOffColStage + kTile * kTile;    // ROW then COL scale bytes, 512 B each
-  static constexpr int kOffBars = kOffScales + 1024;
+  static constexpr int kOffWeights = kOffScales + 1024;              // gather: per-row weights of each stage
+  static constexpr int kOffPadMask = kOffWeights + (kMode == kCastGather ? kStages * kTile * 4 : 0);
+  static constexpr int kOffBars = kOffPadMask + (kMode == kCastGather ? kStages * 16 : 0);
   static constexpr int kSmem = kOffBars + 2 * kStages * 8 + 128;     // + alignment slack
   static constexpr int kCtasPerSm = 2;
 };
+
+// bf16(w * x) for the two bf16 of a word (fp32 product, one rounding to bf16)
+__device__ __forceinline__ uint32_t scale_bf16x2(uint32_t x, float w) {
+  return pack_bf16x2(w * bf16lo_to_f32(x), w * bf16hi_to_f32(x));
+}
 
 __device__ __forceinline__ uint32_t swiglu_pair(uint32_t g, uint32_t u) {
   float h0 = silu_mul(bf16lo_to_f32(g), bf16lo_to_f32(u));
@@ -120,22 +140,37 @@ __device__ __forceinline__ uint32_t col_quant32(const uint32_t (&w)[32], uint4 (
 // SwiGLU: the gate and up tiles arrive together; the ROW pass computes
 // h = bf16(silu(gate) * up), quantizes it and parks it over the gate tile
 // for the COL pass (one barrier among the 256 consumer threads).
-template <bool kSwiglu>
-__global__ void __launch_bounds__(kCastThreads, CastCfg<kSwiglu>::kCtasPerSm)
+template <int kMode>
+__global__ void __launch_bounds__(kCastThreads, CastCfg<kMode>::kCtasPerSm)
 mx_cast_kernel(const __grid_constant__ CUtensorMap tin, const CastArgs p) {
-  using C = CastCfg<kSwiglu>;
+  using C = CastCfg<kMode>;
+  constexpr bool kSwiglu = kMode == kCastSwiglu, kGather = kMode == kCastGather;
+  const bool weighted = kGather && p.slot_weight != nullptr;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBars);
   uint8_t* cstage = smem + C::kOffColStage;     // COL codes: column c at c*128, 16-byte chunk k at k ^ ((c>>1)&7)
   uint8_t* rsc = smem + C::kOffScales;          // ROW scales of the tile: [128 rows][4 blocks]
   uint8_t* csc = rsc + 512;                     // COL scales of the tile: [128 cols][4 blocks]
+  float* wsm = reinterpret_cast<float*>(smem + C::kOffWeights);   // gather: [stage][row] weights
+  uint32_t* padm = reinterpret_cast<uint32_t*>(smem + C::kOffPadMask);   // gather: [stage][4] pad-row bits
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t rows = p.rows, cols = p.cols;
   const int64_t ntiles = p.batch * p.tiles_r * p.tiles_c;
   int64_t rows_lim = rows;
   if (p.dev_rows != nullptr) rows_lim = min(rows, int64_t(*p.dev_rows));
   const bool do_row = p.modes & 1, do_col = p.modes & 2;
+  // Tile sequence of this CTA.  TMA modes: grid stride.  Gather: a contiguous
+  // run of the valid tiles (row bands below the device row limit), so that a
+  // row band's slots are read once for all of its column tiles.
+  int64_t t_begin = blockIdx.x, t_end = ntiles, t_step = gridDim.x;
+  if constexpr (kGather) {
+    const int64_t nvalid_tiles = min(ntiles, (max(rows_lim, int64_t(0)) + kTile - 1) / kTile * p.tiles_c);
+    const int64_t per = (nvalid_tiles + gridDim.x - 1) / gridDim.x;
+    t_begin = int64_t(blockIdx.x) * per;
+    t_end = min(nvalid_tiles, t_begin + per);
+    t_step = 1;
+  }
 
   if (tid == 0) {
     for (int s = 0; s < C::kStages; ++s) {
@@ -147,6 +182,74 @@ mx_cast_kernel(const __grid_constant__ CUtensorMap tin, const CastArgs p) {
   __syncthreads();
 
   const int64_t per_batch = p.tiles_r * p.tiles_c;
+  if (kGather && warp == 8) {
+    // ---------------- gather producer: lane g owns rows 4g..4g+3 of each
+    // tile and fetches them with one four-row gather (tensor map over the
+    // token matrix, box 128 x 1).  A pad row borrows a real row of its group
+    // (the consumers zero it); a group without a real row is not fetched.
+    if (lane == 0) sm100::prefetch_tmap(&tin);
+    int stage = 0;
+    uint32_t phase = 0;
+    int64_t band = -1;
+    int trow[4] = {0, 0, 0, 0};
+    float wreg[4] = {0.f, 0.f, 0.f, 0.f};
+    uint32_t padword = 0, ngroups = 0;
+    bool fetch = false;
+    for (int64_t t = t_begin; t < t_end; t += t_step) {
+      const int64_t r0 = (t / p.tiles_c) * kTile, c0 = (t % p.tiles_c) * kTile;
+      if (r0 >= rows_lim) continue;
+      if (r0 != band) {                           // new row band: its slots, once
+        band = r0;
+        const int vrows = int(min(int64_t(kTile), rows_lim - r0));
+        uint32_t pad = 0;
+        int first = -1;
+        int tok[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int rr = 4 * lane + i;
+          int64_t sl = rr < vrows ? int64_t(p.row_slot[r0 + rr]) : -1;
+          if (sl >= p.n_slots) {
+            raise_device_error(4);
+            sl = -1;
+          }
+          tok[i] = sl >= 0 ? int(sl / p.top_k) : -1;
+          if (sl < 0) pad |= 1u << i;
+          if (sl >= 0 && first < 0) first = tok[i];
+          wreg[i] = (weighted && sl >= 0) ? p.slot_weight[sl] : 0.0f;
+        }
+        fetch = first >= 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) trow[i] = tok[i] >= 0 ? tok[i] : first;
+        ngroups = __popc(__ballot_sync(0xffffffffu, fetch));
+        // pad bits of rows 32w..32w+31 gathered into lane 8w
+        uint32_t wd = pad << (4 * (lane & 7));
+        wd |= __shfl_xor_sync(0xffffffffu, wd, 1);
+        wd |= __shfl_xor_sync(0xffffffffu, wd, 2);
+        wd |= __shfl_xor_sync(0xffffffffu, wd, 4);
+        padword = wd;
+      }
+      bool ok = true;
+      if (lane == 0) ok = sm100::mbar_wait(sm100::smem_u32(&bars[C::kStages + stage]), phase ^ 1);
+      if (!__shfl_sync(0xffffffffu, ok, 0)) {
+        if (lane == 0) raise_device_error(7);
+        break;
+      }
+      if (weighted) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) wsm[stage * kTile + 4 * lane + i] = wreg[i];
+      }
+      if ((lane & 7) == 0) padm[stage * 4 + (lane >> 3)] = padword;
+      __syncwarp();
+      const uint32_t fb = sm100::smem_u32(&bars[stage]);
+      if (lane == 0) sm100::mbar_arrive_expect_tx(fb, ngroups * 4u * kTile * 2u);
+      __syncwarp();
+      if (fetch)
+        sm100::tma_gather4(sm100::smem_u32(smem + stage * C::kStageBytes + lane * 4 * 256), &tin, fb, int(c0),
+                           trow[0], trow[1], trow[2], trow[3]);
+      if (++stage == C::kStages) { stage = 0; phase ^= 1; }
+    }
+    return;
+  }
   if (warp == 8) {
     // ---------------- producer
     if (lane == 0) {
@@ -178,7 +281,7 @@ mx_cast_kernel(const __grid_constant__ CUtensorMap tin, const CastArgs p) {
   const bool plain = p.mma_layout == 0;
   int stage = 0;
   uint32_t phase = 0;
-  for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x) {
+  for (int64_t t = t_begin; t < t_end; t += t_step) {
     const int64_t b = t / per_batch, rem = t - b * per_batch;
     const int64_t r0 = (rem / p.tiles_c) * kTile, c0 = (rem % p.tiles_c) * kTile;
     if (r0 >= rows_lim) continue;
@@ -188,10 +291,23 @@ mx_cast_kernel(const __grid_constant__ CUtensorMap tin, const CastArgs p) {
     }
     uint8_t* tile = smem + stage * C::kStageBytes;
     const int vrows = int(min(int64_t(kTile), rows_lim - r0));   // valid rows of the tile (multiple of 32 for COL)
+    if constexpr (kGather) {
+      // pad rows (and rows past the limit) hold a borrowed row or nothing: zero them
+      const uint4 pm = *reinterpret_cast<const uint4*>(padm + stage * 4);
+      if ((pm.x | pm.y | pm.z | pm.w) != 0u) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const int idx = q * kCastConsumers + tid, row = idx >> 4;   // row = 8q + tid/16: word q/4
+          const uint32_t w = q < 4 ? (q < 2 ? pm.x : pm.y) : (q < 6 ? pm.z : pm.w);
+          if ((w >> (row & 31)) & 1u) reinterpret_cast<uint4*>(tile)[idx] = make_uint4(0u, 0u, 0u, 0u);
+        }
+        sm100::named_bar_sync(1, kCastConsumers);
+      }
+    }
     const int vcols = int(min(int64_t(kTile), cols - c0));       // valid columns (multiple of 32)
 
     // ---- ROW pass (and SwiGLU): codes straight to global, scales to shared
-    if (do_row || kSwiglu) {
+    if (do_row || kSwiglu || weighted) {
       const int64_t col = c0 + ch * 8;
       const int64_t Rb = b * rows + r0 + rr0;                    // matrix row of chunk 0
       uint8_t* rcode = p.row_codes + Rb * cols + col;            // advances 16 rows per chunk
@@ -208,6 +324,14 @@ mx_cast_kernel(const __grid_constant__ CUtensorMap tin, const CastArgs p) {
           v.w = swiglu_pair(v.w, u.w);
           *reinterpret_cast<uint4*>(srow) = v;
         }
+        if (weighted) {
+          const float w = wsm[stage * kTile + rr];
+          v.x = scale_bf16x2(v.x, w);
+          v.y = scale_bf16x2(v.y, w);
+          v.z = scale_bf16x2(v.z, w);
+          v.w = scale_bf16x2(v.w, w);
+          *reinterpret_cast<uint4*>(srow) = v;
+        }
         if (do_row) {
           uint32_t byte;
           const uint2 q = row_quant8(v, &byte);
@@ -218,7 +342,7 @@ mx_cast_kernel(const __grid_constant__ CUtensorMap tin, const CastArgs p) {
         }
       }
     }
-    if (kSwiglu && do_col) sm100::named_bar_sync(1, kCastConsumers);   // h parked for the COL pass
+    if ((kSwiglu || weighted) && do_col) sm100::named_bar_sync(1, kCastConsumers);   // h parked for the COL pass
 
     // ---- COL pass: codes into the shared staging tile
     if (do_col) {
@@ -240,7 +364,10 @@ mx_cast_kernel(const __grid_constant__ CUtensorMap tin, const CastArgs p) {
         }
       }
     }
-    // the input tile is no longer read: hand it back to the producer
+    // the input tile is no longer read: hand it back to the producer (after
+    // ordering this thread's shared-memory writes into it, if any, before the
+    // producer's next asynchronous copy into the same bytes)
+    if constexpr (kSwiglu || kGather) sm100::fence_proxy_async();
     __syncwarp();
     if (lane == 0) sm100::mbar_arrive(sm100::smem_u32(&bars[C::kStages + stage]));
     if (++stage == C::kStages) { stage = 0; phase ^= 1; }
@@ -262,12 +389,18 @@ mx_cast_kernel(const __grid_constant__ CUtensorMap tin, const CastArgs p) {
       if (!plain) {
         // the tile's 128 rows x 4 blocks are exactly one 512-byte MMA atom:
         // atom byte (r%32)*16 + (r/32)*4 + kb  <-  staged byte r*4 + kb
-        if (tid < 32 && vrows == kTile && vcols == kTile) {
-          uint32_t wv[4];
+        const int64_t atom = ((b * rows + r0) >> 7) * (cols >> 7) + (c0 >> 7);
+        if (vrows == kTile) {
+          if (tid < 32) {
+            uint32_t wv[4];
 #pragma unroll
-          for (int g = 0; g < 4; ++g) wv[g] = *reinterpret_cast<const uint32_t*>(rsc + (g * 32 + tid) * 4);
-          const int64_t atom = ((b * rows + r0) >> 7) * (cols >> 7) + (c0 >> 7);
-          *reinterpret_cast<uint4*>(p.row_scales + atom * 512 + tid * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+            for (int g = 0; g < 4; ++g) wv[g] = *reinterpret_cast<const uint32_t*>(rsc + (g * 32 + tid) * 4);
+            *reinterpret_cast<uint4*>(p.row_scales + atom * 512 + tid * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+          }
+        } else if (tid < vrows) {
+          // a tile cut by the device row limit: only its valid rows' 4 bytes
+          *reinterpret_cast<uint32_t*>(p.row_scales + atom * 512 + (tid & 31) * 16 + (tid >> 5) * 4) =
+              *reinterpret_cast<const uint32_t*>(rsc + tid * 4);
         }
       } else if (tid < vrows) {
         const int nb = vcols >> 5;
@@ -281,13 +414,19 @@ mx_cast_kernel(const __grid_constant__ CUtensorMap tin, const CastArgs p) {
     }
     if (do_col) {
       if (!plain) {
-        if (tid >= 64 && tid < 96 && vrows == kTile && vcols == kTile) {
-          const int l = tid - 64;
-          uint32_t wv[4];
+        const int64_t atom = ((b * cols + c0) >> 7) * (rows >> 7) + (r0 >> 7);
+        if (vrows == kTile) {
+          if (tid >= 64 && tid < 96) {
+            const int l = tid - 64;
+            uint32_t wv[4];
 #pragma unroll
-          for (int g = 0; g < 4; ++g) wv[g] = *reinterpret_cast<const uint32_t*>(csc + (g * 32 + l) * 4);
-          const int64_t atom = ((b * cols + c0) >> 7) * (rows >> 7) + (r0 >> 7);
-          *reinterpret_cast<uint4*>(p.col_scales + atom * 512 + l * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+            for (int g = 0; g < 4; ++g) wv[g] = *reinterpret_cast<const uint32_t*>(csc + (g * 32 + l) * 4);
+            *reinterpret_cast<uint4*>(p.col_scales + atom * 512 + l * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+          }
+        } else if (tid >= 128) {
+          // a tile cut by the device row limit: only the valid 32-row blocks
+          const int c = tid - 128;
+          for (int k = 0; k < (vrows >> 5); ++k) p.col_scales[atom * 512 + (c & 31) * 16 + (c >> 5) * 4 + k] = csc[c * 4 + k];
         }
       } else if (tid >= 128 && tid - 128 < vcols) {
         const int c = tid - 128;
@@ -357,6 +496,56 @@ mx_dequant_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__
   const float s = e8m0_to_f32(scales[r * ncb + (c >> 5)]);
   const float v = e4m3_to_f32(codes[i]) * s;
   out[i] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+}
+
+// Vector path (cols % 16 == 0, 16-B aligned codes and output): one thread
+// per 16 codes, which share one scale.  The E4M3 bits are placed in an fp32
+// word so that the word reads as the code's value times 2^-120 (normals and
+// subnormals alike); multiplying by 2^(byte-7) -- split in two factors when
+// that power is not an fp32 normal -- then rounds the exact product
+// code*2^(byte-127) once, exactly as the scalar path does.
+__device__ __forceinline__ uint32_t dequant_pair(uint32_t b0, uint32_t b1, float m1, float m2) {
+  const float y0 = __uint_as_float(((b0 & 0x80u) << 24) | ((b0 & 0x7Fu) << 20)) * m1 * m2;
+  const float y1 = __uint_as_float(((b1 & 0x80u) << 24) | ((b1 & 0x7Fu) << 20)) * m1 * m2;
+  const __nv_bfloat162 h = __floats2bfloat162_rn(y0, y1);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+__device__ __forceinline__ void dequant_word(uint32_t w, float m1, float m2, uint32_t& lo, uint32_t& hi) {
+  lo = dequant_pair(w & 0xFFu, (w >> 8) & 0xFFu, m1, m2);
+  hi = dequant_pair((w >> 16) & 0xFFu, w >> 24, m1, m2);
+  // S.1111.111 is the E4M3 NaN; those lanes become the canonical bf16 NaN.
+  if ((((w & 0x7F7F7F7Fu) + 0x01010101u) & 0x80808080u) != 0u) {
+    if ((w & 0x7Fu) == 0x7Fu) lo = (lo & 0xFFFF0000u) | 0x7FFFu;
+    if ((w & 0x7F00u) == 0x7F00u) lo = (lo & 0x0000FFFFu) | 0x7FFF0000u;
+    if ((w & 0x7F0000u) == 0x7F0000u) hi = (hi & 0xFFFF0000u) | 0x7FFFu;
+    if ((w & 0x7F000000u) == 0x7F000000u) hi = (hi & 0x0000FFFFu) | 0x7FFF0000u;
+  }
+}
+
+template <typename Idx>
+__global__ void __launch_bounds__(256)
+mx_dequant16_kernel(const uint4* __restrict__ codes, const uint8_t* __restrict__ scales, Idx n16, Idx chunks_per_row,
+                    Idx ncb, uint4* __restrict__ out) {
+  const Idx stride = Idx(gridDim.x) * blockDim.x;
+  for (Idx i = Idx(blockIdx.x) * blockDim.x + threadIdx.x; i < n16; i += stride) {
+    const Idx r = i / chunks_per_row, c = i - r * chunks_per_row;
+    const uint32_t byte = __ldg(scales + r * ncb + (c >> 1));
+    const uint4 q = __ldcs(codes + i);
+    uint4 o0, o1;
+    if (byte == 0xFFu) {
+      o0 = o1 = make_uint4(0x7FFF7FFFu, 0x7FFF7FFFu, 0x7FFF7FFFu, 0x7FFF7FFFu);
+    } else {
+      const float m1 = __uint_as_float(byte <= 134u ? (byte + 120u) << 23 : (byte - 7u) << 23);
+      const float m2 = byte <= 134u ? 1.0f : __uint_as_float(254u << 23);
+      dequant_word(q.x, m1, m2, o0.x, o0.y);
+      dequant_word(q.y, m1, m2, o0.z, o0.w);
+      dequant_word(q.z, m1, m2, o1.x, o1.y);
+      dequant_word(q.w, m1, m2, o1.z, o1.w);
+    }
+    __stcs(out + 2 * i, o0);
+    __stcs(out + 2 * i + 1, o1);
+  }
 }
 
 }  // namespace mxmoe

@@ -103,6 +103,16 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* tmap, uint
       "l"(tmap), "r"(x), "r"(y), "r"(z), "r"(bar)
       : "memory");
 }
+// Four rows of a 2-D tensor map (box one row high) at arbitrary row indices,
+// landing back to back in shared memory.
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const void* tmap, uint32_t bar, int x, int r0, int r1,
+                                            int r2, int r3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
+      "l"(tmap), "r"(bar), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+      : "memory");
+}
 // CTA-pair form: data lands in this CTA's shared memory, the transaction
 // bytes are credited to `bar_cluster`, a shared::cluster mbarrier address that
 // may belong to the peer CTA (the even CTA's barrier in this kernel).

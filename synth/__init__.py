@@ -155,6 +155,7 @@ class MoEInputs:
     w13: torch.Tensor        # [E, 2F, D] bf16, rows 0..F-1 gate (w1), F..2F-1 up (w3)
     w2: torch.Tensor         # [E, D, F] bf16
     dy: torch.Tensor         # [M, D] bf16, pad rows zero
+    x_tok: torch.Tensor | None = None   # [tokens, D] bf16 token rows before routing (device draw only)
 
 
 def make_moe_inputs(spec: Spec | str, seed: int = 0, counts_override=None,
@@ -227,7 +228,8 @@ def device_moe_inputs(spec: Spec | str, seed: int = 0, device="cuda"):
     src = torch.from_numpy(routing.src_token).to(device)
     real = src >= 0
     x = torch.zeros(routing.M, D, device=device, dtype=torch.bfloat16)
-    x[real] = tok[src[real]].to(torch.bfloat16)
+    x_tok = tok.to(torch.bfloat16)
+    x[real] = x_tok[src[real]]
     del tok
     w13 = torch.empty(E, 2 * F, D, device=device, dtype=torch.bfloat16)
     w2 = torch.empty(E, D, F, device=device, dtype=torch.bfloat16)
@@ -237,4 +239,4 @@ def device_moe_inputs(spec: Spec | str, seed: int = 0, device="cuda"):
     dy = torch.zeros(routing.M, D, device=device, dtype=torch.bfloat16)
     nreal = int(real.sum())
     dy[real] = (torch.randn(nreal, D, generator=gen, device=device) * spec.dy_std).to(torch.bfloat16)
-    return MoEInputs(spec, routing, x, w13, w2, dy)
+    return MoEInputs(spec, routing, x, w13, w2, dy, x_tok)

@@ -97,3 +97,42 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(mxk, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="not built"):
         mxk.lib()
+
+
+def test_route_capacity_and_workspace_arithmetic(L):
+    # 16384 tokens x top-8 over 256 experts padded to 256: at most 255 pad rows per expert
+    assert L.mxmoe_route_capacity(16384, 8, 256, 256) == 131072 + 256 * 255
+    assert L.mxmoe_route_capacity(3, 2, 3, 4) == 128                 # 6 + 3*3 = 15 -> one 128-row tile
+    assert L.mxmoe_route_capacity(1, 1, 64, 128) == 128               # only one expert can be busy
+    assert L.mxmoe_route_capacity(0, 8, 64, 256) == 0
+    assert L.mxmoe_route_capacity(-1, 8, 64, 256) == -1
+    assert L.mxmoe_route_capacity(10, 2, 4, 0) == -1
+    assert L.mxmoe_route_workspace_size(16384, 8, 256) == 32 * 256 * 4
+    assert L.mxmoe_route_workspace_size(1, 1, 7) == 7 * 4
+    assert L.mxmoe_route_workspace_size(0, 1, 7) == 0
+
+
+def test_dispatcher_rejects(L):
+    s = L.mxmoe_route(P(FAKE), 16, 2, 2048, 128, 1024, P(FAKE), P(FAKE), P(FAKE), P(FAKE), 1 << 20, None)
+    assert s == 2 and "E=2048" in _err(L)
+    s = L.mxmoe_route(P(FAKE), 16, 2, 8, 0, 1024, P(FAKE), P(FAKE), P(FAKE), P(FAKE), 1 << 20, None)
+    assert s == 9
+    s = L.mxmoe_route(P(FAKE), 16, 2, 8, 128, 1024, P(FAKE), P(FAKE), P(FAKE), P(FAKE), 4, None)
+    assert s == 8 and "workspace" in _err(L)
+    s = L.mxmoe_route(None, 16, 2, 8, 128, 1024, P(FAKE), P(FAKE), P(FAKE), P(FAKE), 1 << 20, None)
+    assert s == 1
+    s = L.mxmoe_permute_quant(P(FAKE), 16, 200, P(FAKE), 2, None, 256, None, 3, 1, P(FAKE), P(FAKE), P(FAKE),
+                              P(FAKE), None)
+    assert s == 2
+    s = L.mxmoe_permute_quant(P(MIS), 16, 256, P(FAKE), 2, None, 256, None, 3, 1, P(FAKE), P(FAKE), P(FAKE),
+                              P(FAKE), None)
+    assert s == 3
+    s = L.mxmoe_permute_quant(P(FAKE), 16, 256, P(FAKE), 2, None, 256, None, 2, 1, P(FAKE), P(FAKE), None,
+                              P(FAKE), None)
+    assert s == 1
+    s = L.mxmoe_unpermute_combine(P(FAKE), 256, 100, P(FAKE), None, 16, 2, P(FAKE), None)
+    assert s == 2 and "D=100" in _err(L)
+    s = L.mxmoe_unpermute_combine(P(FAKE), 256, 128, P(FAKE), None, 16, 65, P(FAKE), None)
+    assert s == 2
+    s = L.mxmoe_combine_weight_grad(P(FAKE), P(MIS), 256, 128, P(FAKE), 16, 2, P(FAKE), None)
+    assert s == 3

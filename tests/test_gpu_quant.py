@@ -148,3 +148,31 @@ def test_dequantize_endpoints_and_random():
     np.testing.assert_array_equal(got[fin], ref[fin])
     assert got[0, 0] == 2.0 ** -123
     assert np.isnan(got[1]).all()
+
+
+def _dequant_check(codes, scales):
+    out = mxk.mxfp8_dequantize(torch.from_numpy(codes).to(DEV), torch.from_numpy(scales).to(DEV))
+    got = bf16_np(out)
+    ref = mx.round_to_bf16(mx.dequantize_rows(codes, scales))
+    np.testing.assert_array_equal(np.isnan(got), np.isnan(ref))
+    fin = ~np.isnan(ref)
+    np.testing.assert_array_equal(got[fin], ref[fin])
+
+
+def test_dequantize_every_code_with_every_scale():
+    # Row r carries scale byte r on all its blocks and every code once: all
+    # 65536 (code, scale) pairs, including overflow to inf, bf16 subnormals
+    # and both NaN sources.
+    codes = np.tile(np.arange(256, dtype=np.uint8), (256, 1))
+    scales = np.repeat(np.arange(256, dtype=np.uint8)[:, None], 8, axis=1)
+    _dequant_check(codes, scales)
+
+
+@pytest.mark.parametrize("rows,cols", [(37, 48), (130, 40), (5, 16), (2048, 7168)])
+def test_dequantize_shapes(rows, cols):
+    # cols % 32 == 16 (a half block at the row end), cols % 16 != 0 (scalar
+    # path) and a payload-sized tensor on the vector path.
+    g = np.random.default_rng(rows * 7 + cols)
+    codes = g.integers(0, 256, (rows, cols), dtype=np.uint8)
+    scales = g.integers(100, 150, (rows, (cols + 31) // 32), dtype=np.uint8)
+    _dequant_check(codes, scales)
