@@ -14,7 +14,8 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libmxmoe.so")
-SOURCES = [os.path.join(HERE, "csrc", f) for f in ("mxmoe.cu", "mx_common.cuh", "quant.cuh", "gemm.cuh", "sm100.cuh")]
+SOURCES = [os.path.join(HERE, "csrc", f)
+           for f in ("mxmoe.cu", "mx_common.cuh", "quant.cuh", "gemm.cuh", "sm100.cuh", "route.cuh")]
 HEADER = os.path.join(ROOT, "include", "mxmoe.h")
 
 

@@ -513,18 +513,37 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
       const uint32_t t_row = tmem_base + (uint32_t(q * 32) << 16) + acc * BN;
       uint32_t va[kChunks * 16];
       uint32_t vb[(kEpi == kEpiSwiGLU) ? kChunks * 16 : 1];
+      auto release = [&]() {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if constexpr (kPair) mbar_arrive_remote(tempty_bar(acc), 0); else mbar_arrive(tempty_bar(acc));
+        }
+        if (++acc == C::kAcc) { acc = 0; acc_phase ^= 1; }
+      };
+      if constexpr (kEpi == kEpiBF16) {
+        // all of this warp's columns in flight at once, one wait, and the
+        // accumulator goes back to the MMA warp before any conversion: with a
+        // single accumulator the next tile's MMAs start that much sooner
+        uint32_t r[kChunks][32];
 #pragma unroll
-      for (int c = 0; c < kChunks; ++c) drain32_bf16(t_row + h * kHalf + 32 * c, va + 16 * c);
-      if constexpr (kEpi == kEpiSwiGLU) {
+        for (int c = 0; c < kChunks; ++c) tmem_ld_32x32b_x32(t_row + h * kHalf + 32 * c, r[c]);
+        tmem_wait_ld();
+        release();
 #pragma unroll
-        for (int c = 0; c < kChunks; ++c) drain32_bf16(t_row + 128 + h * kHalf + 32 * c, vb + 16 * c);
+        for (int c = 0; c < kChunks; ++c)
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            va[16 * c + j] = pack_bf16x2(__uint_as_float(r[c][2 * j]), __uint_as_float(r[c][2 * j + 1]));
+      } else {
+#pragma unroll
+        for (int c = 0; c < kChunks; ++c) drain32_bf16(t_row + h * kHalf + 32 * c, va + 16 * c);
+        if constexpr (kEpi == kEpiSwiGLU) {
+#pragma unroll
+          for (int c = 0; c < kChunks; ++c) drain32_bf16(t_row + 128 + h * kHalf + 32 * c, vb + 16 * c);
+        }
+        release();
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        if constexpr (kPair) mbar_arrive_remote(tempty_bar(acc), 0); else mbar_arrive(tempty_bar(acc));
-      }
-      if (++acc == C::kAcc) { acc = 0; acc_phase ^= 1; }
 
       if constexpr (kEpi == kEpiBF16) {
         const int64_t orow = (kMode == kRaggedK) ? int64_t(T.e) * p.rows_a + row0 : row0;
