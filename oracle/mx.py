@@ -18,6 +18,11 @@ Everything is plain numpy in float64, written as the definition of each step:
   underflow is -0, code 0x80).
 * A block holding NaN or Inf gets scale byte 0xFF (the E8M0 NaN) and every
   element code 0x7F | sign (the E4M3 NaN).
+* E5M2 elements (A2E transport page, "quant_mode=4": the activation goes out
+  as E4M3 or E5M2 with its E8M0 block scale): same block rule with the E5M2
+  largest exponent 15 (floor(log2(amax)) - 15), nearest-even rounding onto the
+  E5M2 grid (subnormal spacing 2^-16), saturation at 57344, NaN/Inf blocks
+  -> 0xFF and codes 0x7F | sign.
 * E8M0 decode: byte b -> 2^(b-127) for b in [0, 254], 0xFF -> NaN; byte 0x00
   is 2^-127, not zero (A2E transport page, review "[P2] Handle the two E8M0
   endpoint encodings before shifting").
@@ -48,6 +53,8 @@ E4M3_EMAX = 8          # 448 = 1.75 * 2^8
 E8M0_BIAS = 127
 E8M0_NAN = 0xFF
 E4M3_NAN = 0x7F
+E5M2_MAX = 57344.0     # 1.75 * 2^15
+E5M2_EMAX = 15
 
 
 # ----------------------------------------------------------------------------
@@ -78,6 +85,33 @@ E4M3_TABLE = e4m3_decode_table()
 
 def e4m3_decode(codes: np.ndarray) -> np.ndarray:
     return E4M3_TABLE[np.asarray(codes, dtype=np.uint8)]
+
+
+def e5m2_decode_table() -> np.ndarray:
+    """All 256 E5M2 codes decoded from the format definition.
+
+    sign bit, 5-bit exponent (bias 15), 2-bit mantissa; exponent field 0 is
+    subnormal m/4 * 2^-14; exponent field 31 is infinity (m = 0) or NaN.
+    """
+    t = np.empty(256, dtype=np.float64)
+    for c in range(256):
+        s = -1.0 if c & 0x80 else 1.0
+        e = (c >> 2) & 0x1F
+        m = c & 0x3
+        if e == 0x1F:
+            t[c] = s * np.inf if m == 0 else np.nan
+        elif e == 0:
+            t[c] = s * (m / 4.0) * 2.0 ** -14
+        else:
+            t[c] = s * (1.0 + m / 4.0) * 2.0 ** (e - 15)
+    return t
+
+
+E5M2_TABLE = e5m2_decode_table()
+
+
+def e5m2_decode(codes: np.ndarray) -> np.ndarray:
+    return E5M2_TABLE[np.asarray(codes, dtype=np.uint8)]
 
 
 def e8m0_decode(b: np.ndarray) -> np.ndarray:
@@ -127,17 +161,18 @@ def f64_to_bf16_bits(x: np.ndarray) -> np.ndarray:
 # ----------------------------------------------------------------------------
 # MX quantization
 # ----------------------------------------------------------------------------
-def scale_byte(amax: np.ndarray) -> np.ndarray:
+def scale_byte(amax: np.ndarray, emax: int = E4M3_EMAX) -> np.ndarray:
     """E8M0 byte of a block from its largest magnitude (OCP MX v1.0 rule).
 
-    shared_exp = floor(log2(amax)) - 8, byte = clamp(shared_exp + 127, 0, 254);
-    amax == 0 gives byte 0; a non-finite amax gives 0xFF.
+    shared_exp = floor(log2(amax)) - emax (8 for E4M3, 15 for E5M2),
+    byte = clamp(shared_exp + 127, 0, 254); amax == 0 gives byte 0; a
+    non-finite amax gives 0xFF.
     """
     amax = np.asarray(amax, dtype=np.float64)
     out = np.zeros(amax.shape, dtype=np.int64)
     pos = np.isfinite(amax) & (amax > 0)
     _, e = np.frexp(amax[pos])          # amax in [2^(e-1), 2^e) -> floor(log2) = e-1
-    out[pos] = np.clip((e - 1) - E4M3_EMAX + E8M0_BIAS, 0, 254)
+    out[pos] = np.clip((e - 1) - emax + E8M0_BIAS, 0, 254)
     out[~np.isfinite(amax)] = E8M0_NAN
     return out.astype(np.uint8)
 
@@ -175,12 +210,55 @@ def e4m3_code_of(q: np.ndarray) -> np.ndarray:
     return (code | sign).astype(np.uint8)
 
 
-def quantize_rows(x: np.ndarray):
+def e5m2_round(v: np.ndarray) -> np.ndarray:
+    """Round float64 to the E5M2 grid: nearest, ties to even, saturate at 57344.
+
+    In the binade [2^k, 2^(k+1)), k >= -14, E5M2 values are spaced 2^(k-2);
+    below 2^-14 (subnormals) the spacing is 2^-16.
+    """
+    v = np.asarray(v, dtype=np.float64)
+    a = np.abs(v)
+    out = np.zeros_like(a)
+    nz = a > 0
+    _, e = np.frexp(a[nz])
+    ulp_exp = np.maximum(e - 3, -16)
+    out[nz] = np.ldexp(np.rint(np.ldexp(a[nz], -ulp_exp)), ulp_exp)
+    out = np.minimum(out, E5M2_MAX)
+    return np.copysign(out, v)
+
+
+def e5m2_code_of(q: np.ndarray) -> np.ndarray:
+    """Bit pattern of a float64 already on the E5M2 grid (|q| <= 57344)."""
+    q = np.asarray(q, dtype=np.float64)
+    a = np.abs(q)
+    sign = np.signbit(q).astype(np.int64) << 7
+    code = np.zeros(a.shape, dtype=np.int64)
+    sub = a < 2.0 ** -14
+    code[sub] = np.rint(a[sub] / 2.0 ** -16).astype(np.int64)
+    nrm = ~sub
+    _, e = np.frexp(a[nrm])
+    k = e - 1
+    mant = np.rint((np.ldexp(a[nrm], -k) - 1.0) * 4).astype(np.int64)
+    code[nrm] = ((k + 15) << 2) | mant
+    return (code | sign).astype(np.uint8)
+
+
+# element formats: (largest exponent, rounding onto the grid, bit pattern, decode)
+ELEMENTS = {
+    "e4m3": (E4M3_EMAX, e4m3_round, e4m3_code_of, e4m3_decode),
+    "e5m2": (E5M2_EMAX, e5m2_round, e5m2_code_of, e5m2_decode),
+}
+
+
+def quantize_rows(x: np.ndarray, elem: str = "e4m3"):
     """ROW MX quantization of a 2-D array of bf16 values (given as float64).
 
     Blocks of 32 along the last dimension; the last block of a row may be
     shorter.  Returns (codes uint8 [rows, cols], scales uint8 [rows, ceil(cols/32)]).
+    ``elem`` picks the element format (E4M3 by default, or E5M2; the A2E
+    transport page, "quant_mode=4": E4M3 or E5M2 with an E8M0 block scale).
     """
+    emax, rnd, code_of, _ = ELEMENTS[elem]
     x = np.asarray(x, dtype=np.float64)
     rows, cols = x.shape
     nb = -(-cols // BLOCK)
@@ -191,19 +269,19 @@ def quantize_rows(x: np.ndarray):
     absb = np.abs(blocks)
     bad = ~np.isfinite(absb).all(axis=2)
     amax = np.where(bad, np.inf, np.nanmax(np.where(np.isfinite(absb), absb, 0.0), axis=2))
-    sb = scale_byte(amax)                                   # [rows, nb]
+    sb = scale_byte(amax, emax)                             # [rows, nb]
     shared = sb.astype(np.int64) - E8M0_BIAS
     v = np.ldexp(blocks, -shared[:, :, None])               # exact: power-of-two scaling
     with np.errstate(invalid="ignore"):
-        q = e4m3_round(np.where(np.isfinite(v), v, 0.0))
-    codes = e4m3_code_of(q)
+        q = rnd(np.where(np.isfinite(v), v, 0.0))
+    codes = code_of(q)
     nan_code = (np.signbit(blocks).astype(np.uint8) << 7) | E4M3_NAN
     codes = np.where(bad[:, :, None], nan_code, codes).astype(np.uint8)
     codes = codes.reshape(rows, padc)[:, :cols]
     return np.ascontiguousarray(codes), sb
 
 
-def quantize_cols(x: np.ndarray):
+def quantize_cols(x: np.ndarray, elem: str = "e4m3"):
     """COL MX quantization: blocks of 32 consecutive rows of one column.
 
     Stored transposed: codes [cols, rows], scales [cols, rows/32].  It is the
@@ -211,16 +289,17 @@ def quantize_cols(x: np.ndarray):
     """
     x = np.asarray(x, dtype=np.float64)
     assert x.shape[0] % BLOCK == 0, "COL quantization needs rows % 32 == 0"
-    return quantize_rows(x.T)
+    return quantize_rows(x.T, elem)
 
 
-def dequantize_rows(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+def dequantize_rows(codes: np.ndarray, scales: np.ndarray, elem: str = "e4m3") -> np.ndarray:
     """codes [rows, cols] * per-block scale -> float64 [rows, cols]."""
     codes = np.asarray(codes)
     rows, cols = codes.shape
     s = e8m0_decode(scales)                                 # [rows, nb]
     s_full = np.repeat(s, BLOCK, axis=1)[:, :cols]
-    return e4m3_decode(codes) * s_full
+    with np.errstate(invalid="ignore"):
+        return ELEMENTS[elem][3](codes) * s_full
 
 
 # ----------------------------------------------------------------------------

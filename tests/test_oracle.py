@@ -171,6 +171,88 @@ def test_e4m3_encoder_vs_torch_in_range():
         np.testing.assert_array_equal(ours, ref)
 
 
+# ---------------------------------------------------------------- E5M2 element format
+def test_e5m2_table_closed_form():
+    t = mx.E5M2_TABLE
+    assert t[0x7B] == 57344.0 and t[0xFB] == -57344.0       # largest finite
+    assert t[0x04] == 2.0 ** -14                            # smallest normal
+    assert t[0x01] == 2.0 ** -16                            # smallest subnormal
+    assert t[0x03] == 3 * 2.0 ** -16                        # largest subnormal
+    assert t[0x3C] == 1.0 and t[0x40] == 2.0 and t[0x3E] == 1.5
+    assert t[0x7C] == np.inf and t[0xFC] == -np.inf
+    assert np.isnan(t[[0x7D, 0x7E, 0x7F, 0xFD, 0xFE, 0xFF]]).all()
+    assert t[0x80] == 0.0 and math.copysign(1, t[0x80]) < 0
+    assert np.isfinite(t).sum() == 248
+
+
+def test_e5m2_table_vs_torch():
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    ref = codes.view(torch.float8_e5m2).to(torch.float64).numpy()
+    ours = mx.e5m2_decode(np.arange(256))
+    np.testing.assert_array_equal(np.isnan(ref), np.isnan(ours))
+    ok = ~np.isnan(ref)
+    np.testing.assert_array_equal(ref[ok], ours[ok])
+    np.testing.assert_array_equal(np.signbit(ref[ok]), np.signbit(ours[ok]))
+
+
+_POS5 = np.arange(0x7C)                   # finite non-negative E5M2 codes 0x00..0x7B
+_POS5_VAL = mx.E5M2_TABLE[_POS5]
+
+
+def _e5m2_bruteforce(v):
+    """Nearest finite E5M2 by search over the decode table, ties -> even code."""
+    a = np.minimum(np.abs(v), 1e9)
+    d = np.abs(a[:, None] - _POS5_VAL[None, :])
+    dmin = d.min(axis=1, keepdims=True)
+    cand = np.where(d == dmin, _POS5[None, :], 10 ** 6)
+    even = np.where((cand % 2 == 0) & (cand < 10 ** 6), cand, 10 ** 6)
+    pick = np.where(even.min(axis=1) < 10 ** 6, even.min(axis=1), cand.min(axis=1))
+    return (pick | (np.signbit(v).astype(np.int64) << 7)).astype(np.uint8)
+
+
+@pytest.mark.parametrize("byte", [0, 100, 112, 127, 141, 254])
+def test_e5m2_encoder_exhaustive_bf16(byte):
+    x = mx.bf16_bits_to_f64(np.arange(65536, dtype=np.uint32).astype(np.uint16))
+    x = x[np.isfinite(x)]
+    v = np.ldexp(x, -(byte - 127))
+    ours = mx.e5m2_code_of(mx.e5m2_round(v))
+    for lo in range(0, v.size, 8192):
+        ref = _e5m2_bruteforce(v[lo:lo + 8192])
+        np.testing.assert_array_equal(ours[lo:lo + 8192], ref)
+
+
+def test_e5m2_encoder_vs_torch_in_range():
+    x = mx.bf16_bits_to_f64(np.arange(65536, dtype=np.uint32).astype(np.uint16))
+    for byte in (112, 127, 135):
+        v = np.ldexp(x, -(byte - 127))
+        v = v[np.isfinite(v) & (np.abs(v) <= 57344.0)]
+        ref = torch.from_numpy(v).to(torch.float8_e5m2).view(torch.uint8).numpy()
+        ours = mx.e5m2_code_of(mx.e5m2_round(v))
+        np.testing.assert_array_equal(ours, ref)
+
+
+def test_e5m2_scale_rule_and_special_blocks():
+    g = np.random.default_rng(13)
+    x = mx.round_to_bf16(g.standard_normal((16, 256)) * 2.0 ** g.integers(-90, 90, (16, 1)))
+    codes, sc = mx.quantize_rows(x, "e5m2")
+    amax = np.abs(x).reshape(16, 8, 32).max(axis=2)
+    ratio = amax / np.ldexp(1.0, sc.astype(np.int64) - 127)
+    assert ((ratio >= 2.0 ** 15) & (ratio < 2.0 ** 16)).all()       # emax 15: max lands in [2^15, 2^16)
+    deq = mx.dequantize_rows(codes, sc, "e5m2")
+    s = np.repeat(np.ldexp(1.0, sc.astype(np.int64) - 127), 32, axis=1)
+    a = np.abs(x) / s
+    ulp = np.ldexp(1.0, np.maximum(np.frexp(a)[1] - 3, -16))
+    unsat = a <= 57344
+    assert (np.abs(deq - x)[unsat] <= 0.5 * ulp[unsat] * s[unsat]).all()
+    y = np.zeros((1, 96))
+    y[0, 0] = np.inf
+    y[0, 1] = -2.0
+    y[0, 32:64] = -0.0
+    c, b = mx.quantize_rows(y, "e5m2")
+    assert b[0, 0] == 0xFF and c[0, 0] == 0x7F and c[0, 1] == 0xFF
+    assert b[0, 1] == 0 and (c[0, 32:64] == 0x80).all() and b[0, 2] == 0
+
+
 # ---------------------------------------------------------------- block quantizer
 def test_scale_rule_puts_block_max_in_256_512():
     g = np.random.default_rng(3)
