@@ -250,6 +250,14 @@ class Step:
              lambda: L.mxmoe_combine_weight_grad(p(self.dout), p(self.y), M, D, p(self.r_slot_row), T, k, p(self.dwr),
                                                  st)),
         ]
+        # the transport payload with E5M2 elements (cast and restore)
+        self.e5m2_ops = [
+            ("cast_payload_e5m2_8192x7168", "hbm", 3.03125 * CAST_ROWS * CAST_COLS,
+             lambda: L.mxfp8_quantize_e5m2(p(self.c_in), 1, CAST_ROWS, CAST_COLS, 1, 0, p(self.c_rc), p(self.c_rs),
+                                           None, None, st)),
+            ("dequant_payload_e5m2_8192x7168", "hbm", 3.03125 * CAST_ROWS * CAST_COLS,
+             lambda: L.mxfp8_dequantize_e5m2(p(self.c_rc), p(self.c_rs), CAST_ROWS, CAST_COLS, p(self.c_deq), st)),
+        ]
 
     def run(self, events=None):
         for i, (name, _, _, fn) in enumerate(self.ops):
@@ -502,16 +510,21 @@ def main():
                         "what": "x cast + FC1 (+SwiGLU + dual quant fused in the epilogue) + FC2, vs x cast + FC1 "
                                 "to bf16 h13 + standalone SwiGLU + dual quant + FC2; same padding (pad-matched)"}
 
-    # dispatcher kernels (not part of the step): each timed alone, n launches
-    dispatcher = {}
-    for name, bound, work, fn in step.disp_ops:
-        if fn() != 0:
-            raise RuntimeError(f"{name}: {step.L.mxmoe_last_error().decode()}")
-        ms = time_it(fn, n=10)
-        ach = work / (ms * 1e-3) / 1e9
-        dispatcher[name] = {"ms": round(ms, 4), "GB/s": round(ach, 1), "frac": round(ach / hbm, 3)}
-    if mxk.device_error() != 0:
-        raise RuntimeError("device error in the dispatcher kernels")
+    # kernels outside the step (the token dispatcher, the E5M2 transport
+    # variant): each timed alone over n launches
+    def time_group(ops):
+        res = {}
+        for name, bound, work, fn in ops:
+            if fn() != 0:
+                raise RuntimeError(f"{name}: {step.L.mxmoe_last_error().decode()}")
+            ms = time_it(fn, n=10)
+            ach = work / (ms * 1e-3) / 1e9
+            res[name] = {"ms": round(ms, 4), "GB/s": round(ach, 1), "frac": round(ach / hbm, 3)}
+        if mxk.device_error() != 0:
+            raise RuntimeError("device error outside the step")
+        return res
+
+    outside_step = {"dispatcher": time_group(step.disp_ops), "e5m2_transport": time_group(step.e5m2_ops)}
 
     # dominant kernel and its roofline
     imax = int(np.argmax(mean_ms[: step.mlp_ops]))
@@ -619,7 +632,7 @@ def main():
         "mlp_no_weight_cast_tflops": round(useful / ((mlp_ms - cast_w_ms) * 1e-3) / 1e12, 2),
         "fwd_useful_tflops_prequantized_weights": round(6.0 * step.R * spec.D * spec.F / (fwd_ms * 1e-3) / 1e12, 2),
         "swiglu_quant_gbs": sw["GB/s"], "swiglu_quant_frac_hbm": sw["frac"],
-        "kernels": kernels, "fused_vs_unfused": fused_vs_unfused, "dispatcher": dispatcher, "roofline": roof, "clocks": clk,
+        "kernels": kernels, "fused_vs_unfused": fused_vs_unfused, "outside_step": outside_step, "roofline": roof, "clocks": clk,
         "gpu_launches": n_ops * args.steps,
         "e2e": e2e, "cpu_baseline": cpu, "source_hash": src_hash(),
     }

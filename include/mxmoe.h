@@ -114,6 +114,17 @@ int mxfp8_quantize(const void* x, int64_t batch, int64_t rows, int64_t cols,
                    uint8_t* col_codes, uint8_t* col_scales,
                    cudaStream_t stream);
 
+/* mxfp8_quantize with E5M2 elements (A2E transport page, "quant_mode=4": the
+ * activation is quantized to E4M3 or E5M2 with its E8M0 block scale).  Same
+ * arguments, layouts and rules; the block exponent is floor(log2(amax)) - 15
+ * (15 = largest E5M2 exponent), elements round to nearest-even E5M2 and
+ * saturate at +-57344; NaN/Inf blocks get byte 0xFF and codes 0x7F | sign. */
+int mxfp8_quantize_e5m2(const void* x, int64_t batch, int64_t rows, int64_t cols,
+                        int modes, int scale_layout,
+                        uint8_t* row_codes, uint8_t* row_scales,
+                        uint8_t* col_codes, uint8_t* col_scales,
+                        cudaStream_t stream);
+
 /* -------------------------------------------------------------------------
  * mxfp8_swiglu_quant -- fused SwiGLU + dual MXFP8 quantization.
  * (SwiGLU-boundary page, "Summary": fused SwiGLU + dual MXFP8 quantization;
@@ -139,6 +150,11 @@ int mxfp8_swiglu_quant(const void* h13, int64_t rows, int64_t F,
  * ------------------------------------------------------------------------- */
 int mxfp8_dequantize(const uint8_t* codes, const uint8_t* scales,
                      int64_t rows, int64_t cols, void* out, cudaStream_t stream);
+
+/* mxfp8_dequantize for E5M2 codes (+-infinity codes stay infinite, NaN codes
+ * give NaN). */
+int mxfp8_dequantize_e5m2(const uint8_t* codes, const uint8_t* scales,
+                          int64_t rows, int64_t cols, void* out, cudaStream_t stream);
 
 /* -------------------------------------------------------------------------
  * mxfp8_grouped_gemm -- ragged-M grouped GEMM (FC2 / dgrad form).

@@ -55,6 +55,8 @@ _SIGS = {
     "mxmoe_version": ([], ctypes.c_char_p),
     "mxmoe_device_error": ([_P, _I, ctypes.POINTER(ctypes.c_int)], _I),
     "mxfp8_quantize": ([_P, _L, _L, _L, _I, _I, _P, _P, _P, _P, _P], _I),
+    "mxfp8_quantize_e5m2": ([_P, _L, _L, _L, _I, _I, _P, _P, _P, _P, _P], _I),
+    "mxfp8_dequantize_e5m2": ([_P, _P, _L, _L, _P, _P], _I),
     "mxfp8_swiglu_quant": ([_P, _L, _L, _I, _I, _P, _P, _P, _P, _P], _I),
     "mxfp8_dequantize": ([_P, _P, _L, _L, _P, _P], _I),
     "mxfp8_grouped_gemm": ([_P, _P, _L, _L, _P, _P, _I, _L, _P, _I, _P, _P], _I),
@@ -144,8 +146,8 @@ def device_error(reset: bool = True, device=None) -> int:
 
 
 # ----------------------------------------------------------------------------- casts
-def mxfp8_quantize(x: torch.Tensor, modes: int = ROW | COL, scale_layout: int = PLAIN):
-    """bf16 [rows, cols] or [batch, rows, cols] -> dict of MXFP8 tensors.
+def mxfp8_quantize(x: torch.Tensor, modes: int = ROW | COL, scale_layout: int = PLAIN, elem: str = "e4m3"):
+    """bf16 [rows, cols] or [batch, rows, cols] -> dict of MXFP8 tensors (E4M3 or E5M2 codes).
 
     Keys: row_codes [.., rows, cols], row_scales, col_codes [.., cols, rows],
     col_scales.  PLAIN scales are [.., rows, ceil(cols/32)] / [.., cols, rows/32];
@@ -166,7 +168,8 @@ def mxfp8_quantize(x: torch.Tensor, modes: int = ROW | COL, scale_layout: int = 
         out["col_codes"] = _u8(lead + (cols, rows), x.device)
         out["col_scales"] = (_u8(lead + (cols, rows // 32), x.device) if scale_layout == PLAIN
                              else _u8((batch * rows * cols // 32,), x.device))
-    _check(lib().mxfp8_quantize(_ptr(x), batch, rows, cols, modes, scale_layout,
+    fn = {"e4m3": lib().mxfp8_quantize, "e5m2": lib().mxfp8_quantize_e5m2}[elem]
+    _check(fn(_ptr(x), batch, rows, cols, modes, scale_layout,
                                 _ptr(out.get("row_codes")), _ptr(out.get("row_scales")),
                                 _ptr(out.get("col_codes")), _ptr(out.get("col_scales")), _stream(x)))
     return out
@@ -192,13 +195,14 @@ def mxfp8_swiglu_quant(h13: torch.Tensor, modes: int = ROW | COL, scale_layout: 
     return out
 
 
-def mxfp8_dequantize(codes: torch.Tensor, scales: torch.Tensor) -> torch.Tensor:
-    """MXFP8 ROW (plain scales) -> bf16."""
+def mxfp8_dequantize(codes: torch.Tensor, scales: torch.Tensor, elem: str = "e4m3") -> torch.Tensor:
+    """MXFP8 ROW (plain scales, E4M3 or E5M2 codes) -> bf16."""
     _need(codes, torch.uint8, "codes")
     _need(scales, torch.uint8, "scales")
     rows, cols = codes.shape
     out = torch.empty(rows, cols, dtype=torch.bfloat16, device=codes.device)
-    _check(lib().mxfp8_dequantize(_ptr(codes), _ptr(scales), rows, cols, _ptr(out), _stream(codes)))
+    fn = {"e4m3": lib().mxfp8_dequantize, "e5m2": lib().mxfp8_dequantize_e5m2}[elem]
+    _check(fn(_ptr(codes), _ptr(scales), rows, cols, _ptr(out), _stream(codes)))
     return out
 
 

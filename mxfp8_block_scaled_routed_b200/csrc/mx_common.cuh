@@ -49,9 +49,9 @@ __device__ __forceinline__ uint32_t absmax_bits8(uint4 v) {
 // floor(log2(amax)) is the unbiased exponent field, so the byte is
 // max(expfield - 8, 0); subnormal or zero maxima land on 0 via the clamp.
 // Returns 0xFF for NaN/Inf blocks.
-__device__ __forceinline__ uint32_t scale_byte_from_bits(uint32_t amax_bits) {
+__device__ __forceinline__ uint32_t scale_byte_from_bits(uint32_t amax_bits, int emax = 8) {
   if (amax_bits >= 0x7F80u) return 0xFFu;
-  int e = int(amax_bits >> 7) - 8;
+  int e = int(amax_bits >> 7) - emax;
   return uint32_t(e < 0 ? 0 : e);
 }
 
@@ -66,6 +66,21 @@ __device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(b), "f"(a));
   return r;
 }
+// Same for E5M2 (saturating at 57344).
+__device__ __forceinline__ uint32_t e5m2x2(float a, float b) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(r) : "f"(b), "f"(a));
+  return r;
+}
+
+// Element formats of an MXFP8 tensor: 0 = E4M3 (largest exponent 8),
+// 1 = E5M2 (largest exponent 15).
+template <int kElem>
+__device__ __forceinline__ uint32_t fp8x2(float a, float b) {
+  if constexpr (kElem == 0) return e4m3x2(a, b); else return e5m2x2(a, b);
+}
+template <int kElem>
+__host__ __device__ constexpr int elem_emax() { return kElem == 0 ? 8 : 15; }
 
 // Eight packed bf16 -> eight E4M3 codes (uint2), scaled by inv (a power of two).
 __device__ __forceinline__ uint2 quant8_bf16(uint4 v, float inv) {
@@ -104,16 +119,17 @@ __device__ __forceinline__ float absmax_nan(float a, float b) {
 
 // E8M0 byte from the block maximum as fp32 (|amax|, NaN/Inf -> 0xFF); same
 // rule as scale_byte_from_bits: max(expfield - 8, 0).
-__device__ __forceinline__ uint32_t scale_byte_from_f32(float amax) {
+__device__ __forceinline__ uint32_t scale_byte_from_f32(float amax, int emax = 8) {
   const uint32_t b = __float_as_uint(amax);
   if (b >= 0x7F800000u) return 0xFFu;
-  const int e = int(b >> 23) - 8;
+  const int e = int(b >> 23) - emax;
   return uint32_t(e < 0 ? 0 : e);
 }
 
-// Two E4M3 codes of two bf16 held in one 32-bit word, scaled by inv.
-__device__ __forceinline__ uint32_t e4m3x2_of_word(uint32_t w, float inv) {
-  return e4m3x2(bf16lo_to_f32(w) * inv, bf16hi_to_f32(w) * inv);
+// Two codes of two bf16 held in one 32-bit word, scaled by inv.
+template <int kElem = 0>
+__device__ __forceinline__ uint32_t fp8x2_of_word(uint32_t w, float inv) {
+  return fp8x2<kElem>(bf16lo_to_f32(w) * inv, bf16hi_to_f32(w) * inv);
 }
 
 // ---------------------------------------------------------------- layouts

@@ -164,7 +164,7 @@ int make_gather_map(CUtensorMap* map, const void* base, int64_t tokens, int64_t 
   return MXMOE_OK;
 }
 
-template <int kMode>
+template <int kMode, int kElem = 0>
 int launch_cast(const void* in, int64_t batch, int64_t rows, int64_t cols, int modes, int layout, uint8_t* rc,
                 uint8_t* rs, uint8_t* cc, uint8_t* cs, const int32_t* dev_rows, cudaStream_t stream,
                 const GatherArgs* g = nullptr) {
@@ -172,8 +172,8 @@ int launch_cast(const void* in, int64_t batch, int64_t rows, int64_t cols, int m
   constexpr bool kSwiglu = kMode == kCastSwiglu;
   DevInfo* d;
   MX_TRY(device_info(&d));
-  const int bit = kMode == kCastPlain ? 7 : kMode == kCastSwiglu ? 8 : 13;   // distinct from the GEMM bits
-  auto kern = mx_cast_kernel<kMode>;
+  const int bit = kElem == 1 ? 15 : kMode == kCastPlain ? 7 : kMode == kCastSwiglu ? 8 : 13;  // not the GEMM bits
+  auto kern = mx_cast_kernel<kMode, kElem>;
   if (!(d->attr_set & (1u << bit))) {
     MX_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem),
                   "cudaFuncSetAttribute");
@@ -340,7 +340,7 @@ int check_ptrs(std::initializer_list<std::pair<const char*, const void*>> ps) {
 // ---------------------------------------------------------------- casts
 int quantize_impl(const void* x, int64_t batch, int64_t rows, int64_t cols, int modes, int layout,
                   uint8_t* rc, uint8_t* rs, uint8_t* cc, uint8_t* cs, cudaStream_t stream,
-                  bool swiglu = false) {
+                  bool swiglu = false, int elem = 0) {
   if (modes < 1 || modes > 3) return fail(MXMOE_ERR_ARG, "modes=%d must be MXFP8_ROW, MXFP8_COL or both", modes);
   if (layout != MXFP8_SCALE_PLAIN && layout != MXFP8_SCALE_MMA)
     return fail(MXMOE_ERR_ARG, "scale_layout=%d invalid", layout);
@@ -368,12 +368,16 @@ int quantize_impl(const void* x, int64_t batch, int64_t rows, int64_t cols, int 
     const int64_t warps = R * ((cols + 31) / 32);
     const int64_t blocks = (warps * 32 + 255) / 256;
     if (blocks > 0x7FFFFFFF) return fail(MXMOE_ERR_SHAPE, "tensor too large");
-    mx_row_generic_kernel<<<unsigned(blocks), 256, 0, stream>>>(in, R, cols, rc, rs);
+    if (elem == 1)
+      mx_row_generic_kernel<1><<<unsigned(blocks), 256, 0, stream>>>(in, R, cols, rc, rs);
+    else
+      mx_row_generic_kernel<0><<<unsigned(blocks), 256, 0, stream>>>(in, R, cols, rc, rs);
     MX_CHECK_CUDA(cudaGetLastError(), "cast launch");
     return MXMOE_OK;
   }
   if (swiglu)
     return launch_cast<kCastSwiglu>(x, 1, rows, cols, modes, layout, rc, rs, cc, cs, nullptr, stream);
+  if (elem == 1) return launch_cast<kCastPlain, 1>(x, batch, rows, cols, modes, layout, rc, rs, cc, cs, nullptr, stream);
   return launch_cast<kCastPlain>(x, batch, rows, cols, modes, layout, rc, rs, cc, cs, nullptr, stream);
 }
 
@@ -622,6 +626,38 @@ __global__ void selftest_wait_kernel() {
 }
 
 // =====================================================================================
+template <int kElem>
+int dequantize_impl(const uint8_t* codes, const uint8_t* scales, int64_t rows, int64_t cols, void* out,
+                    cudaStream_t stream) {
+  if (!codes || !scales || !out) return fail(MXMOE_ERR_NULL, "codes/scales/out is NULL");
+  if (rows <= 0 || cols <= 0) return fail(MXMOE_ERR_SHAPE, "rows and cols must be positive");
+  DevInfo* d;
+  MX_TRY(device_info(&d));
+  const int64_t n = rows * cols;
+  const bool vec = cols % 16 == 0 && reinterpret_cast<uintptr_t>(codes) % 16 == 0 &&
+                   reinterpret_cast<uintptr_t>(out) % 16 == 0;
+  if (vec) {
+    const int64_t n16 = n / 16, cpr = cols / 16, ncb = (cols + 31) / 32;
+    const int64_t blocks = std::min<int64_t>((n16 + 255) / 256, int64_t(d->sms) * 8);
+    const auto* c4 = reinterpret_cast<const uint4*>(codes);
+    auto* o4 = static_cast<uint4*>(out);
+    if (n16 < (int64_t(1) << 31))
+      mx_dequant16_kernel<uint32_t, kElem><<<unsigned(blocks), 256, 0, stream>>>(c4, scales, uint32_t(n16),
+                                                                                 uint32_t(cpr), uint32_t(ncb), o4);
+    else
+      mx_dequant16_kernel<uint64_t, kElem><<<unsigned(blocks), 256, 0, stream>>>(c4, scales, uint64_t(n16),
+                                                                                 uint64_t(cpr), uint64_t(ncb), o4);
+    MX_CHECK_CUDA(cudaGetLastError(), "dequant launch");
+    return MXMOE_OK;
+  }
+  const int64_t blocks = (n + 255) / 256;
+  if (blocks > 0x7FFFFFFF) return fail(MXMOE_ERR_SHAPE, "tensor too large");
+  mx_dequant_kernel<kElem><<<unsigned(blocks), 256, 0, stream>>>(codes, scales, rows, cols,
+                                                                 static_cast<uint16_t*>(out));
+  MX_CHECK_CUDA(cudaGetLastError(), "dequant launch");
+  return MXMOE_OK;
+}
+
 extern "C" {
 
 int mxmoe_selftest_wait_timeout(cudaStream_t stream) {
@@ -656,6 +692,13 @@ int mxfp8_quantize(const void* x, int64_t batch, int64_t rows, int64_t cols, int
                        stream);
 }
 
+int mxfp8_quantize_e5m2(const void* x, int64_t batch, int64_t rows, int64_t cols, int modes, int scale_layout,
+                        uint8_t* row_codes, uint8_t* row_scales, uint8_t* col_codes, uint8_t* col_scales,
+                        cudaStream_t stream) {
+  return quantize_impl(x, batch, rows, cols, modes, scale_layout, row_codes, row_scales, col_codes, col_scales,
+                       stream, false, 1);
+}
+
 int mxfp8_swiglu_quant(const void* h13, int64_t rows, int64_t F, int modes, int scale_layout, uint8_t* row_codes,
                        uint8_t* row_scales, uint8_t* col_codes, uint8_t* col_scales, cudaStream_t stream) {
   if (F % 32 != 0) return fail(MXMOE_ERR_SHAPE, "F=%lld must be a multiple of 32", (long long)F);
@@ -665,32 +708,12 @@ int mxfp8_swiglu_quant(const void* h13, int64_t rows, int64_t F, int modes, int 
 
 int mxfp8_dequantize(const uint8_t* codes, const uint8_t* scales, int64_t rows, int64_t cols, void* out,
                      cudaStream_t stream) {
-  if (!codes || !scales || !out) return fail(MXMOE_ERR_NULL, "codes/scales/out is NULL");
-  if (rows <= 0 || cols <= 0) return fail(MXMOE_ERR_SHAPE, "rows and cols must be positive");
-  DevInfo* d;
-  MX_TRY(device_info(&d));
-  const int64_t n = rows * cols;
-  const bool vec = cols % 16 == 0 && reinterpret_cast<uintptr_t>(codes) % 16 == 0 &&
-                   reinterpret_cast<uintptr_t>(out) % 16 == 0;
-  if (vec) {
-    const int64_t n16 = n / 16, cpr = cols / 16, ncb = (cols + 31) / 32;
-    const int64_t blocks = std::min<int64_t>((n16 + 255) / 256, int64_t(d->sms) * 8);
-    const auto* c4 = reinterpret_cast<const uint4*>(codes);
-    auto* o4 = static_cast<uint4*>(out);
-    if (n16 < (int64_t(1) << 31))
-      mx_dequant16_kernel<uint32_t><<<unsigned(blocks), 256, 0, stream>>>(c4, scales, uint32_t(n16), uint32_t(cpr),
-                                                                          uint32_t(ncb), o4);
-    else
-      mx_dequant16_kernel<uint64_t><<<unsigned(blocks), 256, 0, stream>>>(c4, scales, uint64_t(n16), uint64_t(cpr),
-                                                                          uint64_t(ncb), o4);
-    MX_CHECK_CUDA(cudaGetLastError(), "dequant launch");
-    return MXMOE_OK;
-  }
-  const int64_t blocks = (n + 255) / 256;
-  if (blocks > 0x7FFFFFFF) return fail(MXMOE_ERR_SHAPE, "tensor too large");
-  mx_dequant_kernel<<<unsigned(blocks), 256, 0, stream>>>(codes, scales, rows, cols, static_cast<uint16_t*>(out));
-  MX_CHECK_CUDA(cudaGetLastError(), "dequant launch");
-  return MXMOE_OK;
+  return dequantize_impl<0>(codes, scales, rows, cols, out, stream);
+}
+
+int mxfp8_dequantize_e5m2(const uint8_t* codes, const uint8_t* scales, int64_t rows, int64_t cols, void* out,
+                          cudaStream_t stream) {
+  return dequantize_impl<1>(codes, scales, rows, cols, out, stream);
 }
 
 int mxfp8_grouped_gemm(const uint8_t* a, const uint8_t* a_scales, int64_t M, int64_t K, const uint8_t* w,

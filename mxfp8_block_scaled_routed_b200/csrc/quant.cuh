@@ -81,6 +81,7 @@ __device__ __forceinline__ uint32_t swiglu_pair(uint32_t g, uint32_t u) {
 
 // ROW quantization of 8 bf16 (one uint4) whose 32-block spans 4 consecutive
 // lanes; returns the 8 codes, *byte_out the block's scale byte.
+template <int kElem>
 __device__ __forceinline__ uint2 row_quant8(uint4 v, uint32_t* byte_out) {
   float m = 0.0f;
   m = absmax_nan(m, bf16lo_to_f32(v.x)); m = absmax_nan(m, bf16hi_to_f32(v.x));
@@ -89,26 +90,26 @@ __device__ __forceinline__ uint2 row_quant8(uint4 v, uint32_t* byte_out) {
   m = absmax_nan(m, bf16lo_to_f32(v.w)); m = absmax_nan(m, bf16hi_to_f32(v.w));
   m = absmax_nan(m, __shfl_xor_sync(0xffffffffu, m, 1));
   m = absmax_nan(m, __shfl_xor_sync(0xffffffffu, m, 2));
-  const uint32_t byte = scale_byte_from_f32(m);
+  const uint32_t byte = scale_byte_from_f32(m, elem_emax<kElem>());
   *byte_out = byte;
   if (byte == 0xFFu) return nan8_bf16(v);
   const float inv = inv_scale_from_byte(byte);
   uint2 o;
-  o.x = e4m3x2_of_word(v.x, inv) | (e4m3x2_of_word(v.y, inv) << 16);
-  o.y = e4m3x2_of_word(v.z, inv) | (e4m3x2_of_word(v.w, inv) << 16);
+  o.x = fp8x2_of_word<kElem>(v.x, inv) | (fp8x2_of_word<kElem>(v.y, inv) << 16);
+  o.y = fp8x2_of_word<kElem>(v.z, inv) | (fp8x2_of_word<kElem>(v.w, inv) << 16);
   return o;
 }
 
 // COL quantization of one column of a 32-row block: the column's values are
 // the low (hi_half = false) or high halves of the 32 words w[j] (word j =
 // row j, two adjacent columns).  Returns the scale byte, codes in q.
-template <bool kHi>
+template <bool kHi, int kElem>
 __device__ __forceinline__ uint32_t col_quant32(const uint32_t (&w)[32], uint4 (&q)[2]) {
   auto val = [&](int j) { return kHi ? bf16hi_to_f32(w[j]) : bf16lo_to_f32(w[j]); };
   float m = 0.0f;
 #pragma unroll
   for (int j = 0; j < 32; ++j) m = absmax_nan(m, val(j));
-  const uint32_t byte = scale_byte_from_f32(m);
+  const uint32_t byte = scale_byte_from_f32(m, elem_emax<kElem>());
   uint32_t c[8];
   if (byte == 0xFFu) {
 #pragma unroll
@@ -122,7 +123,8 @@ __device__ __forceinline__ uint32_t col_quant32(const uint32_t (&w)[32], uint4 (
     const float inv = inv_scale_from_byte(byte);
 #pragma unroll
     for (int k = 0; k < 8; ++k)
-      c[k] = e4m3x2(val(4 * k) * inv, val(4 * k + 1) * inv) | (e4m3x2(val(4 * k + 2) * inv, val(4 * k + 3) * inv) << 16);
+      c[k] = fp8x2<kElem>(val(4 * k) * inv, val(4 * k + 1) * inv) |
+             (fp8x2<kElem>(val(4 * k + 2) * inv, val(4 * k + 3) * inv) << 16);
   }
   q[0] = make_uint4(c[0], c[1], c[2], c[3]);
   q[1] = make_uint4(c[4], c[5], c[6], c[7]);
@@ -140,7 +142,7 @@ __device__ __forceinline__ uint32_t col_quant32(const uint32_t (&w)[32], uint4 (
 // SwiGLU: the gate and up tiles arrive together; the ROW pass computes
 // h = bf16(silu(gate) * up), quantizes it and parks it over the gate tile
 // for the COL pass (one barrier among the 256 consumer threads).
-template <int kMode>
+template <int kMode, int kElem = 0>
 __global__ void __launch_bounds__(kCastThreads, CastCfg<kMode>::kCtasPerSm)
 mx_cast_kernel(const __grid_constant__ CUtensorMap tin, const CastArgs p) {
   using C = CastCfg<kMode>;
@@ -334,7 +336,7 @@ mx_cast_kernel(const __grid_constant__ CUtensorMap tin, const CastArgs p) {
         }
         if (do_row) {
           uint32_t byte;
-          const uint2 q = row_quant8(v, &byte);
+          const uint2 q = row_quant8<kElem>(v, &byte);
           if (rr < vrows && ch * 8 < vcols) {
             *reinterpret_cast<uint2*>(rcode + int64_t(i) * 16 * cols) = q;
             if ((ch & 3) == 0) rsc[rr * 4 + (ch >> 2)] = uint8_t(byte);
@@ -354,7 +356,7 @@ mx_cast_kernel(const __grid_constant__ CUtensorMap tin, const CastArgs p) {
 #pragma unroll
         for (int k = 0; k < 2; ++k) {
           uint4 q[2];
-          const uint32_t byte = k ? col_quant32<true>(w, q) : col_quant32<false>(w, q);
+          const uint32_t byte = k ? col_quant32<true, kElem>(w, q) : col_quant32<false, kElem>(w, q);
           const int c = 2 * cp + k;
           uint8_t* dst = cstage + c * 128;
           const int swz = cp & 7;
@@ -446,6 +448,7 @@ mx_cast_kernel(const __grid_constant__ CUtensorMap tin, const CastArgs p) {
 
 // Generic ROW cast for any column count (short last block): one warp per
 // 32-element block, one element per lane.  Plain scale layout only.
+template <int kElem>
 __global__ void __launch_bounds__(256)
 mx_row_generic_kernel(const uint16_t* __restrict__ in, int64_t R, int64_t cols,
                       uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
@@ -458,13 +461,13 @@ mx_row_generic_kernel(const uint16_t* __restrict__ in, int64_t R, int64_t cols,
   const bool valid = col < cols;
   const uint32_t bits = valid ? in[row * cols + col] : 0u;
   const uint32_t am = __reduce_max_sync(0xffffffffu, bits & 0x7FFFu);
-  const uint32_t byte = scale_byte_from_bits(am);
+  const uint32_t byte = scale_byte_from_bits(am, elem_emax<kElem>());
   if (valid) {
     uint32_t code;
     if (byte == 0xFFu) {
       code = ((bits >> 8) & 0x80u) | 0x7Fu;
     } else {
-      code = e4m3x2(__uint_as_float(bits << 16) * inv_scale_from_byte(byte), 0.f) & 0xFFu;
+      code = fp8x2<kElem>(__uint_as_float(bits << 16) * inv_scale_from_byte(byte), 0.f) & 0xFFu;
     }
     codes[row * cols + col] = uint8_t(code);
   }
@@ -480,12 +483,17 @@ __device__ __forceinline__ float e8m0_to_f32(uint32_t byte) {
   return __uint_as_float(byte << 23);
 }
 
-__device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
+template <int kElem>
+__device__ __forceinline__ float fp8_to_f32(uint32_t code) {
   uint32_t h;
-  asm("{ .reg .b16 c; cvt.u16.u32 c, %1; cvt.rn.f16x2.e4m3x2 %0, c; }" : "=r"(h) : "r"(code));
+  if constexpr (kElem == 0)
+    asm("{ .reg .b16 c; cvt.u16.u32 c, %1; cvt.rn.f16x2.e4m3x2 %0, c; }" : "=r"(h) : "r"(code));
+  else
+    asm("{ .reg .b16 c; cvt.u16.u32 c, %1; cvt.rn.f16x2.e5m2x2 %0, c; }" : "=r"(h) : "r"(code));
   return __half2float(__ushort_as_half(uint16_t(h & 0xFFFFu)));
 }
 
+template <int kElem>
 __global__ void __launch_bounds__(256)
 mx_dequant_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
                   int64_t rows, int64_t cols, uint16_t* __restrict__ out) {
@@ -494,36 +502,62 @@ mx_dequant_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__
   if (i >= rows * cols) return;
   const int64_t r = i / cols, c = i % cols;
   const float s = e8m0_to_f32(scales[r * ncb + (c >> 5)]);
-  const float v = e4m3_to_f32(codes[i]) * s;
+  const float v = fp8_to_f32<kElem>(codes[i]) * s;
   out[i] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
 }
 
 // Vector path (cols % 16 == 0, 16-B aligned codes and output): one thread
-// per 16 codes, which share one scale.  The E4M3 bits are placed in an fp32
-// word so that the word reads as the code's value times 2^-120 (normals and
-// subnormals alike); multiplying by 2^(byte-7) -- split in two factors when
-// that power is not an fp32 normal -- then rounds the exact product
-// code*2^(byte-127) once, exactly as the scalar path does.
+// per 16 codes, which share one scale.  The code's exponent and mantissa
+// bits are placed in an fp32 word at the fp32 mantissa's top, so that the
+// word reads as the code's value times 2^-120 (E4M3, exponent bias 7) or
+// 2^-112 (E5M2, bias 15), normals and subnormals alike; multiplying by
+// 2^(byte - bias) -- split in two factors when that power is not an fp32
+// normal -- then rounds the exact product code * 2^(byte-127) once, exactly
+// as the scalar path does.
+template <int kElem>
+struct Fp8Bits {
+  static constexpr int kShift = kElem == 0 ? 20 : 21;     // code bit 0 -> fp32 bit
+  static constexpr uint32_t kOff = kElem == 0 ? 120u : 112u;   // 127 - exponent bias
+};
+
+template <int kElem>
 __device__ __forceinline__ uint32_t dequant_pair(uint32_t b0, uint32_t b1, float m1, float m2) {
-  const float y0 = __uint_as_float(((b0 & 0x80u) << 24) | ((b0 & 0x7Fu) << 20)) * m1 * m2;
-  const float y1 = __uint_as_float(((b1 & 0x80u) << 24) | ((b1 & 0x7Fu) << 20)) * m1 * m2;
+  constexpr int sh = Fp8Bits<kElem>::kShift;
+  const float y0 = __uint_as_float(((b0 & 0x80u) << 24) | ((b0 & 0x7Fu) << sh)) * m1 * m2;
+  const float y1 = __uint_as_float(((b1 & 0x80u) << 24) | ((b1 & 0x7Fu) << sh)) * m1 * m2;
   const __nv_bfloat162 h = __floats2bfloat162_rn(y0, y1);
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
+// bf16 of a code whose exponent field is all ones: E4M3 S.1111.111 is NaN;
+// E5M2 S.11111.00 is +-infinity and S.11111.xx (xx != 0) NaN.
+template <int kElem>
+__device__ __forceinline__ uint32_t special_bf16(uint32_t c) {
+  if constexpr (kElem == 0) return 0x7FFFu;
+  else return (c & 3u) ? 0x7FFFu : (0x7F80u | ((c & 0x80u) << 8));
+}
+
+template <int kElem>
 __device__ __forceinline__ void dequant_word(uint32_t w, float m1, float m2, uint32_t& lo, uint32_t& hi) {
-  lo = dequant_pair(w & 0xFFu, (w >> 8) & 0xFFu, m1, m2);
-  hi = dequant_pair((w >> 16) & 0xFFu, w >> 24, m1, m2);
-  // S.1111.111 is the E4M3 NaN; those lanes become the canonical bf16 NaN.
-  if ((((w & 0x7F7F7F7Fu) + 0x01010101u) & 0x80808080u) != 0u) {
-    if ((w & 0x7Fu) == 0x7Fu) lo = (lo & 0xFFFF0000u) | 0x7FFFu;
-    if ((w & 0x7F00u) == 0x7F00u) lo = (lo & 0x0000FFFFu) | 0x7FFF0000u;
-    if ((w & 0x7F0000u) == 0x7F0000u) hi = (hi & 0xFFFF0000u) | 0x7FFFu;
-    if ((w & 0x7F000000u) == 0x7F000000u) hi = (hi & 0x0000FFFFu) | 0x7FFF0000u;
+  lo = dequant_pair<kElem>(w & 0xFFu, (w >> 8) & 0xFFu, m1, m2);
+  hi = dequant_pair<kElem>((w >> 16) & 0xFFu, w >> 24, m1, m2);
+  // bytes whose special-value field is all ones (E4M3: the low 7 bits; E5M2:
+  // the 5 exponent bits) take their value from special_bf16
+  constexpr uint32_t f = kElem == 0 ? 0x7Fu : 0x7Cu;
+  constexpr uint32_t F4 = f * 0x01010101u, one = kElem == 0 ? 0x01010101u : 0x04040404u;
+  if ((((w & F4) + one) & 0x80808080u) != 0u) {
+    uint32_t v[4] = {lo & 0xFFFFu, lo >> 16, hi & 0xFFFFu, hi >> 16};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t c = (w >> (8 * j)) & 0xFFu;
+      if ((c & f) == f) v[j] = special_bf16<kElem>(c);
+    }
+    lo = v[0] | (v[1] << 16);
+    hi = v[2] | (v[3] << 16);
   }
 }
 
-template <typename Idx>
+template <typename Idx, int kElem>
 __global__ void __launch_bounds__(256)
 mx_dequant16_kernel(const uint4* __restrict__ codes, const uint8_t* __restrict__ scales, Idx n16, Idx chunks_per_row,
                     Idx ncb, uint4* __restrict__ out) {
@@ -536,12 +570,14 @@ mx_dequant16_kernel(const uint4* __restrict__ codes, const uint8_t* __restrict__
     if (byte == 0xFFu) {
       o0 = o1 = make_uint4(0x7FFF7FFFu, 0x7FFF7FFFu, 0x7FFF7FFFu, 0x7FFF7FFFu);
     } else {
-      const float m1 = __uint_as_float(byte <= 134u ? (byte + 120u) << 23 : (byte - 7u) << 23);
-      const float m2 = byte <= 134u ? 1.0f : __uint_as_float(254u << 23);
-      dequant_word(q.x, m1, m2, o0.x, o0.y);
-      dequant_word(q.y, m1, m2, o0.z, o0.w);
-      dequant_word(q.z, m1, m2, o1.x, o1.y);
-      dequant_word(q.w, m1, m2, o1.z, o1.w);
+      constexpr uint32_t off = Fp8Bits<kElem>::kOff;
+      const bool one = byte <= 254u - off;            // 2^(byte - bias) is an fp32 normal
+      const float m1 = __uint_as_float(one ? (byte + off) << 23 : (byte + off - 127u) << 23);
+      const float m2 = one ? 1.0f : __uint_as_float(254u << 23);
+      dequant_word<kElem>(q.x, m1, m2, o0.x, o0.y);
+      dequant_word<kElem>(q.y, m1, m2, o0.z, o0.w);
+      dequant_word<kElem>(q.z, m1, m2, o1.x, o1.y);
+      dequant_word<kElem>(q.w, m1, m2, o1.z, o1.w);
     }
     __stcs(out + 2 * i, o0);
     __stcs(out + 2 * i + 1, o1);

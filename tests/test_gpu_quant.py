@@ -176,3 +176,83 @@ def test_dequantize_shapes(rows, cols):
     codes = g.integers(0, 256, (rows, cols), dtype=np.uint8)
     scales = g.integers(100, 150, (rows, (cols + 31) // 32), dtype=np.uint8)
     _dequant_check(codes, scales)
+
+
+# ---------------------------------------------------------------- E5M2 elements
+def _check_e5m2(xt, out, rows=True, cols=True, plain=True):
+    x = bf16_np(xt)
+    if rows:
+        rc, rs = mx.quantize_rows(x, "e5m2")
+        np.testing.assert_array_equal(u8(out["row_codes"]), rc)
+        gs = u8(out["row_scales"]) if plain else mma_to_plain(u8(out["row_scales"]), *x.shape)
+        np.testing.assert_array_equal(gs.reshape(rs.shape), rs)
+    if cols:
+        cc, cs = mx.quantize_cols(x, "e5m2")
+        np.testing.assert_array_equal(u8(out["col_codes"]), cc)
+        gs = u8(out["col_scales"]) if plain else mma_to_plain(u8(out["col_scales"]), x.shape[1], x.shape[0])
+        np.testing.assert_array_equal(gs.reshape(cs.shape), cs)
+
+
+def test_e5m2_every_bf16_pattern_random_blocks():
+    g = np.random.default_rng(1)
+    bits = g.permutation(65536).reshape(512, 128)
+    xt = _bits_to_bf16(bits)
+    out = mxk.mxfp8_quantize(xt.to(DEV), mxk.ROW | mxk.COL, elem="e5m2")
+    _check_e5m2(xt, out)
+
+
+@pytest.mark.parametrize("byte", [0, 1, 100, 112, 127, 141, 200, 239])
+def test_e5m2_every_finite_pattern_under_fixed_scale(byte):
+    k = byte - 127 + 15 if byte > 0 else -112         # block max in [2^k, 2^(k+1))
+    allv = mx.bf16_bits_to_f64(np.arange(65536, dtype=np.uint32).astype(np.uint16))
+    fin = np.isfinite(allv) & (np.abs(allv) < 2.0 ** (k + 1))
+    pats = np.arange(65536)[fin]
+    nblk = -(-pats.size // 31)
+    pats = np.concatenate([pats, np.zeros(nblk * 31 - pats.size, dtype=pats.dtype)]).reshape(nblk, 31)
+    setter = mx.f64_to_bf16_bits(np.array([2.0 ** k]))[0]
+    blocks = np.concatenate([np.full((nblk, 1), setter), pats], axis=1)
+    rows = -(-nblk // 4) * 4
+    blocks = np.concatenate([blocks, np.zeros(((rows - nblk), 32), dtype=blocks.dtype)])
+    xt = _bits_to_bf16(blocks.reshape(rows // 4, 128))
+    out = mxk.mxfp8_quantize(xt.to(DEV), mxk.ROW, elem="e5m2")
+    _check_e5m2(xt, out, cols=False)
+    assert (u8(out["row_scales"]).reshape(-1)[:nblk] == byte).all()
+
+
+@pytest.mark.parametrize("layout", [mxk.PLAIN, mxk.MMA])
+def test_e5m2_dual_and_short_group(layout):
+    g = synth.rng(6)
+    xt = synth.to_bf16(synth.normal(g, (256, 384), 1.0, 0.01, 1000.0))
+    out = mxk.mxfp8_quantize(xt.to(DEV), mxk.ROW | mxk.COL, layout, elem="e5m2")
+    _check_e5m2(xt, out, plain=layout == mxk.PLAIN)
+    xs = synth.to_bf16(synth.normal(g, (9, 7170), 3.0))
+    out = mxk.mxfp8_quantize(xs.to(DEV), mxk.ROW, elem="e5m2")
+    _check_e5m2(xs, out, cols=False)
+
+
+def test_e5m2_transport_roundtrip_full_size():
+    """The A2E payload in E5M2: cast [8192, 7168] and restore, every element."""
+    xt = synth.make_cast_input()
+    out = mxk.mxfp8_quantize(xt.to(DEV), mxk.ROW, elem="e5m2")
+    back = mxk.mxfp8_dequantize(out["row_codes"], out["row_scales"], elem="e5m2")
+    torch.cuda.synchronize()
+    x = bf16_np(xt)
+    rc, rs = mx.quantize_rows(x, "e5m2")
+    np.testing.assert_array_equal(u8(out["row_codes"]), rc)
+    np.testing.assert_array_equal(u8(out["row_scales"]), rs)
+    ref = mx.round_to_bf16(mx.dequantize_rows(rc, rs, "e5m2"))
+    np.testing.assert_array_equal(bf16_np(back), ref)
+
+
+def test_e5m2_dequantize_every_code_with_every_scale():
+    codes = np.tile(np.arange(256, dtype=np.uint8), (256, 1))
+    scales = np.repeat(np.arange(256, dtype=np.uint8)[:, None], 8, axis=1)
+    for shape_cols in (256, 40):           # vector path and scalar path
+        c = np.ascontiguousarray(codes[:, :shape_cols])
+        s = np.ascontiguousarray(scales[:, :(shape_cols + 31) // 32])
+        out = mxk.mxfp8_dequantize(torch.from_numpy(c).to(DEV), torch.from_numpy(s).to(DEV), elem="e5m2")
+        got = bf16_np(out)
+        ref = mx.round_to_bf16(mx.dequantize_rows(c, s, "e5m2"))
+        np.testing.assert_array_equal(np.isnan(got), np.isnan(ref))
+        fin = ~np.isnan(ref)
+        np.testing.assert_array_equal(got[fin], ref[fin])
