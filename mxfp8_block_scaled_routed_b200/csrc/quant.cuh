@@ -79,56 +79,87 @@ __device__ __forceinline__ uint32_t swiglu_pair(uint32_t g, uint32_t u) {
   return pack_bf16x2(h0, h1);
 }
 
-// ROW quantization of 8 bf16 (one uint4) whose 32-block spans 4 consecutive
-// lanes; returns the 8 codes, *byte_out the block's scale byte.
+// The ROW and COL quantizers work on packed bf16 pairs.  The block maximum
+// comes from max.NaN.xorsign.abs.bf16x2 (magnitude max of two bf16 pairs,
+// NaN-propagating) on the bf16 bits, and the elements are scaled by the exact
+// power of two 2^(127 - byte) in bf16x2 arithmetic: with byte <= 246 (every
+// finite bf16 block) the factor is a bf16 normal and the product is exact
+// unless it falls below 2^-126, where every E4M3/E5M2 code is +-0 anyway and
+// the bf16 product keeps the sign.  The scaled pair is widened to fp32 and
+// converted by cvt.rn.satfinite (nearest-even, saturating).
+__device__ __forceinline__ uint32_t bf16x2_absmax(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+__device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+// bf16 bits of 2^(127 - byte) (byte <= 246).
+__device__ __forceinline__ uint32_t bf16_inv_scale(uint32_t byte) { return (254u - byte) << 7; }
+
 template <int kElem>
-__device__ __forceinline__ uint2 row_quant8(uint4 v, uint32_t* byte_out) {
-  float m = 0.0f;
-  m = absmax_nan(m, bf16lo_to_f32(v.x)); m = absmax_nan(m, bf16hi_to_f32(v.x));
-  m = absmax_nan(m, bf16lo_to_f32(v.y)); m = absmax_nan(m, bf16hi_to_f32(v.y));
-  m = absmax_nan(m, bf16lo_to_f32(v.z)); m = absmax_nan(m, bf16hi_to_f32(v.z));
-  m = absmax_nan(m, bf16lo_to_f32(v.w)); m = absmax_nan(m, bf16hi_to_f32(v.w));
-  m = absmax_nan(m, __shfl_xor_sync(0xffffffffu, m, 1));
-  m = absmax_nan(m, __shfl_xor_sync(0xffffffffu, m, 2));
-  const uint32_t byte = scale_byte_from_f32(m, elem_emax<kElem>());
+__device__ __forceinline__ uint2 row_quant8_packed(uint4 v, uint32_t* byte_out) {
+  uint32_t a = bf16x2_absmax(bf16x2_absmax(v.x, v.y), bf16x2_absmax(v.z, v.w)) & 0x7FFF7FFFu;
+  uint32_t m = max(a & 0xFFFFu, a >> 16);
+  m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
+  m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
+  const uint32_t byte = scale_byte_from_bits(m, elem_emax<kElem>());
   *byte_out = byte;
   if (byte == 0xFFu) return nan8_bf16(v);
-  const float inv = inv_scale_from_byte(byte);
+  const uint32_t s = bf16_inv_scale(byte) * 0x00010001u;
+  const uint32_t x = bf16x2_mul(v.x, s), y = bf16x2_mul(v.y, s), z = bf16x2_mul(v.z, s), w = bf16x2_mul(v.w, s);
   uint2 o;
-  o.x = fp8x2_of_word<kElem>(v.x, inv) | (fp8x2_of_word<kElem>(v.y, inv) << 16);
-  o.y = fp8x2_of_word<kElem>(v.z, inv) | (fp8x2_of_word<kElem>(v.w, inv) << 16);
+  auto cv = [](uint32_t t) { return fp8x2<kElem>(bf16lo_to_f32(t), bf16hi_to_f32(t)); };
+  o.x = cv(x) | (cv(y) << 16);
+  o.y = cv(z) | (cv(w) << 16);
   return o;
 }
 
-// COL quantization of one column of a 32-row block: the column's values are
-// the low (hi_half = false) or high halves of the 32 words w[j] (word j =
-// row j, two adjacent columns).  Returns the scale byte, codes in q.
-template <bool kHi, int kElem>
-__device__ __forceinline__ uint32_t col_quant32(const uint32_t (&w)[32], uint4 (&q)[2]) {
-  auto val = [&](int j) { return kHi ? bf16hi_to_f32(w[j]) : bf16lo_to_f32(w[j]); };
-  float m = 0.0f;
+// Both columns of a 32-row block held as the two halves of w[0..31]: codes
+// of the low-half column in q0, of the high-half column in q1; returns the
+// two scale bytes (low | high << 8).
+template <int kElem>
+__device__ __forceinline__ uint32_t col_quant_pair32(const uint32_t (&w)[32], uint4 (&q0)[2], uint4 (&q1)[2]) {
+  uint32_t a[16];
 #pragma unroll
-  for (int j = 0; j < 32; ++j) m = absmax_nan(m, val(j));
-  const uint32_t byte = scale_byte_from_f32(m, elem_emax<kElem>());
-  uint32_t c[8];
-  if (byte == 0xFFu) {
+  for (int j = 0; j < 16; ++j) a[j] = bf16x2_absmax(w[2 * j], w[2 * j + 1]);
+#pragma unroll
+  for (int st = 8; st >= 1; st >>= 1)
+#pragma unroll
+    for (int j = 0; j < st; ++j) a[j] = bf16x2_absmax(a[j], a[j + st]);
+  const uint32_t m = a[0] & 0x7FFF7FFFu;
+  const uint32_t b0 = scale_byte_from_bits(m & 0xFFFFu, elem_emax<kElem>());
+  const uint32_t b1 = scale_byte_from_bits(m >> 16, elem_emax<kElem>());
+  const uint32_t s = (b0 == 0xFFu ? 0u : bf16_inv_scale(b0)) | ((b1 == 0xFFu ? 0u : bf16_inv_scale(b1)) << 16);
+  uint32_t c0[8], c1[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const uint32_t x0 = bf16x2_mul(w[4 * k], s), x1 = bf16x2_mul(w[4 * k + 1], s);
+    const uint32_t x2 = bf16x2_mul(w[4 * k + 2], s), x3 = bf16x2_mul(w[4 * k + 3], s);
+    c0[k] = fp8x2<kElem>(bf16lo_to_f32(x0), bf16lo_to_f32(x1)) | (fp8x2<kElem>(bf16lo_to_f32(x2), bf16lo_to_f32(x3)) << 16);
+    c1[k] = fp8x2<kElem>(bf16hi_to_f32(x0), bf16hi_to_f32(x1)) | (fp8x2<kElem>(bf16hi_to_f32(x2), bf16hi_to_f32(x3)) << 16);
+  }
+  if (b0 == 0xFFu || b1 == 0xFFu) {                 // NaN/Inf block: codes 0x7F | sign
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-      uint32_t r = 0x7F7F7F7Fu;
+      uint32_t r0 = 0x7F7F7F7Fu, r1 = 0x7F7F7F7Fu;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) r |= ((__float_as_uint(val(4 * k + i)) >> 31) << 7) << (8 * i);
-      c[k] = r;
+      for (int i = 0; i < 4; ++i) {
+        r0 |= ((w[4 * k + i] >> 15) & 1u) << (8 * i + 7);
+        r1 |= (w[4 * k + i] >> 31) << (8 * i + 7);
+      }
+      if (b0 == 0xFFu) c0[k] = r0;
+      if (b1 == 0xFFu) c1[k] = r1;
     }
-  } else {
-    const float inv = inv_scale_from_byte(byte);
-#pragma unroll
-    for (int k = 0; k < 8; ++k)
-      c[k] = fp8x2<kElem>(val(4 * k) * inv, val(4 * k + 1) * inv) |
-             (fp8x2<kElem>(val(4 * k + 2) * inv, val(4 * k + 3) * inv) << 16);
   }
-  q[0] = make_uint4(c[0], c[1], c[2], c[3]);
-  q[1] = make_uint4(c[4], c[5], c[6], c[7]);
-  return byte;
+  q0[0] = make_uint4(c0[0], c0[1], c0[2], c0[3]);
+  q0[1] = make_uint4(c0[4], c0[5], c0[6], c0[7]);
+  q1[0] = make_uint4(c1[0], c1[1], c1[2], c1[3]);
+  q1[1] = make_uint4(c1[4], c1[5], c1[6], c1[7]);
+  return b0 | (b1 << 8);
 }
 
 // Persistent, TMA-fed cast.  Warp 8 streams 128 x 128 bf16 tiles (3-D tensor
@@ -336,7 +367,7 @@ mx_cast_kernel(const __grid_constant__ CUtensorMap tin, const CastArgs p) {
         }
         if (do_row) {
           uint32_t byte;
-          const uint2 q = row_quant8<kElem>(v, &byte);
+          const uint2 q = row_quant8_packed<kElem>(v, &byte);
           if (rr < vrows && ch * 8 < vcols) {
             *reinterpret_cast<uint2*>(rcode + int64_t(i) * 16 * cols) = q;
             if ((ch & 3) == 0) rsc[rr * 4 + (ch >> 2)] = uint8_t(byte);
@@ -353,16 +384,16 @@ mx_cast_kernel(const __grid_constant__ CUtensorMap tin, const CastArgs p) {
         const uint8_t* src = tile + (rb * 32) * 256 + cp * 4;
 #pragma unroll
         for (int j = 0; j < 32; ++j) w[j] = *reinterpret_cast<const uint32_t*>(src + j * 256);
+        uint4 qq[2][2];
+        const uint32_t bytes = col_quant_pair32<kElem>(w, qq[0], qq[1]);
 #pragma unroll
         for (int k = 0; k < 2; ++k) {
-          uint4 q[2];
-          const uint32_t byte = k ? col_quant32<true, kElem>(w, q) : col_quant32<false, kElem>(w, q);
           const int c = 2 * cp + k;
           uint8_t* dst = cstage + c * 128;
           const int swz = cp & 7;
-          *reinterpret_cast<uint4*>(dst + (((2 * rb) ^ swz) << 4)) = q[0];
-          *reinterpret_cast<uint4*>(dst + (((2 * rb + 1) ^ swz) << 4)) = q[1];
-          csc[c * 4 + rb] = uint8_t(byte);
+          *reinterpret_cast<uint4*>(dst + (((2 * rb) ^ swz) << 4)) = qq[k][0];
+          *reinterpret_cast<uint4*>(dst + (((2 * rb + 1) ^ swz) << 4)) = qq[k][1];
+          csc[c * 4 + rb] = uint8_t(bytes >> (8 * k));
         }
       }
     }
