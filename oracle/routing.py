@@ -68,11 +68,12 @@ def route(topk: np.ndarray, E: int, pad: int):
     return {"counts": counts, "offsets": offsets, "row_slot": row_slot, "slot_row": slot_row}
 
 
-def permute(x_tok: np.ndarray, row_slot: np.ndarray, k: int, weights=None) -> np.ndarray:
+def permute(x_tok: np.ndarray, row_slot: np.ndarray, k: int, weights=None, exact=False) -> np.ndarray:
     """Rows of the padded layout: x_tok[slot // k] (zero for pad rows).
 
     With ``weights`` [T, k] (fp32) every row is multiplied by its slot's
-    weight in fp32 and rounded to bf16 (the backward of the combine).
+    weight in fp32 and rounded to bf16 (the backward of the combine);
+    exact=True multiplies in float64 without rounding.
     """
     D = x_tok.shape[1]
     out = np.zeros((len(row_slot), D))
@@ -80,7 +81,9 @@ def permute(x_tok: np.ndarray, row_slot: np.ndarray, k: int, weights=None) -> np
         if s < 0:
             continue
         row = x_tok[s // k]
-        if weights is not None:
+        if weights is not None and exact:
+            row = float(np.asarray(weights, dtype=np.float64).reshape(-1)[s]) * row
+        elif weights is not None:
             w = np.float32(np.asarray(weights, dtype=np.float32).reshape(-1)[s])
             row = mx.round_to_bf16((w * row.astype(np.float32)).astype(np.float64))
         out[m] = row
@@ -113,3 +116,35 @@ def combine_weight_grad(dout: np.ndarray, y: np.ndarray, slot_row: np.ndarray, T
         for j in range(k):
             dw[t, j] = float(np.dot(dout[t], y[slot_row[t * k + j]]))
     return dw
+
+
+def layer_fwd(x_tok, topk, weights, w13, w2, E, pad, exact=False):
+    """Token-major layer forward: route, permute, the MLP over the padded
+    layout (oracle.mx.moe_mlp_fwd), combine with the router weights.
+
+    The MLP output rows are bf16 at the GEMM boundary, so the combine reads
+    them rounded (exact=True: unrounded).  Returns a dict with the route
+    tables, x_rows, the MLP forward ('mlp'), y_rows and out [T, D].
+    """
+    T, k = np.asarray(topk).shape
+    r = route(topk, E, pad)
+    x_rows = permute(x_tok, r["row_slot"], k)
+    fwd = mx.moe_mlp_fwd(x_rows, w13, w2, r["offsets"], exact=exact)
+    y_rows = np.nan_to_num(fwd["y"]) if exact else mx.round_to_bf16(np.nan_to_num(fwd["y"]))
+    out = unpermute_combine(y_rows, r["slot_row"], T, k, weights)
+    return dict(route=r, x_rows=x_rows, mlp=fwd, y_rows=y_rows, out=out)
+
+
+def layer_bwd(dout, fwd, x_tok, topk, weights, w13, w2, pad, exact=False):
+    """Token-major layer backward: dY rows = w * dout[token] (bf16), the MLP
+    backward (oracle.mx.moe_mlp_bwd), dx_tok = sum of a token's dx rows (bf16
+    rows, float64 sum), dweights = <dout, y row>.  Returns dict(dx, dw13, dw2,
+    dweights)."""
+    T, k = np.asarray(topk).shape
+    r = fwd["route"]
+    dy_rows = permute(dout, r["row_slot"], k, weights, exact=exact)
+    bwd = mx.moe_mlp_bwd(dy_rows, fwd["mlp"], fwd["x_rows"], w13, w2, r["offsets"], exact=exact)
+    dx_rows = np.nan_to_num(bwd["dx"]) if exact else mx.round_to_bf16(np.nan_to_num(bwd["dx"]))
+    dx = unpermute_combine(dx_rows, r["slot_row"], T, k)
+    dweights = combine_weight_grad(dout, fwd["y_rows"], r["slot_row"], T, k)
+    return dict(dx=dx, dw13=bwd["dw13"], dw2=bwd["dw2"], dweights=dweights, dy_rows=dy_rows)

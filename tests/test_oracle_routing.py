@@ -114,3 +114,41 @@ def test_weight_grad_is_the_derivative_of_the_combine():
             fp = np.sum(dout * routing.unpermute_combine(y, r["slot_row"], T, k, wp))
             fm = np.sum(dout * routing.unpermute_combine(y, r["slot_row"], T, k, wm))
             assert abs((fp - fm) / (2 * h) - dw[t, j]) < 1e-6 * max(1.0, abs(dw[t, j]))
+
+
+def test_layer_exact_mode_vs_torch_autograd():
+    # the whole token-major layer (route, permute, MLP, weighted combine) and
+    # its backward, without quantization, against float64 autograd of
+    # out[t] = sum_j w[t, j] * MLP_{topk[t, j]}(x[t])
+    import torch
+    T, k, E, D, F, pad = 24, 2, 3, 16, 8, 4
+    g = synth.rng(21)
+    topk = synth.topk_ids(T, k, E, seed=21)
+    w = g.random((T, k))
+    x = g.standard_normal((T, D))
+    w13 = g.standard_normal((E, 2 * F, D)) * 0.3
+    w2 = g.standard_normal((E, D, F)) * 0.3
+    dout = g.standard_normal((T, D))
+    fwd = routing.layer_fwd(x, topk, w, w13, w2, E, pad, exact=True)
+    bwd = routing.layer_bwd(dout, fwd, x, topk, w, w13, w2, pad, exact=True)
+
+    X = torch.tensor(x, requires_grad=True)
+    W13 = torch.tensor(w13, requires_grad=True)
+    W2 = torch.tensor(w2, requires_grad=True)
+    WR = torch.tensor(w, requires_grad=True)
+    outs = []
+    for t in range(T):
+        acc = torch.zeros(D, dtype=torch.float64)
+        for j in range(k):
+            e = int(topk[t, j])
+            h13 = W13[e] @ X[t]
+            h = torch.nn.functional.silu(h13[:F]) * h13[F:]
+            acc = acc + WR[t, j] * (W2[e] @ h)
+        outs.append(acc)
+    out = torch.stack(outs)
+    (out * torch.tensor(dout)).sum().backward()
+    np.testing.assert_allclose(fwd["out"], out.detach().numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(bwd["dx"], X.grad.numpy(), rtol=1e-9, atol=1e-12)
+    np.testing.assert_allclose(bwd["dw13"], W13.grad.numpy(), rtol=1e-9, atol=1e-12)
+    np.testing.assert_allclose(bwd["dw2"], W2.grad.numpy(), rtol=1e-9, atol=1e-12)
+    np.testing.assert_allclose(bwd["dweights"], WR.grad.numpy(), rtol=1e-9, atol=1e-12)
