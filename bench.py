@@ -542,21 +542,27 @@ def main():
                 "frac": round(ach / hbm, 3), "peak_source": f"{peak_src} hbm_gbs",
                 "traffic": ncu_traffic(dname, args.workload)}
 
-    # end to end through the public composite API, host buffers
+    # end to end through the public token-major layer API, host buffers: the
+    # step's inputs (token rows, routing, router weights, upstream gradient)
+    # are copied from pinned host memory every step; weights stay resident
     e2e = None
     if not args.no_e2e:
-        x_h = inp.x.cpu().pin_memory()
-        dy_h = inp.dy.cpu().pin_memory()
-        off_h = torch.from_numpy(inp.routing.offsets).pin_memory()
+        T, k = spec.tokens, spec.top_k
+        host = [inp.x_tok.cpu().pin_memory(), torch.from_numpy(inp.routing.topk).pin_memory(),
+                inp.router_w.cpu().pin_memory(), inp.dout_tok.cpu().pin_memory()]
         # two device slots for the step inputs: the copy of step i+1's inputs
         # (copy stream) overlaps step i's compute; every step's copy is inside
         # the timed region
-        slots = [(torch.empty_like(inp.x), torch.empty_like(inp.dy), torch.empty_like(step.off)) for _ in range(2)]
+        slots = [[torch.empty_like(h, device=dev) for h in host] for _ in range(2)]
         out_h = torch.empty(2, spec.D, dtype=torch.bfloat16).pin_memory()
-        saved = dict(h13=step.h13, h_col_codes=step.h_cc, h_col_scales=step.h_cs, x_col_codes=step.x_cc,
-                     x_col_scales=step.x_cs)
-        ws_f = torch.empty(mxk.workspace_bytes(step.M, spec.D, spec.E, spec.F, 3), dtype=torch.uint8, device=dev)
-        ws_b = torch.empty(mxk.workspace_bytes(step.M, spec.D, spec.E, spec.F, 4), dtype=torch.uint8, device=dev)
+        lsaved = mxk.make_layer_saved(T, k, spec.D, spec.E, spec.F, spec.pad, dev)
+        ws_f = torch.empty(mxk.layer_workspace_bytes(T, k, spec.D, spec.E, spec.F, spec.pad, 1), dtype=torch.uint8,
+                           device=dev)
+        ws_b = torch.empty(mxk.layer_workspace_bytes(T, k, spec.D, spec.E, spec.F, spec.pad, 2), dtype=torch.uint8,
+                           device=dev)
+        out_d = torch.empty(T, spec.D, dtype=torch.bfloat16, device=dev)
+        dx_d = torch.empty(T, spec.D, dtype=torch.bfloat16, device=dev)
+        dwr_d = torch.empty(T, k, dtype=torch.float32, device=dev)
         comp = torch.cuda.current_stream(dev)
         copy_s = torch.cuda.Stream(dev)
         copied = [torch.cuda.Event() for _ in range(2)]
@@ -567,23 +573,21 @@ def main():
             with torch.cuda.stream(copy_s):
                 if i >= 2:
                     copy_s.wait_event(used[sl])        # step i-2 finished reading this slot
-                x_d, dy_d, off_d = slots[sl]
-                x_d.copy_(x_h, non_blocking=True)
-                dy_d.copy_(dy_h, non_blocking=True)
-                off_d.copy_(off_h, non_blocking=True)
+                for d, h in zip(slots[sl], host):
+                    d.copy_(h, non_blocking=True)
                 copied[sl].record(copy_s)
 
         def compute(i):
             sl = i % 2
             comp.wait_event(copied[sl])
-            x_d, dy_d, off_d = slots[sl]
+            x_d, tk_d, w_d, do_d = slots[sl]
             mxk.mxmoe_quantize_weights(step.w13, step.w2, qw=step.qw)
-            mxk.moe_mlp_fwd_q(x_d, step.qw, off_d, spec.pad, y=step.y, saved=saved, workspace=ws_f)
-            mxk.moe_mlp_bwd_q(dy_d, step.qw, off_d, saved, spec.pad, dx=step.dx, dw13=step.dw13, dw2=step.dw2,
-                              workspace=ws_b)
+            mxk.moe_layer_fwd_q(x_d, tk_d, w_d, step.qw, spec.pad, out=out_d, saved=lsaved, workspace=ws_f)
+            mxk.moe_layer_bwd_q(do_d, w_d, step.qw, lsaved, spec.pad, dx=dx_d, dw13=step.dw13, dw2=step.dw2,
+                                dweights=dwr_d, workspace=ws_b)
             used[sl].record(comp)
-            out_h[0].copy_(step.y[0], non_blocking=True)
-            out_h[1].copy_(step.dx[0], non_blocking=True)
+            out_h[0].copy_(out_d[0], non_blocking=True)
+            out_h[1].copy_(dx_d[0], non_blocking=True)
 
         def run(nsteps):
             h2d(0)
@@ -604,13 +608,15 @@ def main():
         b.record(comp)
         torch.cuda.synchronize()
         ms = max_over_ranks(a.elapsed_time(b) / args.steps, dev)
-        h2d_bytes = x_h.numel() * 2 + dy_h.numel() * 2 + off_h.numel() * 4
+        h2d_bytes = sum(h.numel() * h.element_size() for h in host)
         e2e = {"value": round(whole_job_tflops(useful, world, ms), 2), "unit": "TFLOP/s",
                "h2d_bytes_per_step": int(h2d_bytes), "d2h_bytes_per_step": int(out_h.numel() * 2),
                "ms_per_step": round(ms, 3),
-               "how": "public C-ABI composites (mxmoe_quantize_weights, moe_mlp_fwd_q, moe_mlp_bwd_q); x, dY and "
-                      "offsets copied from pinned host memory every step on a copy stream overlapping the previous "
-                      "step's compute; one row of y and dx read back"}
+               "how": "public C-ABI token-major layer (mxmoe_quantize_weights, moe_layer_fwd_q: route + gather/cast + "
+                      "MLP + weighted combine, moe_layer_bwd_q: weighted gather/cast + MLP backward + unpermute + "
+                      "router-weight gradient); token rows, top-k ids, router weights and the upstream gradient "
+                      "copied from pinned host memory every step on a copy stream overlapping the previous step's "
+                      "compute; one row of the output and of dx read back"}
         if mxk.device_error() != 0:
             raise RuntimeError("device error during the e2e run")
 

@@ -425,6 +425,47 @@ int mxmoe_combine_weight_grad(const void* dout, const void* y, int64_t m_rows, i
                               const int32_t* slot_row, int64_t T, int top_k, float* dweights,
                               cudaStream_t stream);
 
+/* -------------------------------------------------------------------------
+ * Token-major layer composites: the dispatcher around the MLP.
+ * (Fully-fused plan page, "What it adds": the padded dispatcher feeding the
+ * four fused ops; SwiGLU-boundary page, "Usage".)
+ *
+ * Forward:  route topk_ids -> padded layout (saved tables); gather x_tokens
+ *           into it fused with the x cast (ROW + COL); FC1 + SwiGLU + dual
+ *           quant; FC2 -> saved y rows; weighted combine -> out_tokens.
+ * Backward: gather dout_tokens scaled by the router weights fused with the
+ *           dY cast; FC2 dgrad + dSwiGLU + dual quant; dW2; dx rows; dW13;
+ *           dx_tokens = sum of a token's dx rows; dweights = <dout, y rows>.
+ *
+ * The layout capacity is m_cap = mxmoe_route_capacity(T, top_k, E,
+ * pad_multiple); every row buffer below has m_cap rows and only the rows
+ * below offsets[E] (known on the device) are touched.  Needs D, F multiples
+ * of 128, pad_multiple a multiple of 128, 1 <= top_k <= min(64, E),
+ * E <= 1024.  Weights come from mxmoe_quantize_weights (ROW copies for the
+ * forward, COL copies for the backward).  topk_weights: fp32 [T, top_k].
+ * ------------------------------------------------------------------------- */
+typedef struct {
+  int32_t* offsets;    /* [E+1] */
+  int32_t* row_slot;   /* [m_cap] */
+  int32_t* slot_row;   /* [T*top_k] */
+  void* y;             /* bf16 [m_cap, D]: FC2 output rows (the combine's input) */
+  mxmoe_saved mlp;     /* h13 [m_cap, 2F], h COL, x COL, each with m_cap rows */
+} mxmoe_layer_saved;
+
+/* which = 1: forward workspace, 2: backward workspace (bytes; 0 on bad sizes). */
+size_t moe_layer_workspace_size(int64_t T, int top_k, int64_t D, int E, int64_t F, int pad_multiple, int which);
+
+int moe_layer_fwd_q(const void* x_tokens, int64_t T, int64_t D, const int32_t* topk_ids,
+                    const float* topk_weights, int top_k, const mxmoe_qweights* qw, int E, int64_t F,
+                    int pad_multiple, void* out_tokens, const mxmoe_layer_saved* saved,
+                    void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* dweights (fp32 [T, top_k]) may be NULL. */
+int moe_layer_bwd_q(const void* dout_tokens, int64_t T, int64_t D, const float* topk_weights, int top_k,
+                    const mxmoe_qweights* qw, int E, int64_t F, int pad_multiple,
+                    const mxmoe_layer_saved* saved, void* dx_tokens, void* dw13, void* dw2, float* dweights,
+                    void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

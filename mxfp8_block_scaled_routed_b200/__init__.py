@@ -22,7 +22,7 @@ __all__ = [
     "moe_mlp_fwd", "moe_mlp_bwd", "device_error", "header_functions",
     "make_qweights", "mxmoe_quantize_weights", "moe_mlp_fwd_q", "moe_mlp_bwd_q", "moe_mlp_fwd_unfused_q",
     "mxmoe_route_capacity", "mxmoe_route", "mxmoe_permute_quant", "mxmoe_unpermute_combine",
-    "mxmoe_combine_weight_grad",
+    "mxmoe_combine_weight_grad", "make_layer_saved", "moe_layer_fwd_q", "moe_layer_bwd_q",
 ]
 
 ROW, COL = 1, 2
@@ -47,6 +47,11 @@ class _Saved(ctypes.Structure):
 class _QWeights(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in ("w13_codes", "w13_scales", "w13t_codes", "w13t_scales",
                                                 "w2_codes", "w2_scales", "w2t_codes", "w2t_scales")]
+
+
+class _LayerSaved(ctypes.Structure):
+    _fields_ = [("offsets", ctypes.c_void_p), ("row_slot", ctypes.c_void_p), ("slot_row", ctypes.c_void_p),
+                ("y", ctypes.c_void_p), ("mlp", _Saved)]
 
 
 _P, _I, _L, _S = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
@@ -81,6 +86,11 @@ _SIGS = {
     "mxmoe_permute_quant": ([_P, _L, _L, _P, _I, _P, _L, _P, _I, _I, _P, _P, _P, _P, _P], _I),
     "mxmoe_unpermute_combine": ([_P, _L, _L, _P, _P, _L, _I, _P, _P], _I),
     "mxmoe_combine_weight_grad": ([_P, _P, _L, _L, _P, _L, _I, _P, _P], _I),
+    "moe_layer_workspace_size": ([_L, _I, _L, _I, _L, _I, _I], _S),
+    "moe_layer_fwd_q": ([_P, _L, _L, _P, _P, _I, ctypes.POINTER(_QWeights), _I, _L, _I, _P,
+                         ctypes.POINTER(_LayerSaved), _P, _S, _P], _I),
+    "moe_layer_bwd_q": ([_P, _L, _L, _P, _I, ctypes.POINTER(_QWeights), _I, _L, _I, ctypes.POINTER(_LayerSaved),
+                         _P, _P, _P, _P, _P, _S, _P], _I),
 }
 
 _lib = None
@@ -473,3 +483,64 @@ def mxmoe_combine_weight_grad(dout: torch.Tensor, y: torch.Tensor, slot_row: tor
     _check(lib().mxmoe_combine_weight_grad(_ptr(dout), _ptr(y), y.shape[0], D, _ptr(slot_row), T, top_k,
                                            _ptr(dw), _stream(dout)))
     return dw
+
+
+# ----------------------------------------------------------------------------- layer composites
+def layer_workspace_bytes(T, top_k, D, E, F, pad_multiple, which):
+    return int(lib().moe_layer_workspace_size(T, top_k, D, E, F, pad_multiple, which))
+
+
+def make_layer_saved(T, top_k, D, E, F, pad_multiple, device):
+    """Buffers the layer forward keeps for its backward (m_cap rows each)."""
+    m = mxmoe_route_capacity(T, top_k, E, pad_multiple)
+    i32 = lambda n: torch.empty(n, dtype=torch.int32, device=device)
+    return dict(offsets=i32(E + 1), row_slot=i32(m), slot_row=i32(T * top_k),
+                y=torch.empty(m, D, dtype=torch.bfloat16, device=device), mlp=make_saved(m, D, F, device))
+
+
+def _layer_struct(s):
+    return _LayerSaved(s["offsets"].data_ptr(), s["row_slot"].data_ptr(), s["slot_row"].data_ptr(),
+                       s["y"].data_ptr(), _saved_struct(s["mlp"]))
+
+
+def moe_layer_fwd_q(x_tokens, topk_ids, topk_weights, qw, pad_multiple=256, out=None, saved=None, workspace=None):
+    """Token-major layer forward: route, gather + cast, MLP, weighted combine. Returns (out, saved)."""
+    _need(x_tokens, torch.bfloat16, "x_tokens")
+    _need(topk_ids, torch.int32, "topk_ids")
+    _need(topk_weights, torch.float32, "topk_weights")
+    T, D = x_tokens.shape
+    k = topk_ids.shape[1]
+    E, F = qw["w13_codes"].shape[0], qw["w13_codes"].shape[1] // 2
+    dev = x_tokens.device
+    out = torch.empty(T, D, dtype=torch.bfloat16, device=dev) if out is None else out
+    saved = make_layer_saved(T, k, D, E, F, pad_multiple, dev) if saved is None else saved
+    ws = _u8((layer_workspace_bytes(T, k, D, E, F, pad_multiple, 1),), dev) if workspace is None else workspace
+    st, q = _layer_struct(saved), _qw_struct(qw)
+    _check(lib().moe_layer_fwd_q(_ptr(x_tokens), T, D, _ptr(topk_ids), _ptr(topk_weights), k, ctypes.byref(q), E, F,
+                                 pad_multiple, _ptr(out), ctypes.byref(st), _ptr(ws), ws.numel(), _stream(x_tokens)))
+    return out, saved
+
+
+def moe_layer_bwd_q(dout_tokens, topk_weights, qw, saved, pad_multiple=256, dx=None, dw13=None, dw2=None,
+                    dweights=True, workspace=None):
+    """Token-major layer backward. Returns (dx_tokens, dw13, dw2, dweights or None)."""
+    _need(dout_tokens, torch.bfloat16, "dout_tokens")
+    _need(topk_weights, torch.float32, "topk_weights")
+    T, D = dout_tokens.shape
+    k = topk_weights.shape[1]
+    E, F = qw["w13t_codes"].shape[0], qw["w13t_codes"].shape[2] // 2
+    dev = dout_tokens.device
+    dx = torch.empty(T, D, dtype=torch.bfloat16, device=dev) if dx is None else dx
+    dw13 = torch.empty(E, 2 * F, D, dtype=torch.bfloat16, device=dev) if dw13 is None else dw13
+    dw2 = torch.empty(E, D, F, dtype=torch.bfloat16, device=dev) if dw2 is None else dw2
+    dwr = None
+    if dweights is True:
+        dwr = torch.empty(T, k, dtype=torch.float32, device=dev)
+    elif isinstance(dweights, torch.Tensor):
+        dwr = dweights
+    ws = _u8((layer_workspace_bytes(T, k, D, E, F, pad_multiple, 2),), dev) if workspace is None else workspace
+    st, q = _layer_struct(saved), _qw_struct(qw)
+    _check(lib().moe_layer_bwd_q(_ptr(dout_tokens), T, D, _ptr(topk_weights), k, ctypes.byref(q), E, F, pad_multiple,
+                                 ctypes.byref(st), _ptr(dx), _ptr(dw13), _ptr(dw2), _ptr(dwr), _ptr(ws), ws.numel(),
+                                 _stream(dout_tokens)))
+    return dx, dw13, dw2, dwr

@@ -612,6 +612,66 @@ uint8_t* align_ws(void* ws) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(ws) + 255) & ~uintptr_t(255));
 }
 
+// ---------------------------------------------------------------- layer composites
+// Token-major layer: routing + gather/cast in front of the MLP, combine behind.
+struct LayerFwdWs {
+  FwdWs mlp;
+  int32_t* route_ws;
+};
+struct LayerBwdWs {
+  BwdWs mlp;
+  uint16_t* dx_rows;   // dx of the padded rows, before the unpermute
+};
+
+int64_t route_chunks(int64_t T, int k) { return (T * k + kRouteChunk - 1) / kRouteChunk; }
+
+size_t carve_layer_fwd(uint8_t* base, int64_t T, int k, int64_t m_cap, int64_t D, int E, int64_t F, LayerFwdWs* w) {
+  Carver c{base};
+  w->mlp.x_rc = c.take<uint8_t>(m_cap * D);
+  w->mlp.x_rs = c.take<uint8_t>(m_cap * D / 32);
+  w->mlp.h_rc = c.take<uint8_t>(m_cap * F);
+  w->mlp.h_rs = c.take<uint8_t>(m_cap * F / 32);
+  w->mlp.qw = mxmoe_qweights{};
+  w->route_ws = c.take<int32_t>(size_t(route_chunks(T, k)) * E * 4 + 16);
+  return c.off + 256;
+}
+
+size_t carve_layer_bwd(uint8_t* base, int64_t m_cap, int64_t D, int E, int64_t F, LayerBwdWs* w) {
+  Carver c{base};
+  BwdWs& b = w->mlp;
+  b.dy_rc = c.take<uint8_t>(m_cap * D);
+  b.dy_rs = c.take<uint8_t>(m_cap * D / 32);
+  b.dy_cc = c.take<uint8_t>(m_cap * D);
+  b.dy_cs = c.take<uint8_t>(m_cap * D / 32);
+  b.g_rc = c.take<uint8_t>(m_cap * 2 * F);
+  b.g_rs = c.take<uint8_t>(m_cap * 2 * F / 32);
+  b.g_cc = c.take<uint8_t>(m_cap * 2 * F);
+  b.g_cs = c.take<uint8_t>(m_cap * 2 * F / 32);
+  b.qw = mxmoe_qweights{};
+  w->dx_rows = c.take<uint16_t>(m_cap * D * 2);
+  return c.off + 256;
+}
+
+int check_layer_args(int64_t T, int64_t D, int top_k, int E, int64_t F, int pad, int64_t* m_cap) {
+  if (T <= 0 || top_k <= 0 || top_k > 64 || top_k > E)
+    return fail(MXMOE_ERR_SHAPE, "T=%lld top_k=%d (1..min(64, E)) E=%d", (long long)T, top_k, E);
+  if (E > kRouteMaxE) return fail(MXMOE_ERR_SHAPE, "E=%d exceeds %d", E, kRouteMaxE);
+  if (pad <= 0 || pad % 128 != 0) return fail(MXMOE_ERR_SHAPE, "pad_multiple=%d must be a positive multiple of 128", pad);
+  MX_TRY(check_mult("D", D, 128));
+  MX_TRY(check_mult("F", F, 128));
+  if (T > 0x7FFFFFFF / top_k) return fail(MXMOE_ERR_SHAPE, "T*top_k must be below 2^31");
+  *m_cap = mxmoe_route_capacity(T, top_k, E, pad);
+  if (*m_cap <= 0 || *m_cap >= (int64_t(1) << 31)) return fail(MXMOE_ERR_SHAPE, "layer too large");
+  return MXMOE_OK;
+}
+
+int check_layer_saved(const mxmoe_layer_saved* s) {
+  if (!s) return fail(MXMOE_ERR_NULL, "layer saved is NULL");
+  MX_TRY(check_ptrs({{"saved.offsets", s->offsets}, {"saved.row_slot", s->row_slot},
+                     {"saved.slot_row", s->slot_row}, {"saved.y", s->y}}));
+  return check_saved(&s->mlp);
+}
+
 }  // namespace
 
 // One thread waits on a barrier nothing arrives on: the bounded wait gives up
@@ -1042,6 +1102,88 @@ int mxmoe_combine_weight_grad(const void* dout, const void* y, int64_t m_rows, i
                                                              static_cast<const uint16_t*>(y), m_rows, slot_row,
                                                              top_k, D, dweights);
   MX_CHECK_CUDA(cudaGetLastError(), "combine weight-grad launch");
+  return MXMOE_OK;
+}
+
+// ---------------------------------------------------------------- layer composites
+size_t moe_layer_workspace_size(int64_t T, int top_k, int64_t D, int E, int64_t F, int pad_multiple, int which) {
+  if (T <= 0 || top_k <= 0 || D <= 0 || E <= 0 || F <= 0 || pad_multiple <= 0) return 0;
+  const int64_t m_cap = mxmoe_route_capacity(T, top_k, E, pad_multiple);
+  if (m_cap <= 0) return 0;
+  LayerFwdWs f;
+  LayerBwdWs b;
+  if (which == 1) return carve_layer_fwd(nullptr, T, top_k, m_cap, D, E, F, &f);
+  if (which == 2) return carve_layer_bwd(nullptr, m_cap, D, E, F, &b);
+  return 0;
+}
+
+int moe_layer_fwd_q(const void* x_tokens, int64_t T, int64_t D, const int32_t* topk_ids, const float* topk_weights,
+                    int top_k, const mxmoe_qweights* qw, int E, int64_t F, int pad_multiple, void* out_tokens,
+                    const mxmoe_layer_saved* saved, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  int64_t m_cap = 0;
+  MX_TRY(check_layer_args(T, D, top_k, E, F, pad_multiple, &m_cap));
+  MX_TRY(check_ptrs({{"x_tokens", x_tokens}, {"out_tokens", out_tokens}}));
+  if (!topk_ids || !topk_weights) return fail(MXMOE_ERR_NULL, "topk_ids/topk_weights is NULL");
+  MX_TRY(check_qweights(qw, true, false));
+  MX_TRY(check_layer_saved(saved));
+  LayerFwdWs w;
+  const size_t need = carve_layer_fwd(nullptr, T, top_k, m_cap, D, E, F, &w);
+  if (!workspace || workspace_bytes < need)
+    return fail(MXMOE_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed", workspace_bytes, need);
+  carve_layer_fwd(align_ws(workspace), T, top_k, m_cap, D, E, F, &w);
+  const int32_t* rows_dev = saved->offsets + E;
+  // routing -> padded expert-major layout
+  MX_TRY(mxmoe_route(topk_ids, T, top_k, E, pad_multiple, m_cap, saved->offsets, saved->row_slot, saved->slot_row,
+                     w.route_ws, size_t(route_chunks(T, top_k)) * E * 4 + 16, stream));
+  // a1 fused with the gather: token rows -> x ROW (FC1) + COL (dW13, saved)
+  GatherArgs g{saved->row_slot, nullptr, T * top_k, top_k};
+  MX_TRY(launch_cast<kCastGather>(x_tokens, 1, m_cap, D, MXFP8_ROW | MXFP8_COL, MXFP8_SCALE_MMA, w.mlp.x_rc,
+                                  w.mlp.x_rs, saved->mlp.x_col_codes, saved->mlp.x_col_scales, rows_dev, stream, &g));
+  // a3, a4
+  MX_TRY(gemm_swiglu(w.mlp.x_rc, w.mlp.x_rs, m_cap, D, qw->w13_codes, qw->w13_scales, E, F, saved->offsets,
+                     pad_multiple, saved->mlp.h13, w.mlp.h_rc, w.mlp.h_rs, saved->mlp.h_col_codes,
+                     saved->mlp.h_col_scales, stream));
+  MX_TRY(gemm_ragged_m(w.mlp.h_rc, w.mlp.h_rs, m_cap, F, qw->w2_codes, qw->w2_scales, E, D, saved->offsets,
+                       pad_multiple, saved->y, stream));
+  // weighted combine back to token order
+  return mxmoe_unpermute_combine(saved->y, m_cap, D, saved->slot_row, topk_weights, T, top_k, out_tokens, stream);
+}
+
+int moe_layer_bwd_q(const void* dout_tokens, int64_t T, int64_t D, const float* topk_weights, int top_k,
+                    const mxmoe_qweights* qw, int E, int64_t F, int pad_multiple, const mxmoe_layer_saved* saved,
+                    void* dx_tokens, void* dw13, void* dw2, float* dweights, void* workspace, size_t workspace_bytes,
+                    cudaStream_t stream) {
+  int64_t m_cap = 0;
+  MX_TRY(check_layer_args(T, D, top_k, E, F, pad_multiple, &m_cap));
+  MX_TRY(check_ptrs({{"dout_tokens", dout_tokens}, {"dx_tokens", dx_tokens}, {"dw13", dw13}, {"dw2", dw2}}));
+  if (!topk_weights) return fail(MXMOE_ERR_NULL, "topk_weights is NULL");
+  MX_TRY(check_qweights(qw, false, true));
+  MX_TRY(check_layer_saved(saved));
+  LayerBwdWs w;
+  const size_t need = carve_layer_bwd(nullptr, m_cap, D, E, F, &w);
+  if (!workspace || workspace_bytes < need)
+    return fail(MXMOE_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed", workspace_bytes, need);
+  carve_layer_bwd(align_ws(workspace), m_cap, D, E, F, &w);
+  const int32_t* rows_dev = saved->offsets + E;
+  // a5 fused with the gather: dY rows = bf16(w * dout[token]) -> ROW (dh) + COL (dW2)
+  GatherArgs g{saved->row_slot, topk_weights, T * top_k, top_k};
+  MX_TRY(launch_cast<kCastGather>(dout_tokens, 1, m_cap, D, MXFP8_ROW | MXFP8_COL, MXFP8_SCALE_MMA, w.mlp.dy_rc,
+                                  w.mlp.dy_rs, w.mlp.dy_cc, w.mlp.dy_cs, rows_dev, stream, &g));
+  const BwdWs& b = w.mlp;
+  const mxmoe_saved* ms = &saved->mlp;
+  // a6 - a9
+  MX_TRY(gemm_dswiglu(b.dy_rc, b.dy_rs, m_cap, D, qw->w2t_codes, qw->w2t_scales, E, F, saved->offsets, pad_multiple,
+                      ms->h13, b.g_rc, b.g_rs, b.g_cc, b.g_cs, stream));
+  MX_TRY(gemm_ragged_k(b.dy_cc, b.dy_cs, D, ms->h_col_codes, ms->h_col_scales, F, m_cap, saved->offsets, E,
+                       pad_multiple, dw2, stream));
+  MX_TRY(gemm_ragged_m(b.g_rc, b.g_rs, m_cap, 2 * F, qw->w13t_codes, qw->w13t_scales, E, D, saved->offsets,
+                       pad_multiple, w.dx_rows, stream));
+  MX_TRY(gemm_ragged_k(b.g_cc, b.g_cs, 2 * F, ms->x_col_codes, ms->x_col_scales, D, m_cap, saved->offsets, E,
+                       pad_multiple, dw13, stream));
+  // unpermute dx (sum over a token's copies) and the router-weight gradient
+  MX_TRY(mxmoe_unpermute_combine(w.dx_rows, m_cap, D, saved->slot_row, nullptr, T, top_k, dx_tokens, stream));
+  if (dweights)
+    MX_TRY(mxmoe_combine_weight_grad(dout_tokens, saved->y, m_cap, D, saved->slot_row, T, top_k, dweights, stream));
   return MXMOE_OK;
 }
 

@@ -239,3 +239,70 @@ def test_layer_forward_routes_runs_the_mlp_and_combines():
     # the FC2 output is bf16 at the GEMM boundary: the combine reads bf16 y
     ref = routing.unpermute_combine(mx.round_to_bf16(fwd["y"]), r["slot_row"], T, k, wr)
     assert_gemm_close(bf16_np(out), ref, "layer output")
+
+
+def _layer_inputs(spec, seed):
+    g = synth.rng(seed)
+    T, k, E, D, F = spec.tokens, spec.top_k, spec.E, spec.D, spec.F
+    topk = synth.make_routing(spec).topk
+    x = synth.to_bf16(synth.normal(g, (T, D)))
+    w13 = synth.to_bf16(synth.normal(g, (E, 2 * F, D), spec.w_std))
+    w2 = synth.to_bf16(synth.normal(g, (E, D, F), spec.w_std))
+    dout = synth.to_bf16(synth.normal(g, (T, D), spec.dy_std))
+    wr = synth.router_weights(T, k, seed=seed)
+    return topk, x, w13, w2, dout, wr
+
+
+def test_layer_composites_match_oracle_tiny():
+    spec = synth.SPECS["tiny"]
+    topk, x, w13, w2, dout, wr = _layer_inputs(spec, 41)
+    qw = mxk.mxmoe_quantize_weights(w13.to(DEV), w2.to(DEV))
+    tk, wt = torch.from_numpy(topk).to(DEV), torch.from_numpy(wr).to(DEV)
+    out, saved = mxk.moe_layer_fwd_q(x.to(DEV), tk, wt, qw, spec.pad)
+    dx, dw13, dw2, dwr = mxk.moe_layer_bwd_q(dout.to(DEV), wt, qw, saved, spec.pad)
+    torch.cuda.synchronize()
+    assert mxk.device_error() == 0
+    xn, w13n, w2n, dn = bf16_np(x), bf16_np(w13), bf16_np(w2), bf16_np(dout)
+    f = routing.layer_fwd(xn, topk, wr, w13n, w2n, spec.E, spec.pad)
+    b = routing.layer_bwd(dn, f, xn, topk, wr, w13n, w2n, spec.pad)
+    M = int(f["route"]["offsets"][-1])
+    np.testing.assert_array_equal(saved["offsets"].cpu().numpy(), f["route"]["offsets"])
+    np.testing.assert_array_equal(saved["row_slot"].cpu().numpy()[:M], f["route"]["row_slot"])
+    np.testing.assert_array_equal(saved["slot_row"].cpu().numpy(), f["route"]["slot_row"])
+    assert_gemm_close(bf16_np(out), f["out"], "layer out")
+    assert_gemm_close(bf16_np(dx), b["dx"], "layer dx")
+    assert_gemm_close(bf16_np(dw13), b["dw13"], "layer dW13")
+    assert_gemm_close(bf16_np(dw2), b["dw2"], "layer dW2")
+    assert_gemm_close(dwr.cpu().numpy(), b["dweights"], "layer router-weight gradient")
+
+
+@pytest.mark.parametrize("name", ["dsv3_16b"])
+def test_layer_composites_equal_the_row_composites_bitwise(name):
+    # the token-major layer = (torch gather) + the row-level composites +
+    # combine, bit for bit, at a DSv3-16B-like size
+    spec = synth.SPECS[name]
+    topk, x, w13, w2, dout, wr = _layer_inputs(spec, 43)
+    T, k, E, D, F = spec.tokens, spec.top_k, spec.E, spec.D, spec.F
+    x, dout = x.to(DEV), dout.to(DEV)
+    qw = mxk.mxmoe_quantize_weights(w13.to(DEV), w2.to(DEV))
+    tk, wt = torch.from_numpy(topk).to(DEV), torch.from_numpy(wr).to(DEV)
+    out, saved = mxk.moe_layer_fwd_q(x, tk, wt, qw, spec.pad)
+    dx, dw13, dw2, dwr = mxk.moe_layer_bwd_q(dout, wt, qw, saved, spec.pad)
+    # the same layout fed to the row composites
+    off, rs, sr = saved["offsets"], saved["row_slot"].long(), saved["slot_row"]
+    real = rs >= 0
+    tok = torch.where(real, rs // k, 0)
+    x_rows = torch.where(real[:, None], x[tok], torch.zeros((), dtype=x.dtype, device=DEV))
+    wflat = wt.reshape(-1)
+    dy_rows = (wflat[torch.where(real, rs, 0)][:, None] * dout[tok].float()).to(torch.bfloat16)
+    dy_rows = torch.where(real[:, None], dy_rows, torch.zeros((), dtype=dy_rows.dtype, device=DEV))
+    y_rows, s2 = mxk.moe_mlp_fwd_q(x_rows, qw, off, spec.pad)
+    dx_rows, dw13b, dw2b = mxk.moe_mlp_bwd_q(dy_rows, qw, off, s2, spec.pad)
+    torch.cuda.synchronize()
+    assert mxk.device_error() == 0
+    M = int(off[-1].item())
+    assert torch.equal(saved["y"][:M], y_rows[:M])
+    assert torch.equal(out, mxk.mxmoe_unpermute_combine(y_rows, sr, k, wt))
+    assert torch.equal(dw13, dw13b) and torch.equal(dw2, dw2b)
+    assert torch.equal(dx, mxk.mxmoe_unpermute_combine(dx_rows, sr, k))
+    assert torch.equal(dwr, mxk.mxmoe_combine_weight_grad(dout, y_rows, sr, k))
