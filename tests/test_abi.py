@@ -136,3 +136,26 @@ def test_dispatcher_rejects(L):
     assert s == 2
     s = L.mxmoe_combine_weight_grad(P(FAKE), P(MIS), 256, 128, P(FAKE), 16, 2, P(FAKE), None)
     assert s == 3
+
+
+def test_layer_composites_reject(L):
+    T, k, D, E, F, pad = 512, 2, 256, 4, 256, 128
+    need_f = L.moe_layer_workspace_size(T, k, D, E, F, pad, 1)
+    need_b = L.moe_layer_workspace_size(T, k, D, E, F, pad, 2)
+    m_cap = L.mxmoe_route_capacity(T, k, E, pad)
+    assert need_f >= m_cap * D + m_cap * F and need_b >= 2 * m_cap * D + 4 * m_cap * F + 2 * m_cap * D
+    assert L.moe_layer_workspace_size(T, k, D, E, F, pad, 3) == 0
+    saved = mxk._LayerSaved(FAKE, FAKE, FAKE, FAKE, mxk._Saved(FAKE, FAKE, FAKE, FAKE, FAKE))
+    qw = mxk._QWeights(*([FAKE] * 8))
+    s = L.moe_layer_fwd_q(P(FAKE), T, D, P(FAKE), P(FAKE), k, ctypes.byref(qw), E, F, 100, P(FAKE),
+                          ctypes.byref(saved), P(FAKE), need_f, None)
+    assert s == 2 and "pad_multiple" in _err(L)
+    s = L.moe_layer_fwd_q(P(FAKE), T, D, P(FAKE), P(FAKE), 5, ctypes.byref(qw), E, F, pad, P(FAKE),
+                          ctypes.byref(saved), P(FAKE), need_f, None)
+    assert s == 2 and "top_k" in _err(L)
+    s = L.moe_layer_fwd_q(P(FAKE), T, D, P(FAKE), P(FAKE), k, ctypes.byref(qw), E, F, pad, P(FAKE),
+                          ctypes.byref(saved), P(FAKE), need_f - 1, None)
+    assert s == 8 and "workspace" in _err(L)
+    s = L.moe_layer_bwd_q(P(FAKE), T, D, None, k, ctypes.byref(qw), E, F, pad, ctypes.byref(saved), P(FAKE),
+                          P(FAKE), P(FAKE), None, P(FAKE), need_b, None)
+    assert s == 1
