@@ -73,8 +73,12 @@ typedef enum {
 /* Text of the last host-side error of the calling thread ("" if none). */
 const char* mxmoe_last_error(void);
 
-/* Device-side error word of the current device (a GEMM kernel that found a
- * bad offsets table or whose bounded mbarrier wait expired sets it).
+/* Device-side error word of the current device.  Kernels set it when they
+ * find a bad table (GEMMs: an offsets table -> MXMOE_ERR_OFFSETS; route: an
+ * expert id outside [0, E) -> MXMOE_ERR_ARG, a layout past m_cap ->
+ * MXMOE_ERR_SHAPE; gather/combine: a slot or row out of range ->
+ * MXMOE_ERR_OFFSETS) or when a bounded mbarrier wait expires
+ * (MXMOE_ERR_DEVICE_TIMEOUT).
  * Synchronizes `stream`, returns the first error code recorded (MXMOE_OK if
  * none) in *code and, if reset != 0, clears it.  Returns MXMOE_ERR_CUDA if
  * the read itself failed. */
