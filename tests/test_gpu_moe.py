@@ -318,3 +318,37 @@ def test_dense_feedforward_is_the_one_expert_case():
     assert_gemm_close(bf16_np(dx), rb["dx"], "dx")
     assert_gemm_close(bf16_np(dw13), rb["dw13"], "dw13")
     assert_gemm_close(bf16_np(dw2), rb["dw2"], "dw2")
+
+
+def _sqnr_db(x, ref):
+    err = np.linalg.norm(np.asarray(x, dtype=np.float64) - ref)
+    return float(20.0 * np.log10(np.linalg.norm(ref) / max(err, 1e-300)))
+
+
+@pytest.mark.parametrize("name", ["tiny", "dsv3_16b"])
+def test_sqnr_against_the_unquantized_layer_tracks_the_oracle(name):
+    # SQNR tracking (SwiGLU-boundary page, "Numerics and tests"): the GPU
+    # MXFP8 outputs, measured against the same layer without quantization
+    # (oracle exact mode, float64), lose no more signal than the oracle's own
+    # MXFP8 arithmetic does: within 0.3 dB of it, and above 20 dB.
+    spec = synth.SPECS[name]
+    inp = synth.make_moe_inputs(spec, 3)
+    y, saved, dx, dw13, dw2 = _run(inp)
+    x, w13, w2, dy = _np(inp)
+    off = inp.routing.offsets
+    experts = None if name == "tiny" else sorted(int(e) for e in np.argsort(-inp.routing.counts)[:2])
+    segs = ([(e, off[e], off[e + 1]) for e in experts] if experts else [(None, 0, int(off[-1]))])
+    f_mx = mx.moe_mlp_fwd(x, w13, w2, off, experts)
+    b_mx = mx.moe_mlp_bwd(dy, f_mx, x, w13, w2, off, experts)
+    f_ex = mx.moe_mlp_fwd(x, w13, w2, off, experts, exact=True)
+    b_ex = mx.moe_mlp_bwd(dy, f_ex, x, w13, w2, off, experts, exact=True)
+    rows = np.concatenate([np.arange(lo, hi) for _, lo, hi in segs])
+    ex = slice(None) if experts is None else experts
+    for what, got, mxv, exv in (
+            ("y", bf16_np(y)[rows], f_mx["y"][rows], f_ex["y"][rows]),
+            ("dx", bf16_np(dx)[rows], b_mx["dx"][rows], b_ex["dx"][rows]),
+            ("dW13", bf16_np(dw13)[ex], b_mx["dw13"][ex], b_ex["dw13"][ex]),
+            ("dW2", bf16_np(dw2)[ex], b_mx["dw2"][ex], b_ex["dw2"][ex])):
+        s_gpu, s_oracle = _sqnr_db(got, exv), _sqnr_db(mxv, exv)
+        assert s_gpu >= 20.0, f"{what}: SQNR {s_gpu:.1f} dB"
+        assert s_gpu >= s_oracle - 0.3, f"{what}: GPU {s_gpu:.2f} dB vs oracle MXFP8 {s_oracle:.2f} dB"
