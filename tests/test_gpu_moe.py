@@ -352,3 +352,45 @@ def test_sqnr_against_the_unquantized_layer_tracks_the_oracle(name):
         s_gpu, s_oracle = _sqnr_db(got, exv), _sqnr_db(mxv, exv)
         assert s_gpu >= 20.0, f"{what}: SQNR {s_gpu:.1f} dB"
         assert s_gpu >= s_oracle - 0.3, f"{what}: GPU {s_gpu:.2f} dB vs oracle MXFP8 {s_oracle:.2f} dB"
+
+
+def _kernels_launched(fn):
+    from torch.profiler import ProfilerActivity, profile
+    torch.cuda.synchronize()
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        fn()
+        torch.cuda.synchronize()
+    names = [e.name for e in prof.events() if e.device_type == torch.autograd.DeviceType.CUDA]
+    return [n for n in names if "grouped_gemm" in n or "mx_" in n or "route_" in n or "combine" in n]
+
+
+def test_kernel_launch_counts():
+    # op-count contract (SwiGLU-boundary page, "Numerics and tests": profiler
+    # op-count contracts; "Summary": the fused boundary replaces the 6 + 6
+    # standalone casts): forward = x cast, FC1 with the fused SwiGLU + dual
+    # quant, FC2; the unfused plan adds one standalone SwiGLU cast; backward =
+    # dY cast, FC2 dgrad with the fused dSwiGLU + dual quant, dW2, dx, dW13.
+    inp = synth.make_moe_inputs("tiny", 0)
+    off = torch.from_numpy(inp.routing.offsets).to(DEV)
+    pad = inp.spec.pad
+    x, w13, w2, dy = (t.to(DEV) for t in (inp.x, inp.w13, inp.w2, inp.dy))
+    qw = mxk.mxmoe_quantize_weights(w13, w2)
+    y, saved = mxk.moe_mlp_fwd_q(x, qw, off, pad)
+    fwd = _kernels_launched(lambda: mxk.moe_mlp_fwd_q(x, qw, off, pad, y=y, saved=saved))
+    unf = _kernels_launched(lambda: mxk.moe_mlp_fwd_unfused_q(x, qw, off, pad, y=y, saved=saved))
+    bwd = _kernels_launched(lambda: mxk.moe_mlp_bwd_q(dy, qw, off, saved, pad))
+    assert len(fwd) == 3 and sum("mx_cast" in n for n in fwd) == 1, fwd
+    assert len(unf) == 4 and sum("mx_cast" in n for n in unf) == 2, unf
+    assert len(bwd) == 5 and sum("mx_cast" in n for n in bwd) == 1, bwd
+    # the token-major layer: 3 routing kernels, gather + cast, FC1, FC2, combine;
+    # backward: gather + cast, 4 GEMMs, unpermute, router-weight gradient
+    spec = inp.spec
+    tk = torch.from_numpy(inp.routing.topk).to(DEV)
+    wt = torch.from_numpy(synth.router_weights(spec.tokens, spec.top_k)).to(DEV)
+    xt = torch.randn(spec.tokens, spec.D, device=DEV).to(torch.bfloat16)
+    out, ls = mxk.moe_layer_fwd_q(xt, tk, wt, qw, pad)
+    lf = _kernels_launched(lambda: mxk.moe_layer_fwd_q(xt, tk, wt, qw, pad, out=out, saved=ls))
+    lb = _kernels_launched(lambda: mxk.moe_layer_bwd_q(xt, wt, qw, ls, pad))
+    assert len(lf) == 7 and sum("route_" in n for n in lf) == 3, lf
+    assert len(lb) == 7 and sum("combine" in n for n in lb) == 2, lb
+    assert mxk.device_error() == 0
