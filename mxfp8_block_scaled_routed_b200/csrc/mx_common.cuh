@@ -30,9 +30,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(b), "f"(a));
   return r;
 }
-__device__ __forceinline__ float round_bf16(float a) {
-  return __bfloat162float(__float2bfloat16_rn(a));
-}
 
 // max over |x| of eight packed bf16 (uint4) as a 15-bit magnitude pattern.
 // For non-negative floats the integer order of the bit patterns is the
@@ -106,30 +103,6 @@ __device__ __forceinline__ uint2 nan8_bf16(uint4 v) {
 // Quantize 8 packed bf16 given the block's scale byte.
 __device__ __forceinline__ uint2 encode8(uint4 v, uint32_t byte) {
   return byte == 0xFFu ? nan8_bf16(v) : quant8_bf16(v, inv_scale_from_byte(byte));
-}
-
-// ---------------------------------------------------------------- float-path helpers
-// max(a, |b|) that propagates NaN (an Inf/NaN anywhere in a block must reach
-// the block maximum).
-__device__ __forceinline__ float absmax_nan(float a, float b) {
-  float r;
-  asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(fabsf(b)));
-  return r;
-}
-
-// E8M0 byte from the block maximum as fp32 (|amax|, NaN/Inf -> 0xFF); same
-// rule as scale_byte_from_bits: max(expfield - 8, 0).
-__device__ __forceinline__ uint32_t scale_byte_from_f32(float amax, int emax = 8) {
-  const uint32_t b = __float_as_uint(amax);
-  if (b >= 0x7F800000u) return 0xFFu;
-  const int e = int(b >> 23) - emax;
-  return uint32_t(e < 0 ? 0 : e);
-}
-
-// Two codes of two bf16 held in one 32-bit word, scaled by inv.
-template <int kElem = 0>
-__device__ __forceinline__ uint32_t fp8x2_of_word(uint32_t w, float inv) {
-  return fp8x2<kElem>(bf16lo_to_f32(w) * inv, bf16hi_to_f32(w) * inv);
 }
 
 // ---------------------------------------------------------------- layouts

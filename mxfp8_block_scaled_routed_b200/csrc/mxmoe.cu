@@ -1064,6 +1064,8 @@ int mxmoe_permute_quant(const void* x_tokens, int64_t T, int64_t D, const int32_
     return fail(MXMOE_ERR_SHAPE, "MMA scale layout needs D and m_cap multiples of 128");
   if (!aligned16(x_tokens) || (row && !aligned16(row_codes)) || (col && !aligned16(col_codes)))
     return fail(MXMOE_ERR_ALIGN, "x_tokens and code buffers must be 16-byte aligned");
+  if (T > 0x7FFFFFFF / top_k || m_cap >= (int64_t(1) << 31))
+    return fail(MXMOE_ERR_SHAPE, "T*top_k and m_cap must be below 2^31");
   GatherArgs g{row_slot, slot_weights, T * top_k, top_k};
   return launch_cast<kCastGather>(x_tokens, 1, m_cap, D, modes, scale_layout, row_codes, row_scales, col_codes,
                                   col_scales, rows_dev, stream, &g);
