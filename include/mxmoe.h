@@ -12,6 +12,11 @@
  *   backward  dh  = dy_e . W2[e]; dh13 = dSwiGLU(dh, h13)  (fused)
  *             dW2[e] = dy_e^T . h_e, dx = dh13_e . W13[e], dW13[e] = dh13_e^T . x_e
  *
+ * around it the token dispatcher (routing to the padded expert-major layout,
+ * gather fused with the cast, weighted combine and its gradients; the
+ * moe_layer_* composites run the whole token-major layer), the standalone
+ * casts and dequantization (E4M3, and E5M2 for the transport payload).
+ *
  * MXFP8 format (A2E MXFP8 pages, "quant_mode=4 ... E4M3 ... E8M0 MX scale"):
  * each block of 32 consecutive elements is stored as 32 E4M3 codes (uint8)
  * plus one E8M0 scale byte.  Scale rule (OCP MX v1.0): shared exponent
