@@ -8,18 +8,20 @@
 //
 // Two schedules over the expert-major padded token layout:
 //  * ragged M: out[m, :] = A[m, :] . B[e]^T for the rows m of expert e
-//    (A = tokens x K, B = per-expert weights [E, N, K]); an M tile of 128
-//    rows never straddles two experts because segments are padded to 128.
-//    Zero-token experts own no M tile and are skipped.
+//    (A = tokens x K, B = per-expert weights [E, N, K]); an M tile (128 rows,
+//    256 on CTA pairs) never straddles two experts because segments are
+//    padded to a multiple of it.  Zero-token experts own no M tile.
 //  * ragged K: out[e] = A_e^T . B_e over expert e's token rows, with both
 //    operands column-quantized and stored transposed ([N, M] and [Kx, M]) so
 //    the token dimension is the contiguous contraction.  Experts without rows
 //    write exact zeros.
 //
-// CTA = 8 warps: warp 0 issues TMA/bulk copies, warp 1 issues tcgen05.mma,
-// warp 2 owns the TMEM allocation, warps 4..7 run the epilogue (warp 4+q
-// reads TMEM lanes 32q..32q+31, i.e. rows 32q.. of the 128-row tile).
-// Tile: 128 x BN x 128 (M x N x K bytes), 128-byte swizzled K-major operands.
+// CTA = 12 warps: warp 0 issues TMA/bulk copies, warp 1 issues tcgen05.mma,
+// warp 2 owns the TMEM allocation, warps 4..11 run the epilogue (warp 4+q and
+// 8+q read TMEM lanes 32q..32q+31, i.e. rows 32q.. of the 128-row tile, each
+// half of the columns).  Tile: 128 x BN x 128 (M x N x K bytes) per CTA,
+// 128-byte swizzled K-major operands; on a CTA pair (cta_group::2) the two
+// CTAs hold 128 rows each of a 256 x BN tile and one half of B each.
 // The E8M0 scales arrive as 512-byte atoms (MMA scale layout), are copied to
 // TMEM with tcgen05.cp and consumed by the block-scaled MMA (scale id = the
 // 32-wide K step inside the 128-wide K block).

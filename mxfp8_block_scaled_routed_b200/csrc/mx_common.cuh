@@ -1,10 +1,11 @@
 // Device-side MXFP8 helpers shared by the cast and GEMM-epilogue kernels.
 //
-// MXFP8 block (A2E MXFP8 pages: E4M3 elements with an E8M0 block scale):
-// 32 elements share one power-of-two scale 2^s with s = floor(log2(amax)) - 8,
-// stored as the byte s + 127 clamped to [0, 254]; elements are x / 2^s rounded
-// to nearest-even E4M3 and saturated to +-448.  A block holding NaN/Inf gets
-// byte 0xFF and codes 0x7F | sign.
+// MXFP8 block (A2E MXFP8 pages: E4M3 or E5M2 elements with an E8M0 block
+// scale): 32 elements share one power-of-two scale 2^s with
+// s = floor(log2(amax)) - emax (8 for E4M3, 15 for E5M2), stored as the byte
+// s + 127 clamped to [0, 254]; elements are x / 2^s rounded to nearest-even
+// and saturated (+-448, +-57344).  A block holding NaN/Inf gets byte 0xFF and
+// codes 0x7F | sign.
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>

@@ -1,9 +1,10 @@
 // libmxmoe: C ABI of the MXFP8 routed-experts MLP (declared in include/mxmoe.h).
 //
 // One translation unit: the cast kernels (quant.cuh), the tcgen05 grouped
-// GEMM (gemm.cuh) and the host code below, which validates every argument,
-// encodes the TMA tensor maps, launches on the caller's stream and chains
-// the forward/backward composites.  Nothing here allocates device memory.
+// GEMM (gemm.cuh), the token dispatcher (route.cuh) and the host code below,
+// which validates every argument, encodes the TMA tensor maps, launches on
+// the caller's stream and chains the composites.  Nothing here calls a
+// device allocator.
 #include <cuda.h>
 #include <cuda_runtime.h>
 

@@ -1,6 +1,7 @@
-// MXFP8 cast kernels: bf16 -> (E4M3 codes, E8M0 scales), row-wise and/or
-// column-wise in one pass, plus the fused SwiGLU + dual quantization and the
-// E8M0-endpoint-correct dequantization.
+// MXFP8 cast kernels: bf16 -> (E4M3 or E5M2 codes, E8M0 scales), row-wise
+// and/or column-wise in one pass, plus the fused SwiGLU + dual quantization,
+// the gather (token dispatcher) variant and the E8M0-endpoint-correct
+// dequantization.
 //
 // Standalone casts: SwiGLU-boundary page, "Summary" (the unfused path's
 // standalone cast kernels); A2E MXFP8 page ("the payload halves").
