@@ -403,9 +403,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
-    world, rank, local = dist_setup(args)
     if args.impl == "reference":
-        return run_reference(args, world, rank)
+        # rank 0 alone times the oracle; no process group, no collectives
+        return run_reference(args, int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")))
+    world, rank, local = dist_setup(args)
 
     assert torch.cuda.is_available(), "bench.py needs a GPU"
     dev = torch.device("cuda", local)
