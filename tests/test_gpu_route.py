@@ -276,15 +276,27 @@ def test_layer_composites_match_oracle_tiny():
     assert_gemm_close(dwr.cpu().numpy(), b["dweights"], "layer router-weight gradient")
 
 
-@pytest.mark.parametrize("name", ["dsv3_16b"])
+@pytest.mark.parametrize("name", ["dsv3_16b", "dsv3"])
 def test_layer_composites_equal_the_row_composites_bitwise(name):
     # the token-major layer = (torch gather) + the row-level composites +
-    # combine, bit for bit, at a DSv3-16B-like size
+    # combine, bit for bit, at the DSv3-16B-like size and at the DSv3 size the
+    # end-to-end measurement runs (there with device-drawn inputs)
     spec = synth.SPECS[name]
-    topk, x, w13, w2, dout, wr = _layer_inputs(spec, 43)
     T, k, E, D, F = spec.tokens, spec.top_k, spec.E, spec.D, spec.F
+    if name == "dsv3":
+        dinp = synth.device_moe_inputs(spec, 43, device=DEV)
+        topk, w13, w2 = dinp.routing.topk, dinp.w13, dinp.w2
+        x = dinp.x_tok
+        del dinp
+        gen = torch.Generator(device=DEV)
+        gen.manual_seed(44)
+        dout = (torch.randn(T, D, generator=gen, device=DEV) * spec.dy_std).to(torch.bfloat16)
+        wr = synth.router_weights(T, k, seed=43)
+    else:
+        topk, x, w13, w2, dout, wr = _layer_inputs(spec, 43)
     x, dout = x.to(DEV), dout.to(DEV)
     qw = mxk.mxmoe_quantize_weights(w13.to(DEV), w2.to(DEV))
+    del w13, w2
     tk, wt = torch.from_numpy(topk).to(DEV), torch.from_numpy(wr).to(DEV)
     out, saved = mxk.moe_layer_fwd_q(x, tk, wt, qw, spec.pad)
     dx, dw13, dw2, dwr = mxk.moe_layer_bwd_q(dout, wt, qw, saved, spec.pad)
