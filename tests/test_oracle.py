@@ -498,3 +498,95 @@ def test_nan_tail_never_read():
     np.testing.assert_array_equal(b0["dx"][:M], b1["dx"][:M])
     np.testing.assert_array_equal(b0["dw13"], b1["dw13"])
     np.testing.assert_array_equal(b0["dw2"], b1["dw2"])
+
+
+# ---------------------------------------------------------------- blocking axis of each GEMM operand
+# MX blocks run along the contraction dimension of every GEMM operand (the
+# MX definition scales 32 elements that enter the same dot product; the
+# fully-fused plan page, "What it adds": row-wise quantization for the forward,
+# column-wise for the backward contractions).  Each operand below is drawn so
+# that its quantization is the identity when its blocks run along its
+# contraction axis and destroys entries when they run along the other axis:
+# signed powers of two whose exponent is constant along the contraction axis
+# and sweeps 24 binades across any 32 consecutive positions of the other axis
+# (a block that mixes them holds magnitudes 2^24 apart; relative to the block
+# scale E4M3 reaches down to 2^-9 * 2^-8 only, so its small entries flush).
+# The GEMM outputs then have closed forms in terms of the unquantized operand.
+_NB = 160                     # expert rows (a multiple of 32, unlike every other dimension)
+_D, _F = 192, 128
+
+
+def _axis_exact(g, shape, contraction_axis):
+    """Powers of two (10 % zeros), exponent constant along contraction_axis."""
+    n_other = shape[1 - contraction_axis]
+    exp = (7 * np.arange(n_other)) % 25 - 12          # every 25 consecutive positions: all of -12..12
+    e = exp[:, None] if contraction_axis == 1 else exp[None, :]
+    sign = g.choice(np.array([-1.0, 1.0]), size=shape)
+    zero = g.random(shape) < 0.1
+    return np.where(zero, 0.0, sign * np.ldexp(1.0, np.broadcast_to(e, shape)))
+
+
+def _bf16_generic(g, shape, std):
+    return mx.round_to_bf16(g.normal(0.0, std, size=shape))
+
+
+def test_axis_pin_operands_of_the_exact_inputs_are_unchanged():
+    """The construction itself: exact under the contraction-axis blocking,
+    altered under the other blocking."""
+    g = np.random.default_rng(31)
+    a = _axis_exact(g, (_NB, _D), 1)                  # contraction along columns
+    np.testing.assert_array_equal(mx.dequantize_rows(*mx.quantize_rows(a)), a)
+    assert (mx.dequantize_rows(*mx.quantize_cols(a)).T != a).mean() > 0.2
+    b = _axis_exact(g, (_NB, _D), 0)                  # contraction along rows
+    np.testing.assert_array_equal(mx.dequantize_rows(*mx.quantize_cols(b)).T, b)
+    assert (mx.dequantize_rows(*mx.quantize_rows(b)) != b).mean() > 0.2
+
+
+def test_axis_pin_forward_operands():
+    """x, W13 blocked along D and W2 along F (and h along F): h13 and y
+    equal their closed forms on the unquantized x, W13, W2."""
+    g = np.random.default_rng(32)
+    x = _axis_exact(g, (_NB, _D), 1)                  # FC1 contracts D
+    w13 = _axis_exact(g, (2 * _F, _D), 1)             # FC1 contracts D
+    w2 = _axis_exact(g, (_D, _F), 1)                  # FC2 contracts F
+    r = mx.expert_fwd(x, w13, w2)
+    # every h13 entry is 2^k times an integer of at most 192: exact in float64 and bf16
+    np.testing.assert_array_equal(r["h13"], x @ w13.T)
+    hq = mx.dequantize_rows(*r["h_row"])
+    np.testing.assert_array_equal(r["y"], hq @ w2.T)
+    assert (np.abs(r["h13"]) > 0).mean() > 0.5 and (np.abs(r["y"]) > 0).mean() > 0.5
+
+
+def test_axis_pin_backward_dgrad_operands():
+    """dY blocked along D and W2 along D (dh), dh13 along 2F and W13 along 2F
+    (dx): dh and dx equal their closed forms on the unquantized dY, W2, W13."""
+    g = np.random.default_rng(33)
+    x = _bf16_generic(g, (_NB, _D), 1.0)
+    w13 = _axis_exact(g, (2 * _F, _D), 0)             # dx contracts 2F (the rows of W13)
+    w2 = _axis_exact(g, (_D, _F), 0)                  # dh contracts D (the rows of W2)
+    dy = _axis_exact(g, (_NB, _D), 1)                 # dh contracts D
+    f = mx.expert_fwd(x, w13, w2)
+    r = mx.expert_bwd(dy, f, x, w13, w2)
+    np.testing.assert_array_equal(r["dh"], dy @ w2)   # 2^k times integers of at most 192: exact
+    gq = mx.dequantize_rows(*r["dh13_row"])
+    np.testing.assert_array_equal(r["dx"], gq @ w13)
+    assert (np.abs(r["dh"]) > 0).mean() > 0.5 and (np.abs(r["dx"]) > 0).mean() > 0.5
+
+
+def test_axis_pin_backward_wgrad_operands():
+    """dY, h, dh13 and x blocked along the token rows (dW2, dW13): the weight
+    gradients equal their closed forms on the unquantized dY and x."""
+    g = np.random.default_rng(34)
+    x = _axis_exact(g, (_NB, _D), 0)                  # dW13 contracts the rows
+    dy = _axis_exact(g, (_NB, _D), 0)                 # dW2 contracts the rows
+    w13 = _bf16_generic(g, (2 * _F, _D), 0.05)
+    w2 = _bf16_generic(g, (_D, _F), 0.05)
+    f = mx.expert_fwd(x, w13, w2)
+    r = mx.expert_bwd(dy, f, x, w13, w2)
+    hc = mx.dequantize_rows(*f["h_col"])              # [F, n]
+    gc = mx.dequantize_rows(*r["dh13_col"])           # [2F, n]
+    np.testing.assert_array_equal(r["dw2"], dy.T @ hc.T)
+    np.testing.assert_array_equal(r["dw13"], gc @ x)
+    np.testing.assert_array_equal(mx.dequantize_rows(*f["x_col"]).T, x)
+    np.testing.assert_array_equal(mx.dequantize_rows(*r["dy_col"]).T, dy)
+    assert (np.abs(r["dw2"]) > 0).mean() > 0.5 and (np.abs(r["dw13"]) > 0).mean() > 0.5
