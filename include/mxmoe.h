@@ -29,7 +29,7 @@
  *    never allocates device memory (composites take a caller workspace).
  *  - bf16 tensors are passed as void* (IEEE bfloat16, row-major, dense).
  *  - Every call is asynchronous on `stream` and returns an mxmoe_status; on
- *    an error nothing is launched and mxmoe_last_error() names the argument.
+ *    an error nothing is launched and mxmoe_last_error_message() names the argument.
  *  - ROW quantization: blocks along the last (contiguous) dimension;
  *    COL quantization: blocks over 32 consecutive rows of one column, stored
  *    TRANSPOSED (codes [cols, rows]) so the contraction dimension is contiguous.
@@ -44,7 +44,7 @@
  *    every offset a multiple of pad_multiple (itself a multiple of 128), and
  *    offsets[E] <= M.  Rows at or past offsets[E] are never read or written.
  *    The GEMM kernels re-check this on the device; a bad table makes them do
- *    nothing and raises MXMOE_ERR_OFFSETS in mxmoe_device_error().
+ *    nothing and raises MXMOE_ERR_OFFSETS in mxmoe_check_device_error().
  */
 #ifndef MXMOE_H
 #define MXMOE_H
@@ -76,7 +76,7 @@ typedef enum {
 #define MXFP8_SCALE_MMA 1
 
 /* Text of the last host-side error of the calling thread ("" if none). */
-const char* mxmoe_last_error(void);
+const char* mxmoe_last_error_message(void);
 
 /* Device-side error word of the current device.  Kernels set it when they
  * find a bad table (GEMMs: an offsets table -> MXMOE_ERR_OFFSETS; route: an
@@ -87,7 +87,7 @@ const char* mxmoe_last_error(void);
  * Synchronizes `stream`, returns the first error code recorded (MXMOE_OK if
  * none) in *code and, if reset != 0, clears it.  Returns MXMOE_ERR_CUDA if
  * the read itself failed. */
-int mxmoe_device_error(cudaStream_t stream, int reset, int* code);
+int mxmoe_check_device_error(cudaStream_t stream, int reset, int* code);
 
 /* Library version string. */
 const char* mxmoe_version(void);
@@ -97,7 +97,7 @@ const char* mxmoe_version(void);
  * nothing ever arrives on.  After the wait limit (about 2^32 SM cycles, ~2 s)
  * the kernel records MXMOE_ERR_DEVICE_TIMEOUT in the device error word and
  * returns normally, leaving the context usable; read it with
- * mxmoe_device_error(). */
+ * mxmoe_check_device_error(). */
 int mxmoe_selftest_wait_timeout(cudaStream_t stream);
 
 /* -------------------------------------------------------------------------
@@ -341,7 +341,9 @@ int moe_mlp_bwd_q(const void* dy, int64_t M, int64_t D, const mxmoe_qweights* qw
  *    both sizes; nothing is launched.
  *  - The first call on a device looks up the device address of the scratch
  *    array (cudaGetSymbolAddress, with that device current); make that first
- *    call before any CUDA stream capture begins.
+ *    call before any CUDA stream capture begins.  The address is kept per
+ *    device and CUDA context: after cudaDeviceReset, or under another
+ *    context, the next call looks it up again (again outside any capture).
  *  - All calls on a device share the one scratch area, which keeps whatever
  *    the previous call left there (every byte a call reads is written by that
  *    call first).  Calls whose executions overlap on the GPU (different
@@ -387,7 +389,7 @@ size_t mxmoe_route_workspace_size(int64_t T, int top_k, int E);
 /* Build the padded expert-major layout from a top-k routing (three kernels:
  * per-chunk histogram, padded scan, stable ranking).
  *   topk_ids  DEVICE int32 [T, top_k], ids in [0, E) (ids outside raise
- *             MXMOE_ERR_ARG in mxmoe_device_error and their slot gets row -1)
+ *             MXMOE_ERR_ARG in mxmoe_check_device_error and their slot gets row -1)
  *   E <= 1024, pad_multiple >= 1, T*top_k < 2^31
  *   m_cap     rows of row_slot (use mxmoe_route_capacity); a routing that
  *             needs more raises MXMOE_ERR_SHAPE on the device and rows past

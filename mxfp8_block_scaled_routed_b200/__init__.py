@@ -56,9 +56,9 @@ class _LayerSaved(ctypes.Structure):
 
 _P, _I, _L, _S = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
 _SIGS = {
-    "mxmoe_last_error": ([], ctypes.c_char_p),
+    "mxmoe_last_error_message": ([], ctypes.c_char_p),
     "mxmoe_version": ([], ctypes.c_char_p),
-    "mxmoe_device_error": ([_P, _I, ctypes.POINTER(ctypes.c_int)], _I),
+    "mxmoe_check_device_error": ([_P, _I, ctypes.POINTER(ctypes.c_int)], _I),
     "mxfp8_quantize": ([_P, _L, _L, _L, _I, _I, _P, _P, _P, _P, _P], _I),
     "mxfp8_quantize_e5m2": ([_P, _L, _L, _L, _I, _I, _P, _P, _P, _P, _P], _I),
     "mxfp8_dequantize_e5m2": ([_P, _P, _L, _L, _P, _P], _I),
@@ -120,7 +120,7 @@ def header_functions() -> list[str]:
 
 def _check(status: int):
     if status != 0:
-        raise MXMOEError(status, lib().mxmoe_last_error().decode())
+        raise MXMOEError(status, lib().mxmoe_last_error_message().decode())
 
 
 def _stream(t: torch.Tensor):
@@ -150,7 +150,7 @@ def device_error(reset: bool = True, device=None) -> int:
     """First device-side error code recorded by the kernels (0 if none)."""
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
     code = ctypes.c_int(0)
-    _check(lib().mxmoe_device_error(ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream),
+    _check(lib().mxmoe_check_device_error(ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream),
                                     int(reset), ctypes.byref(code)))
     return code.value
 

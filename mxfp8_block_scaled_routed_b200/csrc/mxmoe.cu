@@ -133,17 +133,17 @@ struct GatherArgs {
   int top_k;
 };
 
-// 3-D bf16 cast input [batch, rows, ld], box 128 x 128 x 1, no swizzle, zero fill
-// past the edges.
+// 3-D bf16 cast input [batch, rows, ld], box 64 x 128 x 1 (128-byte rows) in the
+// 128-byte swizzle, zero fill past the edges.
 int make_cast_map(CUtensorMap* map, const void* base, int64_t batch, int64_t rows, int64_t ld) {
   EncodeTiledFn enc;
   MX_TRY(get_encode(&enc));
   cuuint64_t dims[3] = {cuuint64_t(ld), cuuint64_t(rows), cuuint64_t(batch)};
   cuuint64_t strides[2] = {cuuint64_t(ld * 2), cuuint64_t(rows * ld * 2)};
-  cuuint32_t box[3] = {128, 128, 1};
+  cuuint32_t box[3] = {64, 128, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(MXMOE_ERR_CUDA, "cuTensorMapEncodeTiled (cast) failed (%d)", int(r));
   return MXMOE_OK;
@@ -212,7 +212,7 @@ int launch_cast(const void* in, int64_t batch, int64_t rows, int64_t cols, int m
   const int64_t ntiles = batch * a.tiles_r * a.tiles_c;
   const int64_t per_sm = C::kCtasPerSm;
   const int grid = int(ntiles < per_sm * d->sms ? ntiles : per_sm * d->sms);
-  kern<<<grid, kCastThreads, C::kSmem, stream>>>(map, a);
+  kern<<<grid, C::kThreads, C::kSmem, stream>>>(map, a);
   MX_CHECK_CUDA(cudaGetLastError(), "cast launch");
   return MXMOE_OK;
 }
@@ -356,6 +356,8 @@ int quantize_impl(const void* x, int64_t batch, int64_t rows, int64_t cols, int 
   if (layout == MXFP8_SCALE_MMA && (rows % 128 != 0 || cols % 128 != 0))
     return fail(MXMOE_ERR_SHAPE, "MMA scale layout needs rows and cols multiples of 128 (%lld x %lld)",
                 (long long)rows, (long long)cols);
+  if (layout == MXFP8_SCALE_MMA && ((row && !aligned16(rs)) || (col && !aligned16(cs))))
+    return fail(MXMOE_ERR_ALIGN, "MMA-layout scale buffers must be 16-byte aligned");
   const bool vec_ok = cols % 32 == 0 && aligned16(x) && (!row || aligned16(rc)) && (!col || aligned16(cc)) &&
                       (!col || rows % 16 == 0);
   if (swiglu && !vec_ok) return fail(MXMOE_ERR_SHAPE, "SwiGLU quant needs F %% 32 == 0 and 16-byte aligned buffers");
@@ -429,9 +431,12 @@ int gemm_ragged_k(const uint8_t* gt, const uint8_t* gs, int64_t N, const uint8_t
   p.out = static_cast<uint16_t*>(dw);
   // (CTA pairs measured slower here: experts' short K leave little mainloop
   // to hide the pair's per-tile accumulator hand-off)
-  if (MXMOE_WGRAD_PAIRS && Kx % 256 == 0 && N % 256 == 0)
+  if (MXMOE_WGRAD_PAIRS == 1 && Kx % 256 == 0 && N % 256 == 0)
     return launch_gemm<gemm::kRaggedK, gemm::kEpiBF16, 256, true>(gt, N, xt, Kx, p,
                                                                   int64_t(E) * (N / 256) * (Kx / 256), stream, 10);
+  if (MXMOE_WGRAD_PAIRS == 2 && N % 256 == 0)
+    return launch_gemm<gemm::kRaggedK, gemm::kEpiBF16, 128, true>(gt, N, xt, Kx, p,
+                                                                  int64_t(E) * (N / 256) * (Kx / 128), stream, 16);
   if (Kx % 256 == 0 && MXMOE_WGRAD_BN == 256)
     return launch_gemm<gemm::kRaggedK, gemm::kEpiBF16, 256, false>(gt, N, xt, Kx, p,
                                                                    int64_t(E) * (N / 128) * (Kx / 256), stream, 2);
@@ -729,11 +734,11 @@ int mxmoe_selftest_wait_timeout(cudaStream_t stream) {
   return MXMOE_OK;
 }
 
-const char* mxmoe_last_error(void) { return g_err; }
+const char* mxmoe_last_error_message(void) { return g_err; }
 
 const char* mxmoe_version(void) { return "mxmoe 0.1 (sm_100a, tcgen05 block-scaled MXFP8)"; }
 
-int mxmoe_device_error(cudaStream_t stream, int reset, int* code) {
+int mxmoe_check_device_error(cudaStream_t stream, int reset, int* code) {
   if (!code) return fail(MXMOE_ERR_NULL, "code is NULL");
   MX_CHECK_CUDA(cudaStreamSynchronize(stream), "cudaStreamSynchronize");
   int v = 0;
@@ -952,15 +957,62 @@ int moe_mlp_bwd_q(const void* dy, int64_t M, int64_t D, const mxmoe_qweights* qw
   return bwd_core(dy, M, D, *qw, E, F, expert_offsets, pad_multiple, saved, dx, dw13, dw2, w, stream);
 }
 
+}  // extern "C"
+
 // Forward composite for callers that cannot allocate (see the header): the
-// workspace is a static device array of this translation unit.  Its device
-// address is looked up once per device and cached.
+// workspace is a static device array of this translation unit.  Host code
+// cannot use the array's name as a device address, so its address is looked
+// up with cudaGetSymbolAddress, once per device and CUDA context (a reset
+// device or a new context gets a fresh lookup), and passed to the kernels.
 static __device__ __align__(256) uint8_t g_noalloc_scratch[MXMOE_NOALLOC_SCRATCH_BYTES];
 
-int moe_mlp_fwd_noalloc(const void* x, int64_t M, int64_t D, const void* w13, const void* w2, int E, int64_t F,
-                        const int32_t* expert_offsets, int pad_multiple, void* y, const mxmoe_saved* saved,
-                        cudaStream_t stream) {
-  static void* scratch_ptr[kMaxDevices] = {};
+namespace {
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+
+int current_context(CUcontext* ctx) {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  if (!fn) return fail(MXMOE_ERR_CUDA, "cuCtxGetCurrent unavailable");
+  if (fn(ctx) != CUDA_SUCCESS) return fail(MXMOE_ERR_CUDA, "cuCtxGetCurrent failed");
+  return MXMOE_OK;
+}
+
+struct ScratchAddr {
+  CUcontext ctx = nullptr;
+  void* ptr = nullptr;
+};
+ScratchAddr g_scratch[kMaxDevices];
+
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  MX_CHECK_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(MXMOE_ERR_CUDA, "device index %d out of range", dev);
+  CUcontext ctx = nullptr;
+  MX_TRY(current_context(&ctx));
+  std::lock_guard<std::mutex> lk(g_mu);
+  ScratchAddr& a = g_scratch[dev];
+  if (ctx == nullptr || a.ptr == nullptr || a.ctx != ctx) {
+    void* p = nullptr;
+    MX_CHECK_CUDA(cudaGetSymbolAddress(&p, g_noalloc_scratch), "cudaGetSymbolAddress(scratch)");
+    MX_TRY(current_context(&ctx));     // the lookup made the device's context current if it was not
+    a.ctx = ctx;
+    a.ptr = p;
+  }
+  *out = a.ptr;
+  return MXMOE_OK;
+}
+}  // namespace
+
+extern "C" int moe_mlp_fwd_noalloc(const void* x, int64_t M, int64_t D, const void* w13, const void* w2, int E,
+                                   int64_t F, const int32_t* expert_offsets, int pad_multiple, void* y,
+                                   const mxmoe_saved* saved, cudaStream_t stream) {
   MX_TRY(check_mlp_shapes(M, D, E, F, expert_offsets, pad_multiple));
   FwdWs w;
   const size_t need = carve_fwd(nullptr, M, D, E, F, &w, true);
@@ -969,23 +1021,13 @@ int moe_mlp_fwd_noalloc(const void* x, int64_t M, int64_t D, const void* w13, co
                 "moe_mlp_fwd_noalloc: this layer needs %zu bytes of scratch, the static scratch holds %zu; "
                 "use moe_mlp_fwd with a caller workspace",
                 need, (size_t)MXMOE_NOALLOC_SCRATCH_BYTES);
-  int dev = 0;
-  MX_CHECK_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
-  if (dev < 0 || dev >= kMaxDevices) return fail(MXMOE_ERR_CUDA, "device index %d out of range", dev);
   void* ws = nullptr;
-  {
-    std::lock_guard<std::mutex> lk(g_mu);
-    if (!scratch_ptr[dev]) {
-      void* p = nullptr;
-      MX_CHECK_CUDA(cudaGetSymbolAddress(&p, g_noalloc_scratch), "cudaGetSymbolAddress(scratch)");
-      scratch_ptr[dev] = p;
-    }
-    ws = scratch_ptr[dev];
-  }
+  MX_TRY(noalloc_scratch(&ws));
   return moe_mlp_fwd(x, M, D, w13, w2, E, F, expert_offsets, pad_multiple, y, saved, ws,
                      MXMOE_NOALLOC_SCRATCH_BYTES, stream);
 }
 
+extern "C" {
 // ---------------------------------------------------------------- dispatcher
 int64_t mxmoe_route_capacity(int64_t T, int top_k, int E, int pad_multiple) {
   if (T < 0 || top_k <= 0 || E <= 0 || pad_multiple <= 0) return -1;
@@ -1065,6 +1107,8 @@ int mxmoe_permute_quant(const void* x_tokens, int64_t T, int64_t D, const int32_
     return fail(MXMOE_ERR_SHAPE, "MMA scale layout needs D and m_cap multiples of 128");
   if (!aligned16(x_tokens) || (row && !aligned16(row_codes)) || (col && !aligned16(col_codes)))
     return fail(MXMOE_ERR_ALIGN, "x_tokens and code buffers must be 16-byte aligned");
+  if (scale_layout == MXFP8_SCALE_MMA && ((row && !aligned16(row_scales)) || (col && !aligned16(col_scales))))
+    return fail(MXMOE_ERR_ALIGN, "MMA-layout scale buffers must be 16-byte aligned");
   if (T > 0x7FFFFFFF / top_k || m_cap >= (int64_t(1) << 31))
     return fail(MXMOE_ERR_SHAPE, "T*top_k and m_cap must be below 2^31");
   GatherArgs g{row_slot, slot_weights, T * top_k, top_k};

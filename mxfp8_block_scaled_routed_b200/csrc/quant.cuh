@@ -10,11 +10,11 @@
 // endpoint encodings before shifting".
 //
 // HBM-bound work: persistent CTAs, a TMA producer warp keeps 128 x 128 tiles
-// streaming into shared memory while eight consumer warps quantize the
-// previous ones (ROW pass: 4 lanes per 32-block, shuffle amax; COL pass: one
-// thread per column pair of a 32-row block, stores of 32 contiguous codes).
-// With the MMA scale layout the tile's 512 scale bytes of each direction land
-// in one contiguous atom.
+// streaming into shared memory while consumer warps quantize the previous
+// ones.  Each consumer warp owns a 32-row x 64-column sub-tile of a tile, so
+// the warps never wait for each other: ROW blocks one per lane (no shuffles),
+// COL blocks one column pair per lane, codes staged per warp and stored as
+// whole 32-byte sectors, scale bytes written straight into their atoms.
 #pragma once
 #include <cuda.h>
 #include "mx_common.cuh"
@@ -48,25 +48,38 @@ struct CastArgs {
 
 constexpr int kCastPlain = 0;    // TMA tiles of a [batch, rows, cols] tensor
 constexpr int kCastSwiglu = 1;   // TMA gate + up tiles, h = silu(gate) * up
-constexpr int kCastGather = 2;   // rows gathered by bulk copies through a slot table
+constexpr int kCastGather = 2;   // rows gathered by four-row TMA gathers through a slot table
 
 constexpr int kTile = 128;
-constexpr int kCastConsumers = 256;                 // 8 warps
-constexpr int kCastThreads = kCastConsumers + 32;   // + 1 TMA producer warp
 constexpr int kTileBytes = kTile * kTile * 2;       // one bf16 128 x 128 tile
+constexpr int kHalfBytes = kTileBytes / 2;          // one 64-column half of it
+constexpr int kStagingBytes = 2048;                 // per consumer warp: 32 x 64 codes
 
+// A tile is consumed by 8 warps, each owning a 32-row x 64-column sub-tile
+// (warp w: rows 32*(w&3).., columns 64*(w>>2)..) from the moment the tile
+// lands until it is released: the warps never wait for one another.
 template <int kMode>
 struct CastCfg {
   static constexpr bool kSwiglu = kMode == kCastSwiglu;
-  static constexpr int kStages = kSwiglu ? 1 : 2;       // SwiGLU: two CTAs per SM take turns instead
-  static constexpr int kStageBytes = kSwiglu ? 2 * kTileBytes : kTileBytes;
-  static constexpr int kOffColStage = kStages * kStageBytes;         // COL codes of one tile, 128 x 128 B
-  static constexpr int kOffScales = kOffColStage + kTile * kTile;    // ROW then COL scale bytes, 512 B each
-  static constexpr int kOffWeights = kOffScales + 1024;              // gather: per-row weights of each stage
-  static constexpr int kOffPadMask = kOffWeights + (kMode == kCastGather ? kStages * kTile * 4 : 0);
-  static constexpr int kOffBars = kOffPadMask + (kMode == kCastGather ? kStages * 16 : 0);
-  static constexpr int kSmem = kOffBars + 2 * kStages * 8 + 128;     // + alignment slack
-  static constexpr int kCtasPerSm = 2;
+  static constexpr bool kGather = kMode == kCastGather;
+  // plain / SwiGLU: each input tile arrives as two 64-column boxes in the
+  // 128-byte TMA swizzle (16-byte chunk j of row r at chunk j ^ (r & 7)), so a
+  // lane reading one row and a warp reading one column are both free of bank
+  // conflicts.  Gather: 128 unswizzled rows of 256 bytes (four-row gathers).
+  static constexpr bool kSwz = !kGather;
+  static constexpr int kInputs = kSwiglu ? 2 : 1;
+  static constexpr int kStageBytes = kInputs * kTileBytes;
+  static constexpr int kGroups = kSwiglu ? 2 : 1;    // consumer groups of 8 warps; group g takes every kGroups-th tile
+  static constexpr int kStages = kSwiglu ? 3 : 2;
+  static constexpr int kConsumerWarps = 8 * kGroups;
+  static constexpr int kThreads = 32 * (kConsumerWarps + 1);   // + 1 producer warp
+  static constexpr int kOffStaging = kStages * kStageBytes;
+  static constexpr int kOffWeights = kOffStaging + kConsumerWarps * kStagingBytes;
+  static constexpr int kOffPadMask = kOffWeights + (kGather ? kStages * kTile * 4 : 0);
+  static constexpr int kOffBars = kOffPadMask + (kGather ? kStages * 16 : 0);
+  static constexpr int kSmem = kOffBars + 2 * kStages * 8 + 1024;   // + 1024-byte alignment slack
+  static constexpr int kCtasPerSm = kSwiglu ? 1 : 2;
+  static_assert(kSmem * kCtasPerSm <= 232448, "shared memory budget");
 };
 
 // bf16(w * x) for the two bf16 of a word (fp32 product, one rounding to bf16)
@@ -102,6 +115,42 @@ __device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
 __device__ __forceinline__ uint32_t bf16_inv_scale(uint32_t byte) { return (254u - byte) << 7; }
 
 template <int kElem>
+__device__ __forceinline__ uint32_t cvt_pair(uint32_t t) {
+  return fp8x2<kElem>(bf16lo_to_f32(t), bf16hi_to_f32(t));
+}
+
+// One ROW block of 32 elements held by one lane as 16 packed bf16 words:
+// returns the scale byte; c[j] holds the codes of elements 4j..4j+3.
+template <int kElem>
+__device__ __forceinline__ uint32_t quant_block32(const uint32_t (&w)[16], uint32_t (&c)[8]) {
+  uint32_t a[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) a[j] = bf16x2_absmax(w[2 * j], w[2 * j + 1]);
+#pragma unroll
+  for (int st = 4; st >= 1; st >>= 1)
+#pragma unroll
+    for (int j = 0; j < st; ++j) a[j] = bf16x2_absmax(a[j], a[j + st]);
+  const uint32_t m2 = a[0] & 0x7FFF7FFFu;
+  const uint32_t byte = scale_byte_from_bits(max(m2 & 0xFFFFu, m2 >> 16), elem_emax<kElem>());
+  if (byte == 0xFFu) {                               // NaN/Inf block: codes 0x7F | sign
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint2 n = nan8_bf16(make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]));
+      c[2 * j] = n.x;
+      c[2 * j + 1] = n.y;
+    }
+  } else {
+    const uint32_t s = bf16_inv_scale(byte) * 0x00010001u;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      c[j] = cvt_pair<kElem>(bf16x2_mul(w[2 * j], s)) | (cvt_pair<kElem>(bf16x2_mul(w[2 * j + 1], s)) << 16);
+  }
+  return byte;
+}
+
+// Eight elements of a ROW block whose 32 elements are spread over 4
+// consecutive lanes (lanes 4i..4i+3): block maximum by two shuffles.
+template <int kElem>
 __device__ __forceinline__ uint2 row_quant8_packed(uint4 v, uint32_t* byte_out) {
   uint32_t a = bf16x2_absmax(bf16x2_absmax(v.x, v.y), bf16x2_absmax(v.z, v.w)) & 0x7FFF7FFFu;
   uint32_t m = max(a & 0xFFFFu, a >> 16);
@@ -111,11 +160,9 @@ __device__ __forceinline__ uint2 row_quant8_packed(uint4 v, uint32_t* byte_out) 
   *byte_out = byte;
   if (byte == 0xFFu) return nan8_bf16(v);
   const uint32_t s = bf16_inv_scale(byte) * 0x00010001u;
-  const uint32_t x = bf16x2_mul(v.x, s), y = bf16x2_mul(v.y, s), z = bf16x2_mul(v.z, s), w = bf16x2_mul(v.w, s);
   uint2 o;
-  auto cv = [](uint32_t t) { return fp8x2<kElem>(bf16lo_to_f32(t), bf16hi_to_f32(t)); };
-  o.x = cv(x) | (cv(y) << 16);
-  o.y = cv(z) | (cv(w) << 16);
+  o.x = cvt_pair<kElem>(bf16x2_mul(v.x, s)) | (cvt_pair<kElem>(bf16x2_mul(v.y, s)) << 16);
+  o.y = cvt_pair<kElem>(bf16x2_mul(v.z, s)) | (cvt_pair<kElem>(bf16x2_mul(v.w, s)) << 16);
   return o;
 }
 
@@ -163,34 +210,44 @@ __device__ __forceinline__ uint32_t col_quant_pair32(const uint32_t (&w)[32], ui
   return b0 | (b1 << 8);
 }
 
-// Persistent, TMA-fed cast.  Warp 8 streams 128 x 128 bf16 tiles (3-D tensor
-// map [batch, rows, cols], zero fill past the edges) into a ring of shared
-// memory stages; warps 0..7 quantize each tile straight from shared memory:
-//  ROW: lane = 8 consecutive elements, 4 lanes = one 32-block (amax by two
-//       shuffles), codes stored 8 bytes per lane (two 128-byte rows per warp
-//       store);
-//  COL: thread = two adjacent columns of one 32-row block (32 four-byte
-//       shared loads), 32 codes per column stored as two 16-byte stores.
-// SwiGLU: the gate and up tiles arrive together; the ROW pass computes
-// h = bf16(silu(gate) * up), quantizes it and parks it over the gate tile
-// for the COL pass (one barrier among the 256 consumer threads).
+// Per-warp staging buffer of 128 sixteen-byte chunks: chunk L at position
+// L ^ ((L >> 3) & 3).  Written with chunk L = 4*lane + j (a lane's four
+// chunks) and read with L = 32*k + lane, both patterns hit the 8 distinct
+// 16-byte bank groups within every 8-lane phase.
+__device__ __forceinline__ uint32_t staging_off(int L) { return uint32_t(L ^ ((L >> 3) & 3)) << 4; }
+
+__device__ __forceinline__ uint4 lds128(const uint8_t* p) { return *reinterpret_cast<const uint4*>(p); }
+__device__ __forceinline__ void sts128(uint8_t* p, uint4 v) { *reinterpret_cast<uint4*>(p) = v; }
+
+// Persistent, TMA-fed cast.  The producer warp streams 128 x 128 bf16 tiles
+// into a ring of shared-memory stages; each consumer warp quantizes its own
+// 32 x 64 sub-tile of a tile and releases it, with no barrier among warps:
+//  ROW: one lane per row, one 32-element block at a time (four 16-byte
+//       loads, block maximum without shuffles), codes staged per warp and
+//       stored as whole 32-byte sectors (8 rows x 64 bytes per store);
+//  COL: one lane per column pair of the 32-row block (32 four-byte loads),
+//       codes staged and stored as 16 columns x 32 bytes per store.
+// SwiGLU: the ROW pass forms h = bf16(silu(gate) * up) from the gate and up
+// tiles and parks it over the gate sub-tile for the COL pass.  Gather: rows
+// arrive by four-row TMA gathers, unswizzled; the ROW pass there spreads a
+// block over 4 lanes (the row layout would serialize a lane-per-row read),
+// zeroes pad rows and, with router weights, parks bf16(w * x) for the COL pass.
 template <int kMode, int kElem = 0>
-__global__ void __launch_bounds__(kCastThreads, CastCfg<kMode>::kCtasPerSm)
+__global__ void __launch_bounds__(CastCfg<kMode>::kThreads, CastCfg<kMode>::kCtasPerSm)
 mx_cast_kernel(const __grid_constant__ CUtensorMap tin, const CastArgs p) {
   using C = CastCfg<kMode>;
-  constexpr bool kSwiglu = kMode == kCastSwiglu, kGather = kMode == kCastGather;
+  constexpr bool kSwiglu = C::kSwiglu, kGather = C::kGather;
+  constexpr int S = C::kStages;
   const bool weighted = kGather && p.slot_weight != nullptr;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBars);
-  uint8_t* cstage = smem + C::kOffColStage;     // COL codes: column c at c*128, 16-byte chunk k at k ^ ((c>>1)&7)
-  uint8_t* rsc = smem + C::kOffScales;          // ROW scales of the tile: [128 rows][4 blocks]
-  uint8_t* csc = rsc + 512;                     // COL scales of the tile: [128 cols][4 blocks]
-  float* wsm = reinterpret_cast<float*>(smem + C::kOffWeights);   // gather: [stage][row] weights
-  uint32_t* padm = reinterpret_cast<uint32_t*>(smem + C::kOffPadMask);   // gather: [stage][4] pad-row bits
+  float* wsm = reinterpret_cast<float*>(smem + C::kOffWeights);           // gather: [stage][row] weights
+  uint32_t* padm = reinterpret_cast<uint32_t*>(smem + C::kOffPadMask);    // gather: [stage][4] pad-row bits
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t rows = p.rows, cols = p.cols;
   const int64_t ntiles = p.batch * p.tiles_r * p.tiles_c;
+  const int64_t per_batch = p.tiles_r * p.tiles_c;
   int64_t rows_lim = rows;
   if (p.dev_rows != nullptr) rows_lim = min(rows, int64_t(*p.dev_rows));
   const bool do_row = p.modes & 1, do_col = p.modes & 2;
@@ -207,28 +264,28 @@ mx_cast_kernel(const __grid_constant__ CUtensorMap tin, const CastArgs p) {
   }
 
   if (tid == 0) {
-    for (int s = 0; s < C::kStages; ++s) {
-      sm100::mbar_init(sm100::smem_u32(&bars[s]), 1);                                  // full
-      sm100::mbar_init(sm100::smem_u32(&bars[C::kStages + s]), kCastConsumers / 32);  // empty
+    for (int s = 0; s < S; ++s) {
+      sm100::mbar_init(sm100::smem_u32(&bars[s]), 1);        // full: the producer's arrival + bytes
+      sm100::mbar_init(sm100::smem_u32(&bars[S + s]), 8);    // empty: the 8 warps of the consuming group
     }
     sm100::fence_mbar_init();
   }
   __syncthreads();
 
-  const int64_t per_batch = p.tiles_r * p.tiles_c;
-  if (kGather && warp == 8) {
+  // Tiles past the valid rows are skipped by every role alike; n counts the
+  // processed tiles: stage n % S (its (n / S)-th use), consumer group n % kGroups.
+  if (kGather && warp == C::kConsumerWarps) {
     // ---------------- gather producer: lane g owns rows 4g..4g+3 of each
     // tile and fetches them with one four-row gather (tensor map over the
     // token matrix, box 128 x 1).  A pad row borrows a real row of its group
     // (the consumers zero it); a group without a real row is not fetched.
     if (lane == 0) sm100::prefetch_tmap(&tin);
-    int stage = 0;
-    uint32_t phase = 0;
     int64_t band = -1;
     int trow[4] = {0, 0, 0, 0};
     float wreg[4] = {0.f, 0.f, 0.f, 0.f};
     uint32_t padword = 0, ngroups = 0;
     bool fetch = false;
+    int n = 0;
     for (int64_t t = t_begin; t < t_end; t += t_step) {
       const int64_t r0 = (t / p.tiles_c) * kTile, c0 = (t % p.tiles_c) * kTile;
       if (r0 >= rows_lim) continue;
@@ -262,219 +319,250 @@ mx_cast_kernel(const __grid_constant__ CUtensorMap tin, const CastArgs p) {
         wd |= __shfl_xor_sync(0xffffffffu, wd, 4);
         padword = wd;
       }
+      const int s = n % S;
+      const uint32_t ph = uint32_t(n / S) & 1u;
+      ++n;
       bool ok = true;
-      if (lane == 0) ok = sm100::mbar_wait(sm100::smem_u32(&bars[C::kStages + stage]), phase ^ 1);
+      if (lane == 0) ok = sm100::mbar_wait(sm100::smem_u32(&bars[S + s]), ph ^ 1);
       if (!__shfl_sync(0xffffffffu, ok, 0)) {
         if (lane == 0) raise_device_error(7);
         break;
       }
       if (weighted) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) wsm[stage * kTile + 4 * lane + i] = wreg[i];
+        for (int i = 0; i < 4; ++i) wsm[s * kTile + 4 * lane + i] = wreg[i];
       }
-      if ((lane & 7) == 0) padm[stage * 4 + (lane >> 3)] = padword;
+      if ((lane & 7) == 0) padm[s * 4 + (lane >> 3)] = padword;
       __syncwarp();
-      const uint32_t fb = sm100::smem_u32(&bars[stage]);
+      const uint32_t fb = sm100::smem_u32(&bars[s]);
       if (lane == 0) sm100::mbar_arrive_expect_tx(fb, ngroups * 4u * kTile * 2u);
       __syncwarp();
       if (fetch)
-        sm100::tma_gather4(sm100::smem_u32(smem + stage * C::kStageBytes + lane * 4 * 256), &tin, fb, int(c0),
+        sm100::tma_gather4(sm100::smem_u32(smem + s * C::kStageBytes + lane * 4 * 256), &tin, fb, int(c0),
                            trow[0], trow[1], trow[2], trow[3]);
-      if (++stage == C::kStages) { stage = 0; phase ^= 1; }
     }
     return;
   }
-  if (warp == 8) {
-    // ---------------- producer
+  if (warp == C::kConsumerWarps) {
+    // ---------------- producer: two 64-column boxes per input tile
     if (lane == 0) {
       sm100::prefetch_tmap(&tin);
-      int stage = 0;
-      uint32_t phase = 0;
-      for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x) {
+      int n = 0;
+      for (int64_t t = t_begin; t < t_end; t += t_step) {
         const int64_t b = t / per_batch, rem = t - b * per_batch;
         const int64_t r0 = (rem / p.tiles_c) * kTile, c0 = (rem % p.tiles_c) * kTile;
         if (r0 >= rows_lim) continue;             // past the valid rows: never read
-        if (!sm100::mbar_wait(sm100::smem_u32(&bars[C::kStages + stage]), phase ^ 1)) {
+        const int s = n % S;
+        const uint32_t ph = uint32_t(n / S) & 1u;
+        ++n;
+        if (!sm100::mbar_wait(sm100::smem_u32(&bars[S + s]), ph ^ 1)) {
           raise_device_error(7);
           break;
         }
-        const uint32_t fb = sm100::smem_u32(&bars[stage]);
-        const uint32_t dst = sm100::smem_u32(smem + stage * C::kStageBytes);
+        const uint32_t fb = sm100::smem_u32(&bars[s]);
+        const uint32_t dst = sm100::smem_u32(smem + s * C::kStageBytes);
         sm100::mbar_arrive_expect_tx(fb, C::kStageBytes);
-        sm100::tma_load_3d(dst, &tin, fb, int(c0), int(r0), int(b));
-        if constexpr (kSwiglu) sm100::tma_load_3d(dst + kTileBytes, &tin, fb, int(p.up_off + c0), int(r0), int(b));
-        if (++stage == C::kStages) { stage = 0; phase ^= 1; }
+#pragma unroll
+        for (int i = 0; i < C::kInputs; ++i)
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh)
+            sm100::tma_load_3d(dst + i * kTileBytes + hh * kHalfBytes, &tin, fb,
+                               int((i ? p.up_off : 0) + c0 + 64 * hh), int(r0), int(b));
       }
     }
     return;
   }
 
   // ---------------- consumers
-  const int ch = tid & 15, rr0 = tid >> 4;      // ROW: chunk i = row i*16 + rr0, columns ch*8..ch*8+7
-  const int cp = tid & 63, rb = tid >> 6;       // COL: columns 2cp, 2cp+1 of 32-row block rb
-  const bool plain = p.mma_layout == 0;
-  int stage = 0;
-  uint32_t phase = 0;
+  const int grp = warp >> 3, wl = warp & 7;
+  const int q = wl & 3, h = wl >> 2;            // rows 32q.., columns 64h.. of each tile
+  uint8_t* sb = smem + C::kOffStaging + warp * kStagingBytes;
+  const bool mma = p.mma_layout != 0;
+  int n = 0;
   for (int64_t t = t_begin; t < t_end; t += t_step) {
     const int64_t b = t / per_batch, rem = t - b * per_batch;
     const int64_t r0 = (rem / p.tiles_c) * kTile, c0 = (rem % p.tiles_c) * kTile;
     if (r0 >= rows_lim) continue;
-    if (!__all_sync(0xffffffffu, sm100::mbar_wait(sm100::smem_u32(&bars[stage]), phase))) {
+    const int s = n % S;
+    const uint32_t ph = uint32_t(n / S) & 1u;
+    const bool mine = (n % C::kGroups) == grp;
+    ++n;
+    if (!mine) continue;
+    if (!__all_sync(0xffffffffu, sm100::mbar_wait(sm100::smem_u32(&bars[s]), ph))) {
       raise_device_error(7);
       break;
     }
-    uint8_t* tile = smem + stage * C::kStageBytes;
+    uint8_t* tile = smem + s * C::kStageBytes;
     const int vrows = int(min(int64_t(kTile), rows_lim - r0));   // valid rows of the tile (multiple of 32 for COL)
-    if constexpr (kGather) {
-      // pad rows (and rows past the limit) hold a borrowed row or nothing: zero them
-      const uint4 pm = *reinterpret_cast<const uint4*>(padm + stage * 4);
-      if ((pm.x | pm.y | pm.z | pm.w) != 0u) {
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const int idx = q * kCastConsumers + tid, row = idx >> 4;   // row = 8q + tid/16: word q/4
-          const uint32_t w = q < 4 ? (q < 2 ? pm.x : pm.y) : (q < 6 ? pm.z : pm.w);
-          if ((w >> (row & 31)) & 1u) reinterpret_cast<uint4*>(tile)[idx] = make_uint4(0u, 0u, 0u, 0u);
-        }
-        sm100::named_bar_sync(1, kCastConsumers);
-      }
-    }
     const int vcols = int(min(int64_t(kTile), cols - c0));       // valid columns (multiple of 32)
+    const int qrows = vrows - 32 * q;                            // valid rows of this warp's quarter (may exceed 32)
+    const int hcols = vcols - 64 * h;                            // valid columns of this warp's half (may exceed 64)
+    const bool active = qrows > 0 && hcols > 0;
+    const int64_t R0 = b * rows + r0 + 32 * q;                   // matrix row of the sub-tile's first row
+    bool released = false;
+    auto release = [&]() {
+      // the stage is no longer read by this warp: hand it back (ordering this
+      // warp's shared-memory writes into it, if any, before the producer's
+      // next asynchronous copy into the same bytes)
+      if constexpr (kSwiglu || kGather) sm100::fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) sm100::mbar_arrive(sm100::smem_u32(&bars[S + s]));
+      released = true;
+    };
 
-    // ---- ROW pass (and SwiGLU): codes straight to global, scales to shared
-    if (do_row || kSwiglu || weighted) {
-      const int64_t col = c0 + ch * 8;
-      const int64_t Rb = b * rows + r0 + rr0;                    // matrix row of chunk 0
-      uint8_t* rcode = p.row_codes + Rb * cols + col;            // advances 16 rows per chunk
-#pragma unroll 2
-      for (int i = 0; i < 8; ++i) {
-        const int rr = i * 16 + rr0;
-        uint8_t* srow = tile + rr * 256 + ch * 16;
-        uint4 v = *reinterpret_cast<const uint4*>(srow);
-        if constexpr (kSwiglu) {
-          const uint4 u = *reinterpret_cast<const uint4*>(srow + kTileBytes);
-          v.x = swiglu_pair(v.x, u.x);
-          v.y = swiglu_pair(v.y, u.y);
-          v.z = swiglu_pair(v.z, u.z);
-          v.w = swiglu_pair(v.w, u.w);
-          *reinterpret_cast<uint4*>(srow) = v;
+    // ---- ROW pass (and the SwiGLU / gather transforms)
+    if (active && (do_row || kSwiglu || kGather)) {
+      if constexpr (C::kSwz) {
+        const int rr = 32 * q + lane;            // tile row of this lane
+        uint8_t* rp = tile + h * kHalfBytes + rr * 128;
+        const int sw = rr & 7;
+        uint32_t bytes = 0;
+#pragma unroll
+        for (int blk = 0; blk < 2; ++blk) {
+          uint32_t w[16];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint4 v = lds128(rp + (((4 * blk + k) ^ sw) << 4));
+            w[4 * k] = v.x; w[4 * k + 1] = v.y; w[4 * k + 2] = v.z; w[4 * k + 3] = v.w;
+          }
+          if constexpr (kSwiglu) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const uint4 u = lds128(rp + kTileBytes + (((4 * blk + k) ^ sw) << 4));
+              w[4 * k] = swiglu_pair(w[4 * k], u.x);
+              w[4 * k + 1] = swiglu_pair(w[4 * k + 1], u.y);
+              w[4 * k + 2] = swiglu_pair(w[4 * k + 2], u.z);
+              w[4 * k + 3] = swiglu_pair(w[4 * k + 3], u.w);
+            }
+            if (do_col) {
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                sts128(rp + (((4 * blk + k) ^ sw) << 4), make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]));
+            }
+          }
+          if (do_row) {
+            uint32_t c[8];
+            bytes |= quant_block32<kElem>(w, c) << (8 * blk);
+            sts128(sb + staging_off(4 * lane + 2 * blk), make_uint4(c[0], c[1], c[2], c[3]));
+            sts128(sb + staging_off(4 * lane + 2 * blk + 1), make_uint4(c[4], c[5], c[6], c[7]));
+          }
         }
-        if (weighted) {
-          const float w = wsm[stage * kTile + rr];
-          v.x = scale_bf16x2(v.x, w);
-          v.y = scale_bf16x2(v.y, w);
-          v.z = scale_bf16x2(v.z, w);
-          v.w = scale_bf16x2(v.w, w);
-          *reinterpret_cast<uint4*>(srow) = v;
-        }
+        if (!do_col) release();
         if (do_row) {
-          uint32_t byte;
-          const uint2 q = row_quant8_packed<kElem>(v, &byte);
-          if (rr < vrows && ch * 8 < vcols) {
-            *reinterpret_cast<uint2*>(rcode + int64_t(i) * 16 * cols) = q;
-            if ((ch & 3) == 0) rsc[rr * 4 + (ch >> 2)] = uint8_t(byte);
+          // scales of this lane's row: blocks 2h, 2h+1 of the tile
+          if (lane < qrows) {
+            if (mma) {
+              const int64_t atom = ((b * rows + r0) >> 7) * (cols >> 7) + (c0 >> 7);
+              uint8_t* d = p.row_scales + atom * 512 + lane * 16 + q * 4 + 2 * h;
+              if (hcols >= 64) *reinterpret_cast<uint16_t*>(d) = uint16_t(bytes);
+              else d[0] = uint8_t(bytes);
+            } else {
+              uint8_t* d = p.row_scales + (R0 + lane) * (cols >> 5) + (c0 >> 5) + 2 * h;
+              d[0] = uint8_t(bytes);
+              if (hcols >= 64) d[1] = uint8_t(bytes >> 8);
+            }
+          }
+          __syncwarp();
+          // staged codes -> 8 rows x 64 bytes per store
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int L = 32 * k + lane, sr = L >> 2, j = L & 3;
+            if (sr < qrows && 16 * j < hcols)
+              *reinterpret_cast<uint4*>(p.row_codes + (R0 + sr) * cols + c0 + 64 * h + 16 * j) = lds128(sb + staging_off(L));
+          }
+          __syncwarp();
+        }
+      } else {
+        // gather: 256-byte rows; lane = 16-byte chunk (lane & 7) of rows
+        // 4i + (lane >> 3) of the quarter, 4 lanes per 32-element block
+        const uint32_t pm = padm[s * 4 + q];
+        const int ch = lane & 7;
+        const bool park = do_col;                 // pad zeros / weighted rows must be seen by the COL pass
+#pragma unroll 2
+        for (int i = 0; i < 8; ++i) {
+          const int lr = 4 * i + (lane >> 3);
+          uint8_t* a = tile + (32 * q + lr) * 256 + 128 * h + 16 * ch;
+          uint4 v = lds128(a);
+          const bool pad = (pm >> lr) & 1u;
+          if (pad) v = make_uint4(0u, 0u, 0u, 0u);
+          if (weighted) {
+            const float wt = wsm[s * kTile + 32 * q + lr];
+            v.x = scale_bf16x2(v.x, wt);
+            v.y = scale_bf16x2(v.y, wt);
+            v.z = scale_bf16x2(v.z, wt);
+            v.w = scale_bf16x2(v.w, wt);
+          }
+          if (park && (pad || weighted)) sts128(a, v);
+          if (do_row) {
+            uint32_t byte;
+            const uint2 q8 = row_quant8_packed<kElem>(v, &byte);
+            if (lr < qrows && 8 * ch < hcols) {
+              *reinterpret_cast<uint2*>(p.row_codes + (R0 + lr) * cols + c0 + 64 * h + 8 * ch) = q8;
+              if ((ch & 3) == 0) {
+                const int kb = 2 * h + (ch >> 2);
+                if (mma) {
+                  const int64_t atom = ((b * rows + r0) >> 7) * (cols >> 7) + (c0 >> 7);
+                  p.row_scales[atom * 512 + lr * 16 + q * 4 + kb] = uint8_t(byte);
+                } else {
+                  p.row_scales[(R0 + lr) * (cols >> 5) + (c0 >> 5) + kb] = uint8_t(byte);
+                }
+              }
+            }
           }
         }
+        if (!do_col) release();
+        __syncwarp();
       }
     }
-    if ((kSwiglu || weighted) && do_col) sm100::named_bar_sync(1, kCastConsumers);   // h parked for the COL pass
 
-    // ---- COL pass: codes into the shared staging tile
-    if (do_col) {
-      if (rb * 32 < vrows && 2 * cp < vcols) {
-        uint32_t w[32];
-        const uint8_t* src = tile + (rb * 32) * 256 + cp * 4;
-#pragma unroll
-        for (int j = 0; j < 32; ++j) w[j] = *reinterpret_cast<const uint32_t*>(src + j * 256);
-        uint4 qq[2][2];
-        const uint32_t bytes = col_quant_pair32<kElem>(w, qq[0], qq[1]);
-#pragma unroll
-        for (int k = 0; k < 2; ++k) {
-          const int c = 2 * cp + k;
-          uint8_t* dst = cstage + c * 128;
-          const int swz = cp & 7;
-          *reinterpret_cast<uint4*>(dst + (((2 * rb) ^ swz) << 4)) = qq[k][0];
-          *reinterpret_cast<uint4*>(dst + (((2 * rb + 1) ^ swz) << 4)) = qq[k][1];
-          csc[c * 4 + rb] = uint8_t(bytes >> (8 * k));
-        }
-      }
-    }
-    // the input tile is no longer read: hand it back to the producer (after
-    // ordering this thread's shared-memory writes into it, if any, before the
-    // producer's next asynchronous copy into the same bytes)
-    if constexpr (kSwiglu || kGather) sm100::fence_proxy_async();
-    __syncwarp();
-    if (lane == 0) sm100::mbar_arrive(sm100::smem_u32(&bars[C::kStages + stage]));
-    if (++stage == C::kStages) { stage = 0; phase ^= 1; }
-    sm100::named_bar_sync(1, kCastConsumers);                          // COL codes and scales staged
+    __syncwarp();                                  // parked rows visible to the whole warp
 
-    // ---- write-out: whole 128-byte rows of COL codes, 16-byte scale stores
-    if (do_col) {
+    // ---- COL pass: one lane per column pair (2*lane, 2*lane+1 of the half)
+    if (active && do_col) {
+      uint32_t w[32];
+      if constexpr (C::kSwz) {
+        const uint8_t* cb = tile + h * kHalfBytes + 32 * q * 128 + ((lane & 3) << 2);
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int qd = u * kCastConsumers + tid;                // 16-byte chunk id of the 16 KB tile
-        const int c = qd >> 3, k = qd & 7;                      // output row (input column) c, chunk k
-        if (c < vcols && k * 16 < vrows) {
-          const uint4 v = *reinterpret_cast<const uint4*>(cstage + c * 128 + ((k ^ ((c >> 1) & 7)) << 4));
-          *reinterpret_cast<uint4*>(p.col_codes + (b * cols + c0 + c) * rows + r0 + k * 16) = v;
-        }
+        for (int i = 0; i < 32; ++i)
+          w[i] = *reinterpret_cast<const uint32_t*>(cb + i * 128 + (((lane >> 2) ^ (i & 7)) << 4));
+      } else {
+        const uint8_t* cb = tile + 32 * q * 256 + 128 * h + 4 * lane;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) w[i] = *reinterpret_cast<const uint32_t*>(cb + i * 256);
       }
-    }
-    if (do_row) {
-      if (!plain) {
-        // the tile's 128 rows x 4 blocks are exactly one 512-byte MMA atom:
-        // atom byte (r%32)*16 + (r/32)*4 + kb  <-  staged byte r*4 + kb
-        const int64_t atom = ((b * rows + r0) >> 7) * (cols >> 7) + (c0 >> 7);
-        if (vrows == kTile) {
-          if (tid < 32) {
-            uint32_t wv[4];
+      release();
+      uint4 qq[2][2];
+      const uint32_t bytes = col_quant_pair32<kElem>(w, qq[0], qq[1]);
 #pragma unroll
-            for (int g = 0; g < 4; ++g) wv[g] = *reinterpret_cast<const uint32_t*>(rsc + (g * 32 + tid) * 4);
-            *reinterpret_cast<uint4*>(p.row_scales + atom * 512 + tid * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+      for (int k = 0; k < 2; ++k)
+#pragma unroll
+        for (int m = 0; m < 2; ++m) sts128(sb + staging_off(4 * lane + 2 * k + m), qq[k][m]);
+      // scales of this lane's two columns, block q of the tile
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int ct = 64 * h + 2 * lane + k;    // tile column
+        if (2 * lane + k < hcols) {
+          const uint8_t v = uint8_t(bytes >> (8 * k));
+          if (mma) {
+            const int64_t atom = ((b * cols + c0) >> 7) * (rows >> 7) + (r0 >> 7);
+            p.col_scales[atom * 512 + (ct & 31) * 16 + (ct >> 5) * 4 + q] = v;
+          } else {
+            p.col_scales[(b * cols + c0 + ct) * (rows >> 5) + (r0 >> 5) + q] = v;
           }
-        } else if (tid < vrows) {
-          // a tile cut by the device row limit: only its valid rows' 4 bytes
-          *reinterpret_cast<uint32_t*>(p.row_scales + atom * 512 + (tid & 31) * 16 + (tid >> 5) * 4) =
-              *reinterpret_cast<const uint32_t*>(rsc + tid * 4);
         }
-      } else if (tid < vrows) {
-        const int nb = vcols >> 5;
-        const int64_t R = b * rows + r0 + tid;
-        uint8_t* d = p.row_scales + R * (cols >> 5) + (c0 >> 5);
-        if (nb == 4 && (reinterpret_cast<uintptr_t>(d) & 3) == 0)
-          *reinterpret_cast<uint32_t*>(d) = *reinterpret_cast<const uint32_t*>(rsc + tid * 4);
-        else
-          for (int kb = 0; kb < nb; ++kb) d[kb] = rsc[tid * 4 + kb];
       }
-    }
-    if (do_col) {
-      if (!plain) {
-        const int64_t atom = ((b * cols + c0) >> 7) * (rows >> 7) + (r0 >> 7);
-        if (vrows == kTile) {
-          if (tid >= 64 && tid < 96) {
-            const int l = tid - 64;
-            uint32_t wv[4];
+      __syncwarp();
+      // staged codes -> 16 columns x 32 bytes per store
+      const int64_t cbase = b * cols + c0 + 64 * h;
 #pragma unroll
-            for (int g = 0; g < 4; ++g) wv[g] = *reinterpret_cast<const uint32_t*>(csc + (g * 32 + l) * 4);
-            *reinterpret_cast<uint4*>(p.col_scales + atom * 512 + l * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-          }
-        } else if (tid >= 128) {
-          // a tile cut by the device row limit: only the valid 32-row blocks
-          const int c = tid - 128;
-          for (int k = 0; k < (vrows >> 5); ++k) p.col_scales[atom * 512 + (c & 31) * 16 + (c >> 5) * 4 + k] = csc[c * 4 + k];
-        }
-      } else if (tid >= 128 && tid - 128 < vcols) {
-        const int c = tid - 128;
-        const int nb = vrows >> 5;
-        const int64_t R = b * cols + c0 + c;
-        uint8_t* d = p.col_scales + R * (rows >> 5) + (r0 >> 5);
-        if (nb == 4 && (reinterpret_cast<uintptr_t>(d) & 3) == 0)
-          *reinterpret_cast<uint32_t*>(d) = *reinterpret_cast<const uint32_t*>(csc + c * 4);
-        else
-          for (int k = 0; k < nb; ++k) d[k] = csc[c * 4 + k];
+      for (int k = 0; k < 4; ++k) {
+        const int L = 32 * k + lane, c = L >> 1, m = L & 1;
+        if (c < hcols)
+          *reinterpret_cast<uint4*>(p.col_codes + (cbase + c) * rows + r0 + 32 * q + 16 * m) = lds128(sb + staging_off(L));
       }
+      __syncwarp();
     }
-    // staging buffers are rewritten by the next tile
-    sm100::named_bar_sync(1, kCastConsumers);
+    if (!released) release();
   }
 }
 
@@ -589,30 +677,52 @@ __device__ __forceinline__ void dequant_word(uint32_t w, float m1, float m2, uin
   }
 }
 
+template <int kElem>
+__device__ __forceinline__ void dequant16(const uint4 q, uint32_t byte, uint4& o0, uint4& o1) {
+  if (byte == 0xFFu) {
+    o0 = o1 = make_uint4(0x7FFF7FFFu, 0x7FFF7FFFu, 0x7FFF7FFFu, 0x7FFF7FFFu);
+  } else {
+    constexpr uint32_t off = Fp8Bits<kElem>::kOff;
+    const bool one = byte <= 254u - off;            // 2^(byte - bias) is an fp32 normal
+    const float m1 = __uint_as_float(one ? (byte + off) << 23 : (byte + off - 127u) << 23);
+    const float m2 = one ? 1.0f : __uint_as_float(254u << 23);
+    dequant_word<kElem>(q.x, m1, m2, o0.x, o0.y);
+    dequant_word<kElem>(q.y, m1, m2, o0.z, o0.w);
+    dequant_word<kElem>(q.z, m1, m2, o1.x, o1.y);
+    dequant_word<kElem>(q.w, m1, m2, o1.z, o1.w);
+  }
+}
+
+// Grid-stride over 16-code chunks, four chunks per thread and iteration with
+// their loads issued first, so each thread keeps 64 bytes of codes in flight.
 template <typename Idx, int kElem>
 __global__ void __launch_bounds__(256)
 mx_dequant16_kernel(const uint4* __restrict__ codes, const uint8_t* __restrict__ scales, Idx n16, Idx chunks_per_row,
                     Idx ncb, uint4* __restrict__ out) {
+  constexpr int kU = 4;
   const Idx stride = Idx(gridDim.x) * blockDim.x;
-  for (Idx i = Idx(blockIdx.x) * blockDim.x + threadIdx.x; i < n16; i += stride) {
-    const Idx r = i / chunks_per_row, c = i - r * chunks_per_row;
-    const uint32_t byte = __ldg(scales + r * ncb + (c >> 1));
-    const uint4 q = __ldcs(codes + i);
-    uint4 o0, o1;
-    if (byte == 0xFFu) {
-      o0 = o1 = make_uint4(0x7FFF7FFFu, 0x7FFF7FFFu, 0x7FFF7FFFu, 0x7FFF7FFFu);
-    } else {
-      constexpr uint32_t off = Fp8Bits<kElem>::kOff;
-      const bool one = byte <= 254u - off;            // 2^(byte - bias) is an fp32 normal
-      const float m1 = __uint_as_float(one ? (byte + off) << 23 : (byte + off - 127u) << 23);
-      const float m2 = one ? 1.0f : __uint_as_float(254u << 23);
-      dequant_word<kElem>(q.x, m1, m2, o0.x, o0.y);
-      dequant_word<kElem>(q.y, m1, m2, o0.z, o0.w);
-      dequant_word<kElem>(q.z, m1, m2, o1.x, o1.y);
-      dequant_word<kElem>(q.w, m1, m2, o1.z, o1.w);
+  for (Idx base = Idx(blockIdx.x) * blockDim.x + threadIdx.x; base < n16; base += kU * stride) {
+    uint4 q[kU];
+    uint32_t byte[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const Idx i = base + u * stride;
+      if (i < n16) {
+        const Idx r = i / chunks_per_row, c = i - r * chunks_per_row;
+        byte[u] = __ldg(scales + r * ncb + (c >> 1));
+        q[u] = __ldcs(codes + i);
+      }
     }
-    __stcs(out + 2 * i, o0);
-    __stcs(out + 2 * i + 1, o1);
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const Idx i = base + u * stride;
+      if (i < n16) {
+        uint4 o0, o1;
+        dequant16<kElem>(q[u], byte[u], o0, o1);
+        __stcs(out + 2 * i, o0);
+        __stcs(out + 2 * i + 1, o1);
+      }
+    }
   }
 }
 

@@ -26,11 +26,11 @@ def test_every_header_function_is_exported(L):
 
 def test_version_and_error_string(L):
     assert b"sm_100a" in L.mxmoe_version()
-    assert isinstance(L.mxmoe_last_error(), bytes)
+    assert isinstance(L.mxmoe_last_error_message(), bytes)
 
 
 def _err(L):
-    return L.mxmoe_last_error().decode()
+    return L.mxmoe_last_error_message().decode()
 
 
 def test_gemm_rejects_bad_pad_and_shapes(L):
