@@ -13,9 +13,9 @@ forward is timed against the unfused ("swiglu" plan) forward.
 Prints one JSON line.  `value` is the useful (real routed rows) fwd+bwd
 TFLOP/s of the expert MLP with inputs resident in HBM; every input is larger
 than L2, so no flush is needed between steps.  `e2e` is the same metric
-through the public composite API with the step's token inputs copied from
-pinned host memory and a slice of the result read back inside the timed
-region.  `--impl reference` times the CPU oracle on a bounded sample.
+through the public token-major layer API with the step's token inputs copied
+from pinned host memory and its results (layer output, dx, router-weight
+gradient) copied back to pinned host memory inside the timed region.  `--impl reference` times the CPU oracle on a bounded sample.
 
 Launch: python bench.py [--gpus N --steps K --warmup W]; for N > 1 under
 torch.distributed.run (one rank per GPU; each rank runs its own batch, no
@@ -41,6 +41,7 @@ sys.path.insert(0, ROOT)
 SWIGLU_ROWS, SWIGLU_F = 16384, 4096
 CAST_ROWS, CAST_COLS = 8192, 7168
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FP8_SPEC_TFLOPS = 4500.0          # nominal dense MXFP8 tensor peak of one B200 (context beside the measured ones)
 
 
 def load_peaks():
@@ -263,7 +264,7 @@ class Step:
         for i, (name, _, _, fn) in enumerate(self.ops):
             s = fn()
             if s != 0:
-                raise RuntimeError(f"{name}: {self.L.mxmoe_last_error().decode()}")
+                raise RuntimeError(f"{name}: {self.L.mxmoe_last_error_message().decode()}")
             if events is not None:
                 events[i + 1].record(self.stream)
 
@@ -398,7 +399,7 @@ def main():
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="dsv3", choices=["dsv3", "dsv3_16b", "tiny"])
+    ap.add_argument("--workload", default="dsv3", choices=["dsv3", "dsv3_16b", "dsv3_slice", "tiny"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -462,12 +463,14 @@ def main():
 
     peaks, peak_src = load_peaks()
     fp8_sus = 2.0 * peaks["bf16_tflops_sustained"]     # MXFP8 dense = 2 x bf16 (nominal 4.5 / 2.25 PF)
+    fp8_burst = 2.0 * peaks["bf16_tflops"]
     hbm = peaks["hbm_gbs"]
     kernels = {}
     for (name, bound, work, _), ms in zip(step.ops, mean_ms):
         if bound == "tensor":
             ach = work / (ms * 1e-3) / 1e12
-            kernels[name] = {"ms": round(float(ms), 4), "TFLOP/s": round(ach, 1), "frac": round(ach / fp8_sus, 3)}
+            kernels[name] = {"ms": round(float(ms), 4), "TFLOP/s": round(ach, 1), "frac": round(ach / fp8_sus, 3),
+                             "frac_burst": round(ach / fp8_burst, 3), "frac_spec": round(ach / FP8_SPEC_TFLOPS, 3)}
         else:
             ach = work / (ms * 1e-3) / 1e9
             kernels[name] = {"ms": round(float(ms), 4), "GB/s": round(ach, 1), "frac": round(ach / hbm, 3)}
@@ -517,7 +520,7 @@ def main():
         res = {}
         for name, bound, work, fn in ops:
             if fn() != 0:
-                raise RuntimeError(f"{name}: {step.L.mxmoe_last_error().decode()}")
+                raise RuntimeError(f"{name}: {step.L.mxmoe_last_error_message().decode()}")
             ms = time_it(fn, n=10)
             ach = work / (ms * 1e-3) / 1e9
             res[name] = {"ms": round(ms, 4), "GB/s": round(ach, 1), "frac": round(ach / hbm, 3)}
@@ -534,7 +537,8 @@ def main():
     if dbound == "tensor":
         ach = dwork / (dms * 1e-3) / 1e12
         roof = {"bound": "tensor", "kernel": dname, "achieved": round(ach, 1), "peak": round(fp8_sus, 1),
-                "unit": "TFLOP/s", "frac": round(ach / fp8_sus, 3),
+                "unit": "TFLOP/s", "frac": round(ach / fp8_sus, 3), "frac_burst": round(ach / fp8_burst, 3),
+                "frac_spec": round(ach / FP8_SPEC_TFLOPS, 3),
                 "peak_source": f"{peak_src} bf16 sustained x 2 (MXFP8 nominal ratio)",
                 "traffic": ncu_traffic(dname, args.workload)}
     else:
@@ -545,29 +549,37 @@ def main():
 
     # end to end through the public token-major layer API, host buffers: the
     # step's inputs (token rows, routing, router weights, upstream gradient)
-    # are copied from pinned host memory every step; weights stay resident
+    # are copied from pinned host memory every step and the results copied
+    # back; weights stay resident
     e2e = None
     if not args.no_e2e:
         T, k = spec.tokens, spec.top_k
         host = [inp.x_tok.cpu().pin_memory(), torch.from_numpy(inp.routing.topk).pin_memory(),
                 inp.router_w.cpu().pin_memory(), inp.dout_tok.cpu().pin_memory()]
-        # two device slots for the step inputs: the copy of step i+1's inputs
-        # (copy stream) overlaps step i's compute; every step's copy is inside
-        # the timed region
+        # two device slots for the step inputs and for its outputs: the copy of
+        # step i+1's inputs (H2D stream) and the read-back of step i's outputs
+        # (D2H stream) overlap the neighbouring steps' compute; every step's
+        # copies are inside the timed region
         slots = [[torch.empty_like(h, device=dev) for h in host] for _ in range(2)]
-        out_h = torch.empty(2, spec.D, dtype=torch.bfloat16).pin_memory()
         lsaved = mxk.make_layer_saved(T, k, spec.D, spec.E, spec.F, spec.pad, dev)
         ws_f = torch.empty(mxk.layer_workspace_bytes(T, k, spec.D, spec.E, spec.F, spec.pad, 1), dtype=torch.uint8,
                            device=dev)
         ws_b = torch.empty(mxk.layer_workspace_bytes(T, k, spec.D, spec.E, spec.F, spec.pad, 2), dtype=torch.uint8,
                            device=dev)
-        out_d = torch.empty(T, spec.D, dtype=torch.bfloat16, device=dev)
-        dx_d = torch.empty(T, spec.D, dtype=torch.bfloat16, device=dev)
-        dwr_d = torch.empty(T, k, dtype=torch.float32, device=dev)
+        outs = [[torch.empty(T, spec.D, dtype=torch.bfloat16, device=dev),
+                 torch.empty(T, spec.D, dtype=torch.bfloat16, device=dev),
+                 torch.empty(T, k, dtype=torch.float32, device=dev)] for _ in range(2)]
+        # the step's results in pinned host memory: layer output, dx, router-weight gradient
+        res_h = [torch.empty(T, spec.D, dtype=torch.bfloat16).pin_memory(),
+                 torch.empty(T, spec.D, dtype=torch.bfloat16).pin_memory(),
+                 torch.empty(T, k, dtype=torch.float32).pin_memory()]
         comp = torch.cuda.current_stream(dev)
         copy_s = torch.cuda.Stream(dev)
+        d2h_s = torch.cuda.Stream(dev)
         copied = [torch.cuda.Event() for _ in range(2)]
         used = [torch.cuda.Event() for _ in range(2)]
+        computed = [torch.cuda.Event() for _ in range(2)]
+        read = [torch.cuda.Event() for _ in range(2)]
 
         def h2d(i):
             sl = i % 2
@@ -581,14 +593,24 @@ def main():
         def compute(i):
             sl = i % 2
             comp.wait_event(copied[sl])
+            if i >= 2:
+                comp.wait_event(read[sl])              # step i-2's results have left this slot
             x_d, tk_d, w_d, do_d = slots[sl]
+            out_d, dx_d, dwr_d = outs[sl]
             mxk.mxmoe_quantize_weights(step.w13, step.w2, qw=step.qw)
             mxk.moe_layer_fwd_q(x_d, tk_d, w_d, step.qw, spec.pad, out=out_d, saved=lsaved, workspace=ws_f)
             mxk.moe_layer_bwd_q(do_d, w_d, step.qw, lsaved, spec.pad, dx=dx_d, dw13=step.dw13, dw2=step.dw2,
                                 dweights=dwr_d, workspace=ws_b)
             used[sl].record(comp)
-            out_h[0].copy_(out_d[0], non_blocking=True)
-            out_h[1].copy_(dx_d[0], non_blocking=True)
+            computed[sl].record(comp)
+
+        def d2h(i):
+            sl = i % 2
+            with torch.cuda.stream(d2h_s):
+                d2h_s.wait_event(computed[sl])
+                for h, d in zip(res_h, outs[sl]):
+                    h.copy_(d, non_blocking=True)
+                read[sl].record(d2h_s)
 
         def run(nsteps):
             h2d(0)
@@ -596,6 +618,7 @@ def main():
                 if i + 1 < nsteps:
                     h2d(i + 1)
                 compute(i)
+                d2h(i)
 
         run(2)
         torch.cuda.synchronize()
@@ -603,21 +626,25 @@ def main():
             torch.distributed.barrier()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(comp)
-        copy_s.wait_stream(comp)                        # the first copy starts inside the timed region
+        copy_s.wait_stream(comp)                        # the first copies start inside the timed region
+        d2h_s.wait_stream(comp)
         run(args.steps)
         comp.wait_stream(copy_s)
+        comp.wait_stream(d2h_s)                         # the last read-back ends inside the timed region
         b.record(comp)
         torch.cuda.synchronize()
         ms = max_over_ranks(a.elapsed_time(b) / args.steps, dev)
         h2d_bytes = sum(h.numel() * h.element_size() for h in host)
+        d2h_bytes = sum(h.numel() * h.element_size() for h in res_h)
         e2e = {"value": round(whole_job_tflops(useful, world, ms), 2), "unit": "TFLOP/s",
-               "h2d_bytes_per_step": int(h2d_bytes), "d2h_bytes_per_step": int(out_h.numel() * 2),
+               "h2d_bytes_per_step": int(h2d_bytes), "d2h_bytes_per_step": int(d2h_bytes),
                "ms_per_step": round(ms, 3),
                "how": "public C-ABI token-major layer (mxmoe_quantize_weights, moe_layer_fwd_q: route + gather/cast + "
                       "MLP + weighted combine, moe_layer_bwd_q: weighted gather/cast + MLP backward + unpermute + "
                       "router-weight gradient); token rows, top-k ids, router weights and the upstream gradient "
-                      "copied from pinned host memory every step on a copy stream overlapping the previous step's "
-                      "compute; one row of the output and of dx read back"}
+                      "copied from pinned host memory every step, and the layer output, dx and the router-weight "
+                      "gradient copied back to pinned host memory every step, on two copy streams overlapping the "
+                      "neighbouring steps' compute; expert-weight gradients stay on the device"}
         if mxk.device_error() != 0:
             raise RuntimeError("device error during the e2e run")
 
@@ -639,6 +666,10 @@ def main():
         "mlp_no_weight_cast_tflops": round(useful / ((mlp_ms - cast_w_ms) * 1e-3) / 1e12, 2),
         "fwd_useful_tflops_prequantized_weights": round(6.0 * step.R * spec.D * spec.F / (fwd_ms * 1e-3) / 1e12, 2),
         "swiglu_quant_gbs": sw["GB/s"], "swiglu_quant_frac_hbm": sw["frac"],
+        "kernel_peaks": {"hbm_gbs": hbm, "mxfp8_tflops_sustained": round(fp8_sus, 1),
+                         "mxfp8_tflops_burst": round(fp8_burst, 1), "mxfp8_tflops_spec": FP8_SPEC_TFLOPS,
+                         "source": f"{peak_src}: HBM copy; MXFP8 = 2 x the cuBLAS bf16 figure (frac: sustained, "
+                                   "frac_burst: burst), frac_spec: the nominal 4.5 PFLOP/s"},
         "kernels": kernels, "fused_vs_unfused": fused_vs_unfused, "outside_step": outside_step, "roofline": roof, "clocks": clk,
         "gpu_launches": n_ops * args.steps,
         "e2e": e2e, "cpu_baseline": cpu, "source_hash": src_hash(),

@@ -65,6 +65,10 @@ SPECS = {
     "dsv3_16b": Spec("dsv3_16b", 64, 2048, 1408, 8192, 6, 256, 1.1, 2, 0.02),
     "dsv3": Spec("dsv3", 256, 7168, 2048, 16384, 8, 256, 1.0, 0, 0.006,
                  x_outlier_frac=1e-3, x_outlier_mul=50.0),
+    # 16 experts of the DSv3-scale layer (same D, F, routing law, padding and
+    # per-expert load): a few GB on the device, for profiling its kernels
+    "dsv3_slice": Spec("dsv3_slice", 16, 7168, 2048, 1024, 8, 256, 1.0, 0, 0.006,
+                       x_outlier_frac=1e-3, x_outlier_mul=50.0),
 }
 
 
