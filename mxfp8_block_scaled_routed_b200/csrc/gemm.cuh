@@ -538,13 +538,31 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
           for (int j = 0; j < 16; ++j)
             va[16 * c + j] = pack_bf16x2(__uint_as_float(r[c][2 * j]), __uint_as_float(r[c][2 * j + 1]));
       } else {
+        // the same for the SwiGLU / dSwiGLU epilogues: every TMEM load in
+        // flight, one wait, TMEM handed back, then the bf16 rounding
+        constexpr int kLoads = (kEpi == kEpiSwiGLU) ? 2 * kChunks : kChunks;
+        uint32_t r[kLoads][32];
 #pragma unroll
-        for (int c = 0; c < kChunks; ++c) drain32_bf16(t_row + h * kHalf + 32 * c, va + 16 * c);
+        for (int c = 0; c < kChunks; ++c) tmem_ld_32x32b_x32(t_row + h * kHalf + 32 * c, r[c]);
         if constexpr (kEpi == kEpiSwiGLU) {
 #pragma unroll
-          for (int c = 0; c < kChunks; ++c) drain32_bf16(t_row + 128 + h * kHalf + 32 * c, vb + 16 * c);
+          for (int c = 0; c < kChunks; ++c) tmem_ld_32x32b_x32(t_row + 128 + h * kHalf + 32 * c, r[kChunks + c]);
         }
+        tmem_wait_ld();
         release();
+#pragma unroll
+        for (int c = 0; c < kChunks; ++c)
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            va[16 * c + j] = pack_bf16x2(__uint_as_float(r[c][2 * j]), __uint_as_float(r[c][2 * j + 1]));
+        if constexpr (kEpi == kEpiSwiGLU) {
+#pragma unroll
+          for (int c = 0; c < kChunks; ++c)
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              vb[16 * c + j] = pack_bf16x2(__uint_as_float(r[kChunks + c][2 * j]),
+                                           __uint_as_float(r[kChunks + c][2 * j + 1]));
+        }
       }
 
       if constexpr (kEpi == kEpiBF16) {

@@ -133,14 +133,14 @@ struct GatherArgs {
   int top_k;
 };
 
-// 3-D bf16 cast input [batch, rows, ld], box 64 x 128 x 1 (128-byte rows) in the
-// 128-byte swizzle, zero fill past the edges.
-int make_cast_map(CUtensorMap* map, const void* base, int64_t batch, int64_t rows, int64_t ld) {
+// 3-D bf16 cast input [batch, rows, ld], box 64 x box_rows x 1 (128-byte rows)
+// in the 128-byte swizzle, zero fill past the edges.
+int make_cast_map(CUtensorMap* map, const void* base, int64_t batch, int64_t rows, int64_t ld, uint32_t box_rows) {
   EncodeTiledFn enc;
   MX_TRY(get_encode(&enc));
   cuuint64_t dims[3] = {cuuint64_t(ld), cuuint64_t(rows), cuuint64_t(batch)};
   cuuint64_t strides[2] = {cuuint64_t(ld * 2), cuuint64_t(rows * ld * 2)};
-  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t box[3] = {64, box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -173,7 +173,8 @@ int launch_cast(const void* in, int64_t batch, int64_t rows, int64_t cols, int m
   constexpr bool kSwiglu = kMode == kCastSwiglu;
   DevInfo* d;
   MX_TRY(device_info(&d));
-  const int bit = kElem == 1 ? 15 : kMode == kCastPlain ? 7 : kMode == kCastSwiglu ? 8 : 13;  // not the GEMM bits
+  // attribute bits 17.. (the GEMMs use 0-16): one per (mode, element)
+  const int bit = 17 + kMode * 2 + kElem;
   auto kern = mx_cast_kernel<kMode, kElem>;
   if (!(d->attr_set & (1u << bit))) {
     MX_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem),
@@ -186,7 +187,7 @@ int launch_cast(const void* in, int64_t batch, int64_t rows, int64_t cols, int m
     if (!g) return fail(MXMOE_ERR_ARG, "gather cast without a slot table");
     MX_TRY(make_gather_map(&map, in, g->n_slots / g->top_k, cols));
   } else
-    MX_TRY(make_cast_map(&map, in, batch, rows, kSwiglu ? 2 * cols : cols));
+    MX_TRY(make_cast_map(&map, in, batch, rows, kSwiglu ? 2 * cols : cols, C::kTileRows));
   CastArgs a;
   memset(&a, 0, sizeof(a));
   if (g) {
@@ -201,7 +202,7 @@ int launch_cast(const void* in, int64_t batch, int64_t rows, int64_t cols, int m
   a.batch = batch;
   a.up_off = kSwiglu ? cols : 0;
   a.tiles_c = (cols + 127) / 128;
-  a.tiles_r = (rows + 127) / 128;
+  a.tiles_r = (rows + C::kTileRows - 1) / C::kTileRows;
   a.modes = modes;
   a.mma_layout = layout;
   a.row_codes = rc;
@@ -210,6 +211,7 @@ int launch_cast(const void* in, int64_t batch, int64_t rows, int64_t cols, int m
   a.col_scales = cs;
   a.dev_rows = dev_rows;
   const int64_t ntiles = batch * a.tiles_r * a.tiles_c;
+  if (ntiles >= (int64_t(1) << 31)) return fail(MXMOE_ERR_SHAPE, "cast of %lld tiles: too large", (long long)ntiles);
   const int64_t per_sm = C::kCtasPerSm;
   const int grid = int(ntiles < per_sm * d->sms ? ntiles : per_sm * d->sms);
   kern<<<grid, C::kThreads, C::kSmem, stream>>>(map, a);

@@ -50,14 +50,19 @@ constexpr int kCastPlain = 0;    // TMA tiles of a [batch, rows, cols] tensor
 constexpr int kCastSwiglu = 1;   // TMA gate + up tiles, h = silu(gate) * up
 constexpr int kCastGather = 2;   // rows gathered by four-row TMA gathers through a slot table
 
-constexpr int kTile = 128;
+constexpr int kTile = 128;                          // tile columns (and rows, except SwiGLU)
 constexpr int kTileBytes = kTile * kTile * 2;       // one bf16 128 x 128 tile
-constexpr int kHalfBytes = kTileBytes / 2;          // one 64-column half of it
 constexpr int kStagingBytes = 2048;                 // per consumer warp: 32 x 64 codes
 
-// A tile is consumed by 8 warps, each owning a 32-row x 64-column sub-tile
-// (warp w: rows 32*(w&3).., columns 64*(w>>2)..) from the moment the tile
-// lands until it is released: the warps never wait for one another.
+
+// A tile is consumed by kWarpsPerTile warps, each owning a 32-row x
+// 64-column sub-tile (rows 32*q.., columns 64*h..) from the moment the tile
+// lands until it releases the stage: the warps never wait for one another.
+// The 8 consumer warps of a CTA form groups that take tiles in turn (one
+// group of 8 for 128-row tiles, two of 4 for the SwiGLU's 64-row tiles); two
+// CTAs per SM with 2 stages each.  (One CTA per SM with 16 consumer warps and
+// a 6-stage ring measured the same or slightly slower, interleaved in one
+// process: 0.754 against 0.763 of HBM for the W13 dual cast.)
 template <int kMode>
 struct CastCfg {
   static constexpr bool kSwiglu = kMode == kCastSwiglu;
@@ -67,19 +72,25 @@ struct CastCfg {
   // lane reading one row and a warp reading one column are both free of bank
   // conflicts.  Gather: 128 unswizzled rows of 256 bytes (four-row gathers).
   static constexpr bool kSwz = !kGather;
+  static constexpr int kTileRows = kSwiglu ? 64 : 128;          // SwiGLU: gate + up of 64 rows per stage
+  static constexpr int kQuarters = kTileRows / 32;
+  static constexpr int kWarpsPerTile = 2 * kQuarters;
   static constexpr int kInputs = kSwiglu ? 2 : 1;
-  static constexpr int kStageBytes = kInputs * kTileBytes;
-  static constexpr int kGroups = kSwiglu ? 2 : 1;    // consumer groups of 8 warps; group g takes every kGroups-th tile
-  static constexpr int kStages = kSwiglu ? 3 : 2;
-  static constexpr int kConsumerWarps = 8 * kGroups;
+  static constexpr int kInputBytes = kTileRows * kTile * 2;     // one input tile
+  static constexpr int kHalfBytes = kInputBytes / 2;            // one 64-column box of it
+  static constexpr int kStageBytes = kInputs * kInputBytes;     // 32 KB
+  static constexpr int kCtasPerSm = 2;
+  static constexpr int kConsumerWarps = 8;
+  static constexpr int kGroups = kConsumerWarps / kWarpsPerTile;
+  static constexpr int kStages = 2;
   static constexpr int kThreads = 32 * (kConsumerWarps + 1);   // + 1 producer warp
   static constexpr int kOffStaging = kStages * kStageBytes;
   static constexpr int kOffWeights = kOffStaging + kConsumerWarps * kStagingBytes;
   static constexpr int kOffPadMask = kOffWeights + (kGather ? kStages * kTile * 4 : 0);
   static constexpr int kOffBars = kOffPadMask + (kGather ? kStages * 16 : 0);
   static constexpr int kSmem = kOffBars + 2 * kStages * 8 + 1024;   // + 1024-byte alignment slack
-  static constexpr int kCtasPerSm = kSwiglu ? 1 : 2;
-  static_assert(kSmem * kCtasPerSm <= 232448, "shared memory budget");
+  static_assert((kSmem + 1024) * kCtasPerSm <= 233472, "shared memory budget");
+  static_assert(!kGather || kTileRows == 128, "the gather producer fetches 128-row tiles");
 };
 
 // bf16(w * x) for the two bf16 of a word (fp32 product, one rounding to bf16)
@@ -210,14 +221,55 @@ __device__ __forceinline__ uint32_t col_quant_pair32(const uint32_t (&w)[32], ui
   return b0 | (b1 << 8);
 }
 
+// Position (batch b, row tile tr, column tile tc) of tile t = t0 + i * step,
+// advanced by additions: a 64-bit division per tile and thread would cost
+// as much as quantizing a block.
+struct TileWalk {
+  int tc, tr, b;
+  int dc, dr, db;
+  int tiles_c, tiles_r;
+  __device__ __forceinline__ TileWalk(int64_t t0, int64_t step, int64_t tiles_c_, int64_t tiles_r_)
+      : tiles_c(int(tiles_c_)), tiles_r(int(tiles_r_)) {
+    const int64_t per = tiles_c_ * tiles_r_;
+    b = int(t0 / per);
+    const int64_t rem = t0 - int64_t(b) * per;
+    tr = int(rem / tiles_c_);
+    tc = int(rem - int64_t(tr) * tiles_c_);
+    db = int(step / per);
+    const int64_t srem = step - int64_t(db) * per;
+    dr = int(srem / tiles_c_);
+    dc = int(srem - int64_t(dr) * tiles_c_);
+  }
+  __device__ __forceinline__ void next() {
+    tc += dc;
+    tr += dr;
+    b += db;
+    if (tc >= tiles_c) { tc -= tiles_c; ++tr; }
+    if (tr >= tiles_r) { tr -= tiles_r; ++b; }
+  }
+};
+
 // Per-warp staging buffer of 128 sixteen-byte chunks: chunk L at position
 // L ^ ((L >> 3) & 3).  Written with chunk L = 4*lane + j (a lane's four
 // chunks) and read with L = 32*k + lane, both patterns hit the 8 distinct
 // 16-byte bank groups within every 8-lane phase.
 __device__ __forceinline__ uint32_t staging_off(int L) { return uint32_t(L ^ ((L >> 3) & 3)) << 4; }
 
-__device__ __forceinline__ uint4 lds128(const uint8_t* p) { return *reinterpret_cast<const uint4*>(p); }
-__device__ __forceinline__ void sts128(uint8_t* p, uint4 v) { *reinterpret_cast<uint4*>(p) = v; }
+// Shared-memory accesses on 32-bit shared-window addresses (ld/st.shared,
+// never the generic path).  volatile keeps them after the mbarrier waits.
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint32_t lds32(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ void sts128(uint32_t a, uint4 v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
+}
 
 // Persistent, TMA-fed cast.  The producer warp streams 128 x 128 bf16 tiles
 // into a ring of shared-memory stages; each consumer warp quantizes its own
@@ -232,7 +284,7 @@ __device__ __forceinline__ void sts128(uint8_t* p, uint4 v) { *reinterpret_cast<
 // arrive by four-row TMA gathers, unswizzled; the ROW pass there spreads a
 // block over 4 lanes (the row layout would serialize a lane-per-row read),
 // zeroes pad rows and, with router weights, parks bf16(w * x) for the COL pass.
-template <int kMode, int kElem = 0>
+template <int kMode, int kElem>
 __global__ void __launch_bounds__(CastCfg<kMode>::kThreads, CastCfg<kMode>::kCtasPerSm)
 mx_cast_kernel(const __grid_constant__ CUtensorMap tin, const CastArgs p) {
   using C = CastCfg<kMode>;
@@ -247,7 +299,6 @@ mx_cast_kernel(const __grid_constant__ CUtensorMap tin, const CastArgs p) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t rows = p.rows, cols = p.cols;
   const int64_t ntiles = p.batch * p.tiles_r * p.tiles_c;
-  const int64_t per_batch = p.tiles_r * p.tiles_c;
   int64_t rows_lim = rows;
   if (p.dev_rows != nullptr) rows_lim = min(rows, int64_t(*p.dev_rows));
   const bool do_row = p.modes & 1, do_col = p.modes & 2;
@@ -266,7 +317,7 @@ mx_cast_kernel(const __grid_constant__ CUtensorMap tin, const CastArgs p) {
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
       sm100::mbar_init(sm100::smem_u32(&bars[s]), 1);        // full: the producer's arrival + bytes
-      sm100::mbar_init(sm100::smem_u32(&bars[S + s]), 8);    // empty: the 8 warps of the consuming group
+      sm100::mbar_init(sm100::smem_u32(&bars[S + s]), C::kWarpsPerTile);   // empty: the consuming group's warps
     }
     sm100::fence_mbar_init();
   }
@@ -286,8 +337,9 @@ mx_cast_kernel(const __grid_constant__ CUtensorMap tin, const CastArgs p) {
     uint32_t padword = 0, ngroups = 0;
     bool fetch = false;
     int n = 0;
-    for (int64_t t = t_begin; t < t_end; t += t_step) {
-      const int64_t r0 = (t / p.tiles_c) * kTile, c0 = (t % p.tiles_c) * kTile;
+    TileWalk w(t_begin, t_step, p.tiles_c, p.tiles_r);
+    for (int64_t t = t_begin; t < t_end; t += t_step, w.next()) {
+      const int64_t r0 = int64_t(w.tr) * kTile, c0 = int64_t(w.tc) * kTile;
       if (r0 >= rows_lim) continue;
       if (r0 != band) {                           // new row band: its slots, once
         band = r0;
@@ -348,9 +400,10 @@ mx_cast_kernel(const __grid_constant__ CUtensorMap tin, const CastArgs p) {
     if (lane == 0) {
       sm100::prefetch_tmap(&tin);
       int n = 0;
-      for (int64_t t = t_begin; t < t_end; t += t_step) {
-        const int64_t b = t / per_batch, rem = t - b * per_batch;
-        const int64_t r0 = (rem / p.tiles_c) * kTile, c0 = (rem % p.tiles_c) * kTile;
+      TileWalk w(t_begin, t_step, p.tiles_c, p.tiles_r);
+      for (int64_t t = t_begin; t < t_end; t += t_step, w.next()) {
+        const int64_t b = w.b;
+        const int64_t r0 = int64_t(w.tr) * C::kTileRows, c0 = int64_t(w.tc) * kTile;
         if (r0 >= rows_lim) continue;             // past the valid rows: never read
         const int s = n % S;
         const uint32_t ph = uint32_t(n / S) & 1u;
@@ -366,7 +419,7 @@ mx_cast_kernel(const __grid_constant__ CUtensorMap tin, const CastArgs p) {
         for (int i = 0; i < C::kInputs; ++i)
 #pragma unroll
           for (int hh = 0; hh < 2; ++hh)
-            sm100::tma_load_3d(dst + i * kTileBytes + hh * kHalfBytes, &tin, fb,
+            sm100::tma_load_3d(dst + i * C::kInputBytes + hh * C::kHalfBytes, &tin, fb,
                                int((i ? p.up_off : 0) + c0 + 64 * hh), int(r0), int(b));
       }
     }
@@ -374,31 +427,38 @@ mx_cast_kernel(const __grid_constant__ CUtensorMap tin, const CastArgs p) {
   }
 
   // ---------------- consumers
-  const int grp = warp >> 3, wl = warp & 7;
-  const int q = wl & 3, h = wl >> 2;            // rows 32q.., columns 64h.. of each tile
-  uint8_t* sb = smem + C::kOffStaging + warp * kStagingBytes;
+  const int grp = warp / C::kWarpsPerTile, wl = warp % C::kWarpsPerTile;
+  const int q = wl % C::kQuarters, h = wl / C::kQuarters;   // rows 32q.., columns 64h.. of each tile
+  const uint32_t sbase = sm100::smem_u32(smem);
+  const uint32_t sb = sbase + C::kOffStaging + warp * kStagingBytes;
   const bool mma = p.mma_layout != 0;
   int n = 0;
-  for (int64_t t = t_begin; t < t_end; t += t_step) {
-    const int64_t b = t / per_batch, rem = t - b * per_batch;
-    const int64_t r0 = (rem / p.tiles_c) * kTile, c0 = (rem % p.tiles_c) * kTile;
+  TileWalk w(t_begin, t_step, p.tiles_c, p.tiles_r);
+  for (int64_t t = t_begin; t < t_end; t += t_step, w.next()) {
+    const int64_t b = w.b;
+    const int64_t r0 = int64_t(w.tr) * C::kTileRows, c0 = int64_t(w.tc) * kTile;
     if (r0 >= rows_lim) continue;
     const int s = n % S;
     const uint32_t ph = uint32_t(n / S) & 1u;
     const bool mine = (n % C::kGroups) == grp;
     ++n;
     if (!mine) continue;
-    if (!__all_sync(0xffffffffu, sm100::mbar_wait(sm100::smem_u32(&bars[s]), ph))) {
-      raise_device_error(7);
+    // lane 0 waits for the tile; __syncwarp orders the other lanes' reads after its acquire
+    bool ok = true;
+    if (lane == 0) ok = sm100::mbar_wait(sm100::smem_u32(&bars[s]), ph);
+    __syncwarp();
+    if (!__shfl_sync(0xffffffffu, ok, 0)) {
+      if (lane == 0) raise_device_error(7);
       break;
     }
-    uint8_t* tile = smem + s * C::kStageBytes;
-    const int vrows = int(min(int64_t(kTile), rows_lim - r0));   // valid rows of the tile (multiple of 32 for COL)
+    const uint32_t tile = sbase + s * C::kStageBytes;
+    const int vrows = int(min(int64_t(C::kTileRows), rows_lim - r0));   // valid rows of the tile (multiple of 32 for COL)
     const int vcols = int(min(int64_t(kTile), cols - c0));       // valid columns (multiple of 32)
     const int qrows = vrows - 32 * q;                            // valid rows of this warp's quarter (may exceed 32)
     const int hcols = vcols - 64 * h;                            // valid columns of this warp's half (may exceed 64)
     const bool active = qrows > 0 && hcols > 0;
     const int64_t R0 = b * rows + r0 + 32 * q;                   // matrix row of the sub-tile's first row
+    const int qa = int((r0 & 127) >> 5) + q;                     // 32-row block of the sub-tile inside its 128-row MMA atom
     bool released = false;
     auto release = [&]() {
       // the stage is no longer read by this warp: hand it back (ordering this
@@ -414,7 +474,7 @@ mx_cast_kernel(const __grid_constant__ CUtensorMap tin, const CastArgs p) {
     if (active && (do_row || kSwiglu || kGather)) {
       if constexpr (C::kSwz) {
         const int rr = 32 * q + lane;            // tile row of this lane
-        uint8_t* rp = tile + h * kHalfBytes + rr * 128;
+        const uint32_t rp = tile + h * C::kHalfBytes + rr * 128;
         const int sw = rr & 7;
         uint32_t bytes = 0;
 #pragma unroll
@@ -428,7 +488,7 @@ mx_cast_kernel(const __grid_constant__ CUtensorMap tin, const CastArgs p) {
           if constexpr (kSwiglu) {
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-              const uint4 u = lds128(rp + kTileBytes + (((4 * blk + k) ^ sw) << 4));
+              const uint4 u = lds128(rp + C::kInputBytes + (((4 * blk + k) ^ sw) << 4));
               w[4 * k] = swiglu_pair(w[4 * k], u.x);
               w[4 * k + 1] = swiglu_pair(w[4 * k + 1], u.y);
               w[4 * k + 2] = swiglu_pair(w[4 * k + 2], u.z);
@@ -453,7 +513,7 @@ mx_cast_kernel(const __grid_constant__ CUtensorMap tin, const CastArgs p) {
           if (lane < qrows) {
             if (mma) {
               const int64_t atom = ((b * rows + r0) >> 7) * (cols >> 7) + (c0 >> 7);
-              uint8_t* d = p.row_scales + atom * 512 + lane * 16 + q * 4 + 2 * h;
+              uint8_t* d = p.row_scales + atom * 512 + lane * 16 + qa * 4 + 2 * h;
               if (hcols >= 64) *reinterpret_cast<uint16_t*>(d) = uint16_t(bytes);
               else d[0] = uint8_t(bytes);
             } else {
@@ -481,7 +541,7 @@ mx_cast_kernel(const __grid_constant__ CUtensorMap tin, const CastArgs p) {
 #pragma unroll 2
         for (int i = 0; i < 8; ++i) {
           const int lr = 4 * i + (lane >> 3);
-          uint8_t* a = tile + (32 * q + lr) * 256 + 128 * h + 16 * ch;
+          const uint32_t a = tile + (32 * q + lr) * 256 + 128 * h + 16 * ch;
           uint4 v = lds128(a);
           const bool pad = (pm >> lr) & 1u;
           if (pad) v = make_uint4(0u, 0u, 0u, 0u);
@@ -521,14 +581,13 @@ mx_cast_kernel(const __grid_constant__ CUtensorMap tin, const CastArgs p) {
     if (active && do_col) {
       uint32_t w[32];
       if constexpr (C::kSwz) {
-        const uint8_t* cb = tile + h * kHalfBytes + 32 * q * 128 + ((lane & 3) << 2);
+        const uint32_t cb = tile + h * C::kHalfBytes + 32 * q * 128 + ((lane & 3) << 2);
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
-          w[i] = *reinterpret_cast<const uint32_t*>(cb + i * 128 + (((lane >> 2) ^ (i & 7)) << 4));
+        for (int i = 0; i < 32; ++i) w[i] = lds32(cb + i * 128 + (((lane >> 2) ^ (i & 7)) << 4));
       } else {
-        const uint8_t* cb = tile + 32 * q * 256 + 128 * h + 4 * lane;
+        const uint32_t cb = tile + 32 * q * 256 + 128 * h + 4 * lane;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) w[i] = *reinterpret_cast<const uint32_t*>(cb + i * 256);
+        for (int i = 0; i < 32; ++i) w[i] = lds32(cb + i * 256);
       }
       release();
       uint4 qq[2][2];
@@ -545,7 +604,7 @@ mx_cast_kernel(const __grid_constant__ CUtensorMap tin, const CastArgs p) {
           const uint8_t v = uint8_t(bytes >> (8 * k));
           if (mma) {
             const int64_t atom = ((b * cols + c0) >> 7) * (rows >> 7) + (r0 >> 7);
-            p.col_scales[atom * 512 + (ct & 31) * 16 + (ct >> 5) * 4 + q] = v;
+            p.col_scales[atom * 512 + (ct & 31) * 16 + (ct >> 5) * 4 + qa] = v;
           } else {
             p.col_scales[(b * cols + c0 + ct) * (rows >> 5) + (r0 >> 5) + q] = v;
           }
