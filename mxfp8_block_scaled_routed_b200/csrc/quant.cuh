@@ -159,24 +159,6 @@ __device__ __forceinline__ uint32_t quant_block32(const uint32_t (&w)[16], uint3
   return byte;
 }
 
-// Eight elements of a ROW block whose 32 elements are spread over 4
-// consecutive lanes (lanes 4i..4i+3): block maximum by two shuffles.
-template <int kElem>
-__device__ __forceinline__ uint2 row_quant8_packed(uint4 v, uint32_t* byte_out) {
-  uint32_t a = bf16x2_absmax(bf16x2_absmax(v.x, v.y), bf16x2_absmax(v.z, v.w)) & 0x7FFF7FFFu;
-  uint32_t m = max(a & 0xFFFFu, a >> 16);
-  m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
-  m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
-  const uint32_t byte = scale_byte_from_bits(m, elem_emax<kElem>());
-  *byte_out = byte;
-  if (byte == 0xFFu) return nan8_bf16(v);
-  const uint32_t s = bf16_inv_scale(byte) * 0x00010001u;
-  uint2 o;
-  o.x = cvt_pair<kElem>(bf16x2_mul(v.x, s)) | (cvt_pair<kElem>(bf16x2_mul(v.y, s)) << 16);
-  o.y = cvt_pair<kElem>(bf16x2_mul(v.z, s)) | (cvt_pair<kElem>(bf16x2_mul(v.w, s)) << 16);
-  return o;
-}
-
 // Both columns of a 32-row block held as the two halves of w[0..31]: codes
 // of the low-half column in q0, of the high-half column in q1; returns the
 // two scale bytes (low | high << 8).
@@ -267,6 +249,9 @@ __device__ __forceinline__ uint32_t lds32(uint32_t a) {
   asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
   return v;
 }
+__device__ __forceinline__ void sts64(uint32_t a, uint32_t x, uint32_t y) {
+  asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(a), "r"(x), "r"(y) : "memory");
+}
 __device__ __forceinline__ void sts128(uint32_t a, uint4 v) {
   asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
 }
@@ -281,8 +266,8 @@ __device__ __forceinline__ void sts128(uint32_t a, uint4 v) {
 //       codes staged and stored as 16 columns x 32 bytes per store.
 // SwiGLU: the ROW pass forms h = bf16(silu(gate) * up) from the gate and up
 // tiles and parks it over the gate sub-tile for the COL pass.  Gather: rows
-// arrive by four-row TMA gathers, unswizzled; the ROW pass there spreads a
-// block over 4 lanes (the row layout would serialize a lane-per-row read),
+// arrive by four-row TMA gathers, unswizzled; the ROW pass there reads each
+// lane's block in a rotated chunk order (conflict-free without the swizzle),
 // zeroes pad rows and, with router weights, parks bf16(w * x) for the COL pass.
 template <int kMode, int kElem>
 __global__ void __launch_bounds__(CastCfg<kMode>::kThreads, CastCfg<kMode>::kCtasPerSm)
@@ -533,41 +518,65 @@ mx_cast_kernel(const __grid_constant__ CUtensorMap tin, const CastArgs p) {
           __syncwarp();
         }
       } else {
-        // gather: 256-byte rows; lane = 16-byte chunk (lane & 7) of rows
-        // 4i + (lane >> 3) of the quarter, 4 lanes per 32-element block
+        // gather: unswizzled 256-byte rows.  One lane per (row, 32-element
+        // block): in pass it, lane l takes row 16*it + (l >> 1) of the quarter
+        // and block l & 1 of the half, and reads the block's four 16-byte
+        // chunks in the rotated order (j + rot) & 3, rot = (l >> 1) & 3, so the
+        // 8 lanes of a phase hit 8 different bank groups.  The codes of each
+        // chunk go to the staging buffer at that chunk's own position.
         const uint32_t pm = padm[s * 4 + q];
-        const int ch = lane & 7;
+        const int blk = lane & 1, rot = (lane >> 1) & 3;
         const bool park = do_col;                 // pad zeros / weighted rows must be seen by the COL pass
-#pragma unroll 2
-        for (int i = 0; i < 8; ++i) {
-          const int lr = 4 * i + (lane >> 3);
-          const uint32_t a = tile + (32 * q + lr) * 256 + 128 * h + 16 * ch;
-          uint4 v = lds128(a);
+#pragma unroll
+        for (int it = 0; it < 2; ++it) {
+          const int lr = 16 * it + (lane >> 1);
+          const uint32_t rowa = tile + (32 * q + lr) * 256 + 128 * h + 64 * blk;
+          uint32_t w[16];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint4 v = lds128(rowa + (((j + rot) & 3) << 4));
+            w[4 * j] = v.x; w[4 * j + 1] = v.y; w[4 * j + 2] = v.z; w[4 * j + 3] = v.w;
+          }
           const bool pad = (pm >> lr) & 1u;
-          if (pad) v = make_uint4(0u, 0u, 0u, 0u);
+          const uint32_t keep = pad ? 0u : 0xFFFFFFFFu;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) w[i] &= keep;
           if (weighted) {
             const float wt = wsm[s * kTile + 32 * q + lr];
-            v.x = scale_bf16x2(v.x, wt);
-            v.y = scale_bf16x2(v.y, wt);
-            v.z = scale_bf16x2(v.z, wt);
-            v.w = scale_bf16x2(v.w, wt);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) w[i] = scale_bf16x2(w[i], wt);
           }
-          if (park && (pad || weighted)) sts128(a, v);
+          if (park && (pad || weighted)) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              sts128(rowa + (((j + rot) & 3) << 4), make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]));
+          }
           if (do_row) {
-            uint32_t byte;
-            const uint2 q8 = row_quant8_packed<kElem>(v, &byte);
-            if (lr < qrows && 8 * ch < hcols) {
-              *reinterpret_cast<uint2*>(p.row_codes + (R0 + lr) * cols + c0 + 64 * h + 8 * ch) = q8;
-              if ((ch & 3) == 0) {
-                const int kb = 2 * h + (ch >> 2);
-                if (mma) {
-                  const int64_t atom = ((b * rows + r0) >> 7) * (cols >> 7) + (c0 >> 7);
-                  p.row_scales[atom * 512 + lr * 16 + q * 4 + kb] = uint8_t(byte);
-                } else {
-                  p.row_scales[(R0 + lr) * (cols >> 5) + (c0 >> 5) + kb] = uint8_t(byte);
-                }
+            uint32_t c[8];
+            const uint32_t byte = quant_block32<kElem>(w, c);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int jp = (j + rot) & 3;       // the chunk these 8 codes belong to
+              sts64(sb + staging_off(4 * lr + 2 * blk + (jp >> 1)) + ((jp & 1) << 3), c[2 * j], c[2 * j + 1]);
+            }
+            if (lr < qrows && 32 * blk < hcols) {
+              if (mma) {
+                const int64_t atom = ((b * rows + r0) >> 7) * (cols >> 7) + (c0 >> 7);
+                p.row_scales[atom * 512 + lr * 16 + qa * 4 + 2 * h + blk] = uint8_t(byte);
+              } else {
+                p.row_scales[(R0 + lr) * (cols >> 5) + (c0 >> 5) + 2 * h + blk] = uint8_t(byte);
               }
             }
+          }
+        }
+        if (do_row) {
+          __syncwarp();
+          // staged codes -> 8 rows x 64 bytes per store
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int L = 32 * k + lane, sr = L >> 2, j = L & 3;
+            if (sr < qrows && 16 * j < hcols)
+              *reinterpret_cast<uint4*>(p.row_codes + (R0 + sr) * cols + c0 + 64 * h + 16 * j) = lds128(sb + staging_off(L));
           }
         }
         if (!do_col) release();
