@@ -142,6 +142,18 @@ def _need(t: torch.Tensor, dtype, name: str):
         raise ValueError(f"{name} must be contiguous")
 
 
+def _shape(t: torch.Tensor, shape, name: str):
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _scales(t: torch.Tensor, n: int, name: str):
+    """E8M0 scale bytes: a contiguous uint8 CUDA tensor of exactly n bytes."""
+    _need(t, torch.uint8, name)
+    if t.numel() != n:
+        raise ValueError(f"{name} must hold {n} scale bytes, got {t.numel()}")
+
+
 def _u8(shape, dev):
     return torch.empty(shape, dtype=torch.uint8, device=dev)
 
@@ -208,8 +220,10 @@ def mxfp8_swiglu_quant(h13: torch.Tensor, modes: int = ROW | COL, scale_layout: 
 def mxfp8_dequantize(codes: torch.Tensor, scales: torch.Tensor, elem: str = "e4m3") -> torch.Tensor:
     """MXFP8 ROW (plain scales, E4M3 or E5M2 codes) -> bf16."""
     _need(codes, torch.uint8, "codes")
-    _need(scales, torch.uint8, "scales")
+    if codes.dim() != 2:
+        raise ValueError("codes must be 2-D")
     rows, cols = codes.shape
+    _scales(scales, rows * ((cols + 31) // 32), "scales")
     out = torch.empty(rows, cols, dtype=torch.bfloat16, device=codes.device)
     fn = {"e4m3": lib().mxfp8_dequantize, "e5m2": lib().mxfp8_dequantize_e5m2}[elem]
     _check(fn(_ptr(codes), _ptr(scales), rows, cols, _ptr(out), _stream(codes)))
@@ -225,12 +239,18 @@ def _offs(offsets: torch.Tensor):
 def mxfp8_grouped_gemm(a, a_scales, w, w_scales, offsets, pad_multiple=128, out=None):
     """Ragged-M grouped GEMM: a [M, K] codes, w [E, N, K] codes (MMA scales)."""
     E = _offs(offsets)
+    _need(a, torch.uint8, "a")
+    _need(w, torch.uint8, "w")
     M, K = a.shape
-    _, N, _ = w.shape
+    if w.dim() != 3 or w.shape[0] != E or w.shape[2] != K:
+        raise ValueError(f"w must be [E={E}, N, K={K}], got {tuple(w.shape)}")
+    N = w.shape[1]
+    _scales(a_scales, M * K // 32, "a_scales")
+    _scales(w_scales, E * N * K // 32, "w_scales")
     if out is None:
         out = torch.empty(M, N, dtype=torch.bfloat16, device=a.device)
-    for t, n in ((a, "a"), (a_scales, "a_scales"), (w, "w"), (w_scales, "w_scales")):
-        _need(t, torch.uint8, n)
+    _need(out, torch.bfloat16, "out")
+    _shape(out, (M, N), "out")
     _check(lib().mxfp8_grouped_gemm(_ptr(a), _ptr(a_scales), M, K, _ptr(w), _ptr(w_scales), E, N,
                                     _ptr(offsets), pad_multiple, _ptr(out), _stream(a)))
     return out
@@ -239,10 +259,18 @@ def mxfp8_grouped_gemm(a, a_scales, w, w_scales, offsets, pad_multiple=128, out=
 def mxfp8_grouped_gemm_wgrad(gt, gt_scales, xt, xt_scales, offsets, pad_multiple=128, out=None):
     """Ragged-K grouped GEMM: gt [N, M], xt [Kx, M] COL codes -> dw bf16 [E, N, Kx]."""
     E = _offs(offsets)
+    _need(gt, torch.uint8, "gt")
+    _need(xt, torch.uint8, "xt")
     N, M = gt.shape
+    if xt.dim() != 2 or xt.shape[1] != M:
+        raise ValueError(f"xt must be [Kx, M={M}], got {tuple(xt.shape)}")
     Kx = xt.shape[0]
+    _scales(gt_scales, N * M // 32, "gt_scales")
+    _scales(xt_scales, Kx * M // 32, "xt_scales")
     if out is None:
         out = torch.empty(E, N, Kx, dtype=torch.bfloat16, device=gt.device)
+    _need(out, torch.bfloat16, "out")
+    _shape(out, (E, N, Kx), "out")
     _check(lib().mxfp8_grouped_gemm_wgrad(_ptr(gt), _ptr(gt_scales), N, _ptr(xt), _ptr(xt_scales), Kx, M,
                                           _ptr(offsets), E, pad_multiple, _ptr(out), _stream(gt)))
     return out
@@ -251,8 +279,14 @@ def mxfp8_grouped_gemm_wgrad(gt, gt_scales, xt, xt_scales, offsets, pad_multiple
 def mxfp8_grouped_gemm_swiglu_quant(a, a_scales, w13, w13_scales, offsets, pad_multiple=128, want_h13=True):
     """FC1 + SwiGLU + dual quantization; returns dict(h13, h_row_codes, h_row_scales, h_col_codes, h_col_scales)."""
     E = _offs(offsets)
+    _need(a, torch.uint8, "a")
+    _need(w13, torch.uint8, "w13")
     M, K = a.shape
+    if w13.dim() != 3 or w13.shape[0] != E or w13.shape[2] != K or w13.shape[1] % 2:
+        raise ValueError(f"w13 must be [E={E}, 2F, K={K}], got {tuple(w13.shape)}")
     F = w13.shape[1] // 2
+    _scales(a_scales, M * K // 32, "a_scales")
+    _scales(w13_scales, E * 2 * F * K // 32, "w13_scales")
     dev = a.device
     o = dict(h13=torch.empty(M, 2 * F, dtype=torch.bfloat16, device=dev) if want_h13 else None,
              h_row_codes=_u8((M, F), dev), h_row_scales=_u8((M * F // 32,), dev),
@@ -267,10 +301,18 @@ def mxfp8_grouped_gemm_swiglu_quant(a, a_scales, w13, w13_scales, offsets, pad_m
 def mxfp8_grouped_gemm_dswiglu_quant(dy, dy_scales, w2t, w2t_scales, offsets, h13, pad_multiple=128):
     """FC2 dgrad + dSwiGLU + dual quantization; returns dict(g_row_codes, g_row_scales, g_col_codes, g_col_scales)."""
     E = _offs(offsets)
+    _need(dy, torch.uint8, "dy")
+    _need(w2t, torch.uint8, "w2t")
     M, D = dy.shape
     F = w2t.shape[1]
     dev = dy.device
     _need(h13, torch.bfloat16, "h13")
+    _scales(dy_scales, M * D // 32, "dy_scales")
+    _scales(w2t_scales, E * F * D // 32, "w2t_scales")
+    if w2t.dim() != 3 or w2t.shape[0] != E or w2t.shape[2] != D:
+        raise ValueError(f"w2t must be [E={E}, F, D={D}], got {tuple(w2t.shape)}")
+    if tuple(h13.shape) != (M, 2 * F):
+        raise ValueError(f"h13 must be [M={M}, 2F={2 * F}], got {tuple(h13.shape)}")
     o = dict(g_row_codes=_u8((M, 2 * F), dev), g_row_scales=_u8((M * 2 * F // 32,), dev),
              g_col_codes=_u8((2 * F, M), dev), g_col_scales=_u8((M * 2 * F // 32,), dev))
     _check(lib().mxfp8_grouped_gemm_dswiglu_quant(

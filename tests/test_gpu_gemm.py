@@ -117,15 +117,49 @@ def test_bad_offsets_raise_device_error_and_write_nothing():
     assert (bf16_np(out) == 3.0).all()
 
 
+def test_bindings_reject_mismatched_shapes_before_launch():
+    """A tensor whose shape disagrees with the others would make the kernel
+    read or write outside it; the binding refuses it before any launch."""
+    E, N, K, M, F = 2, 256, 256, 256, 128
+    u8 = lambda *s: torch.zeros(s, dtype=torch.uint8, device=DEV)
+    off = _dev(np.array([0, 128, 256], np.int32))
+    out = torch.zeros(M, N, dtype=torch.bfloat16, device=DEV)
+    good = (u8(M, K), u8(M * K // 32), u8(E, N, K), u8(E * N * K // 32))
+    bad_cases = [
+        (u8(M, K), u8(M * K // 32), u8(E, N, K + 128), u8(E * N * (K + 128) // 32)),   # K of w
+        (u8(M, K), u8(M * K // 32 - 1), u8(E, N, K), u8(E * N * K // 32)),             # a_scales size
+        (u8(M, K), u8(M * K // 32), u8(E + 1, N, K), u8((E + 1) * N * K // 32)),       # experts of w
+    ]
+    for a, sa, w, sw in bad_cases:
+        with pytest.raises(ValueError):
+            mxk.mxfp8_grouped_gemm(a, sa, w, sw, off, 128, out=out)
+    with pytest.raises(ValueError):
+        mxk.mxfp8_grouped_gemm(*good, off, 128, out=torch.zeros(M, N + 128, dtype=torch.bfloat16, device=DEV))
+    with pytest.raises(ValueError):   # xt with another M
+        mxk.mxfp8_grouped_gemm_wgrad(u8(N, M), u8(N * M // 32), u8(K, M + 128), u8(K * (M + 128) // 32), off, 128)
+    with pytest.raises(ValueError):   # w13 with an odd row count
+        mxk.mxfp8_grouped_gemm_swiglu_quant(u8(M, K), u8(M * K // 32), u8(E, 2 * F + 1, K),
+                                            u8(E * (2 * F + 1) * K // 32), off, 128)
+    h13 = torch.zeros(M, 2 * F, dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(ValueError):   # w2t laid out as [E, 2F, D]: h13 would be read past its end
+        mxk.mxfp8_grouped_gemm_dswiglu_quant(u8(M, K), u8(M * K // 32), u8(E, 2 * F, K), u8(E * 2 * F * K // 32),
+                                             off, h13, 128)
+    with pytest.raises(ValueError):
+        mxk.mxfp8_dequantize(u8(M, K), u8(M * K // 32 + 1))
+    assert mxk.device_error() == 0
+
+
 # ------------------------------------------------------------------ ragged K
 def _mx_cols_dev(x_bf16: torch.Tensor):
     o = mxk.mxfp8_quantize(x_bf16.to(DEV), mxk.COL, mxk.MMA)
     return o["col_codes"], o["col_scales"]
 
 
-@pytest.mark.parametrize("N,Kx", [(256, 384), (512, 512)])
+@pytest.mark.parametrize("N,Kx", [(256, 384), (512, 512), (128, 128), (256, 256), (2048, 1536)])
 def test_wgrad_exact_closed_form_and_empty_expert(N, Kx):
-    """N = 256 / Kx = 384 takes the 128-wide tile, 512 / 512 the 256-wide one."""
+    """Kx = 384 and 128 take the 128-wide tile, 512 and 256 the 256-wide one;
+    N x Kx = 2048 x 1536 gives 3 x 96 tiles, more than the SMs, so CTAs walk
+    on to the next expert's tiles."""
     g = np.random.default_rng(4)
     E = 3
     off = _offsets([256, 0, 300], 128)
