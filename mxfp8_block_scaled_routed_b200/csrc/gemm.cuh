@@ -29,6 +29,7 @@
 #include <cuda.h>
 #include "mx_common.cuh"
 #include "sm100.cuh"
+#include "quant.cuh"
 
 namespace mxmoe::gemm {
 
@@ -73,7 +74,8 @@ struct Cfg {
   static constexpr int SFA_BYTES = 512;
   static constexpr int SFB_BYTES = (BN / 128) * 512;          // scales of all BN rows of B
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
-  static constexpr int kStages = kPair ? ((BN == 256) ? 6 : 7) : ((BN == 256) ? 4 : 6);
+  // (the dSwiGLU epilogue's larger staging tile costs one stage)
+  static constexpr int kStages = (kPair ? ((BN == 256) ? 6 : 7) : ((BN == 256) ? 4 : 6)) - (kEpi == kEpiDSwiGLU ? 1 : 0);
   static constexpr int SF_COLS = 4 + BN / 32;           // TMEM columns for one SF buffer
   static constexpr int ACC_COLS = kAcc * BN;
   static constexpr int TMEM_COLS = 512;
@@ -86,7 +88,9 @@ struct Cfg {
   static constexpr int OFF_SFB = OFF_SFA + kStages * SFA_BYTES;
   static constexpr int OFF_EPI = OFF_SFB + kStages * SFB_BYTES;
   static constexpr int EPI_WARPS = 8;
-  static constexpr int EPI_WARP_BYTES = 2560;               // 32x32 bf16 transpose / staging buffer (512-aligned)
+  // per epilogue warp: 32x32 bf16 transpose / staging buffer; dSwiGLU: the
+  // 32 x 64 bf16 dgate|dup tile (then its COL codes) and the ROW codes (512-aligned)
+  static constexpr int EPI_WARP_BYTES = (kEpi == kEpiDSwiGLU) ? 6144 : 2560;
   static constexpr int EPI_BYTES = EPI_WARPS * EPI_WARP_BYTES;
   static constexpr int OFF_BAR = OFF_EPI + EPI_BYTES;
   static constexpr int NUM_BARS = 2 * kStages + 2 * kAcc;
@@ -282,6 +286,74 @@ __device__ __forceinline__ void load64(const uint16_t* src, uint32_t (&v)[16]) {
     uint4 t = s[i];
     v[4 * i] = t.x; v[4 * i + 1] = t.y; v[4 * i + 2] = t.z; v[4 * i + 3] = t.w;
   }
+}
+
+// dSwiGLU outputs of one 32-column chunk, dgate (dg) and dup (du) of this
+// lane's row (row0 + lane), dual-quantized to E4M3.  ROW: each lane
+// quantizes its own two 32-element blocks (columns f.. and F + f.. of the
+// [M, 2F] code matrix); the codes leave through 2 KB of staging as whole
+// 32-byte row segments.  COL: the 32 x 64 bf16 tile dgate|dup is staged
+// (16-byte piece j of row r at piece j ^ (r & 7)) and read back one column
+// pair per lane, as the cast kernel's COL pass does (codes of columns f..
+// and F + f.. of the [2F, M] code matrix, rows row0..row0+31), then leaves
+// through the same 4 KB once it has been read.  tb: this warp's 6 KB of
+// shared memory (tile, then ROW staging at +4096).
+__device__ __forceinline__ void dswiglu_dual_quant(const uint32_t (&dg)[16], const uint32_t (&du)[16], int lane,
+                                                   uint32_t tb, int64_t row0, int64_t f, int64_t F, int64_t M,
+                                                   uint8_t* row_codes, uint8_t* row_scales, uint8_t* col_codes,
+                                                   uint8_t* col_scales) {
+  const uint32_t rs = tb + 4096;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    sts128(tb + lane * 128 + ((j ^ (lane & 7)) << 4), make_uint4(dg[4 * j], dg[4 * j + 1], dg[4 * j + 2], dg[4 * j + 3]));
+    sts128(tb + lane * 128 + (((4 + j) ^ (lane & 7)) << 4),
+           make_uint4(du[4 * j], du[4 * j + 1], du[4 * j + 2], du[4 * j + 3]));
+  }
+  // ROW: block g (0: dgate, 1: dup) of row r staged at 1024 g + 32 r, its two
+  // 16-byte pieces swapped on (r >> 2) & 1
+#pragma unroll
+  for (int g = 0; g < 2; ++g) {
+    uint32_t cc[8];
+    const uint32_t byte = quant_block32<0>(g ? du : dg, cc);
+    row_scales[mma_scale_offset(row0 + lane, (g * F + f) >> 5, 2 * F)] = uint8_t(byte);
+#pragma unroll
+    for (int pc = 0; pc < 2; ++pc)
+      sts128(rs + 1024 * g + lane * 32 + ((pc ^ ((lane >> 2) & 1)) << 4),
+             make_uint4(cc[4 * pc], cc[4 * pc + 1], cc[4 * pc + 2], cc[4 * pc + 3]));
+  }
+  __syncwarp();
+#pragma unroll
+  for (int g = 0; g < 2; ++g)
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int r = 16 * i + (lane >> 1), pc = lane & 1;
+      *reinterpret_cast<uint4*>(row_codes + (row0 + r) * 2 * F + g * F + f + 16 * pc) =
+          lds128(rs + 1024 * g + r * 32 + ((pc ^ ((r >> 2) & 1)) << 4));
+    }
+  // COL
+  uint32_t w[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) w[i] = lds32(tb + i * 128 + ((((lane >> 2) ^ (i & 7))) << 4) + ((lane & 3) << 2));
+  __syncwarp();
+  uint4 qq[2][2];
+  const uint32_t cb = col_quant_pair32<0>(w, qq[0], qq[1]);
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+#pragma unroll
+    for (int mm = 0; mm < 2; ++mm) sts128(tb + staging_off(4 * lane + 2 * k + mm), qq[k][mm]);
+    const int L = 2 * lane + k;
+    const int64_t gcol = (L < 32) ? f + L : F + f + (L - 32);
+    col_scales[mma_scale_offset(gcol, row0 >> 5, M)] = uint8_t(cb >> (8 * k));
+  }
+  __syncwarp();
+  // 16 columns x 32 bytes per store
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int L = 32 * k + lane, col = L >> 1, half = L & 1;
+    const int64_t gcol = (col < 32) ? f + col : F + f + (col - 32);
+    *reinterpret_cast<uint4*>(col_codes + gcol * M + row0 + 16 * half) = lds128(tb + staging_off(L));
+  }
+  __syncwarp();   // the staging is rewritten by the next chunk
 }
 
 // 32 TMEM columns of this lane's row -> 16 packed bf16 words (round to nearest even).
@@ -591,33 +663,34 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
       } else {  // kEpiDSwiGLU
         const int64_t F = p.F;
         const int64_t m = row0 + lane;
+        const uint32_t tb = smem_u32(sbuf);
 #pragma unroll
         for (int c = 0; c < kChunks; ++c) {
           const int64_t f = T.out_c0 + h * kHalf + 32 * c;
-          uint32_t ha[16], hb[16];
-          load64(p.h13 + m * 2 * F + f, ha);
-          load64(p.h13 + m * 2 * F + F + f, hb);
-          uint32_t dg[16], du[16];
+          // h13 gate (hw[0..15]) and up (hw[16..31]) words of this row; dgate
+          // and dup are written over them
+          uint32_t hw[32];
+          load64(p.h13 + m * 2 * F + f, *reinterpret_cast<uint32_t(*)[16]>(&hw[0]));
+          load64(p.h13 + m * 2 * F + F + f, *reinterpret_cast<uint32_t(*)[16]>(&hw[16]));
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const uint32_t dw = va[16 * c + j];
             float d[2], a[2], b[2], og[2], ou[2];
             d[0] = bf16lo_to_f32(dw); d[1] = bf16hi_to_f32(dw);
-            a[0] = bf16lo_to_f32(ha[j]); a[1] = bf16hi_to_f32(ha[j]);
-            b[0] = bf16lo_to_f32(hb[j]); b[1] = bf16hi_to_f32(hb[j]);
+            a[0] = bf16lo_to_f32(hw[j]); a[1] = bf16hi_to_f32(hw[j]);
+            b[0] = bf16lo_to_f32(hw[16 + j]); b[1] = bf16hi_to_f32(hw[16 + j]);
 #pragma unroll
             for (int i = 0; i < 2; ++i) {
               const float s = sigmoid_fast(a[i]);
               og[i] = d[i] * b[i] * s * (1.0f + a[i] * (1.0f - s));
               ou[i] = d[i] * a[i] * s;
             }
-            dg[j] = pack_bf16x2(og[0], og[1]);
-            du[j] = pack_bf16x2(ou[0], ou[1]);
+            hw[j] = pack_bf16x2(og[0], og[1]);        // dgate
+            hw[16 + j] = pack_bf16x2(ou[0], ou[1]);   // dup
           }
-          dual_quant_block(dg, lane, sbuf, row0, f, 2 * F, p.M, p.row_codes, p.row_scales, p.col_codes,
-                           p.col_scales);
-          dual_quant_block(du, lane, sbuf, row0, F + f, 2 * F, p.M, p.row_codes, p.row_scales, p.col_codes,
-                           p.col_scales);
+          dswiglu_dual_quant(*reinterpret_cast<const uint32_t(*)[16]>(&hw[0]),
+                             *reinterpret_cast<const uint32_t(*)[16]>(&hw[16]), lane, tb, row0, f, F, p.M, p.row_codes, p.row_scales, p.col_codes,
+                             p.col_scales);
         }
       }
     }
