@@ -249,6 +249,14 @@ __device__ __forceinline__ uint32_t lds32(uint32_t a) {
   asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
   return v;
 }
+// 32 words of one column pair, rows 0..31 of a 128-byte-swizzled sub-tile:
+// row i's word sits at bases[i & 7] + 128 i, the row offset folded into the
+// load's immediate.
+template <int I = 0>
+__device__ __forceinline__ void lds32_rows(uint32_t (&w)[32], const uint32_t (&bases)[8]) {
+  asm volatile("ld.shared.u32 %0, [%1+%2];" : "=r"(w[I]) : "r"(bases[I & 7]), "n"(I * 128));
+  if constexpr (I + 1 < 32) lds32_rows<I + 1>(w, bases);
+}
 __device__ __forceinline__ void sts64(uint32_t a, uint32_t x, uint32_t y) {
   asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(a), "r"(x), "r"(y) : "memory");
 }
@@ -461,13 +469,14 @@ mx_cast_kernel(const __grid_constant__ CUtensorMap tin, const CastArgs p) {
         const int rr = 32 * q + lane;            // tile row of this lane
         const uint32_t rp = tile + h * C::kHalfBytes + rr * 128;
         const int sw = rr & 7;
+        const uint32_t rpx = rp | uint32_t(sw << 4);   // rp is 128-byte aligned
         uint32_t bytes = 0;
 #pragma unroll
         for (int blk = 0; blk < 2; ++blk) {
           uint32_t w[16];
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            const uint4 v = lds128(rp + (((4 * blk + k) ^ sw) << 4));
+            const uint4 v = lds128(rpx ^ uint32_t((4 * blk + k) << 4));
             w[4 * k] = v.x; w[4 * k + 1] = v.y; w[4 * k + 2] = v.z; w[4 * k + 3] = v.w;
           }
           if constexpr (kSwiglu) {
@@ -591,8 +600,10 @@ mx_cast_kernel(const __grid_constant__ CUtensorMap tin, const CastArgs p) {
       uint32_t w[32];
       if constexpr (C::kSwz) {
         const uint32_t cb = tile + h * C::kHalfBytes + 32 * q * 128 + ((lane & 3) << 2);
+        uint32_t bases[8];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) w[i] = lds32(cb + i * 128 + (((lane >> 2) ^ (i & 7)) << 4));
+        for (int k = 0; k < 8; ++k) bases[k] = cb + (((lane >> 2) ^ k) << 4);
+        lds32_rows(w, bases);
       } else {
         const uint32_t cb = tile + 32 * q * 256 + 128 * h + 4 * lane;
 #pragma unroll
