@@ -30,7 +30,7 @@ using namespace mxmoe;
 #define MXMOE_USE_PAIRS 1
 #endif
 #ifndef MXMOE_WGRAD_PAIRS
-#define MXMOE_WGRAD_PAIRS 0
+#define MXMOE_WGRAD_PAIRS 1
 #endif
 
 namespace {
@@ -431,8 +431,9 @@ int gemm_ragged_k(const uint8_t* gt, const uint8_t* gs, int64_t N, const uint8_t
   p.a_scales = gs;
   p.b_scales = xs;
   p.out = static_cast<uint16_t*>(dw);
-  // (CTA pairs measured slower here: experts' short K leave little mainloop
-  // to hide the pair's per-tile accumulator hand-off)
+  // CTA pairs (256 x 256 tiles, 128 x 256 per CTA) when N and Kx allow: they
+  // halve each SM's B-operand loads; the accumulator hand-off, paid once
+  // per tile over each expert's short K, uses a CTA-scope arrive
   if (MXMOE_WGRAD_PAIRS == 1 && Kx % 256 == 0 && N % 256 == 0)
     return launch_gemm<gemm::kRaggedK, gemm::kEpiBF16, 256, true>(gt, N, xt, Kx, p,
                                                                   int64_t(E) * (N / 256) * (Kx / 256), stream, 10);
