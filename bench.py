@@ -155,6 +155,10 @@ class Step:
         bf = lambda *sh: torch.empty(*sh, dtype=torch.bfloat16, device=dev)
         self.x, self.w13, self.w2, self.dy = inp.x, inp.w13, inp.w2, inp.dy
         self.off = torch.from_numpy(inp.routing.offsets).to(dev)
+        # token rows of each expert: the weight gradients skip the all-pad K blocks
+        counts = np.asarray(inp.routing.counts, dtype=np.int64)
+        self.rows = torch.from_numpy(counts.astype(np.int32)).to(dev)
+        self.Mw = int(((counts + 127) // 128 * 128).sum())   # rows the weight gradients run over
         self.x_rc, self.x_rs, self.x_cc, self.x_cs = u8(M, D), u8(M * D // 32), u8(D, M), u8(M * D // 32)
         self.qw = self.mxk.make_qweights(E, D, F, dev)
         self.h13 = bf(M, 2 * F)
@@ -214,15 +218,15 @@ class Step:
              lambda: L.mxfp8_grouped_gemm_dswiglu_quant(p(self.dy_rc), p(self.dy_rs), M, D, q["w2t_codes"], q["w2t_scales"],
                                                         E, F, off, pad, p(self.h13), p(self.g_rc), p(self.g_rs),
                                                         p(self.g_cc), p(self.g_cs), st)),
-            ("wgrad_dw2", "tensor", 2.0 * M * D * F,
-             lambda: L.mxfp8_grouped_gemm_wgrad(p(self.dy_cc), p(self.dy_cs), D, p(self.h_cc), p(self.h_cs), F, M, off, E, pad,
-                                                p(self.dw2), st)),
+            ("wgrad_dw2", "tensor", 2.0 * self.Mw * D * F,
+             lambda: L.mxfp8_grouped_gemm_wgrad(p(self.dy_cc), p(self.dy_cs), D, p(self.h_cc), p(self.h_cs), F, M, off,
+                                                p(self.rows), E, pad, p(self.dw2), st)),
             ("dgrad_dx", "tensor", 2.0 * M * 2 * F * D,
              lambda: L.mxfp8_grouped_gemm(p(self.g_rc), p(self.g_rs), M, 2 * F, q["w13t_codes"], q["w13t_scales"], E, D, off,
                                           pad, p(self.dx), st)),
-            ("wgrad_dw13", "tensor", 2.0 * M * 2 * F * D,
-             lambda: L.mxfp8_grouped_gemm_wgrad(p(self.g_cc), p(self.g_cs), 2 * F, p(self.x_cc), p(self.x_cs), D, M, off, E,
-                                                pad, p(self.dw13), st)),
+            ("wgrad_dw13", "tensor", 2.0 * self.Mw * 2 * F * D,
+             lambda: L.mxfp8_grouped_gemm_wgrad(p(self.g_cc), p(self.g_cs), 2 * F, p(self.x_cc), p(self.x_cs), D, M, off,
+                                                p(self.rows), E, pad, p(self.dw13), st)),
             ("swiglu_quant_16384x4096", "hbm", 6.0625 * SWIGLU_ROWS * SWIGLU_F,
              lambda: L.mxfp8_swiglu_quant(p(self.sw_in), SWIGLU_ROWS, SWIGLU_F, 3, 1, p(self.sw_rc), p(self.sw_rs),
                                           p(self.sw_cc), p(self.sw_cs), st)),
@@ -477,7 +481,9 @@ def main():
     mlp_ms = float(mean_ms[: step.mlp_ops].sum())
     cast_w_ms = float(sum(mean_ms[i] for i, (n, *_r) in enumerate(step.ops) if n.startswith("cast_w")))
     useful = step.flops(step.R)
-    executed = step.flops(step.M)
+    # executed: the forward and the dgrad GEMMs over the padded rows, the weight
+    # gradients over each expert's rows rounded up to 128 (12 + 6 of the 18 M.D.F)
+    executed = step.flops(step.M) * 12.0 / 18.0 + step.flops(step.Mw) * 6.0 / 18.0
     value = whole_job_tflops(useful, world, ms_step)
     fwd_ms = float(mean_ms[[0, 3, 4]].sum())   # x cast, FC1, FC2 (weights already quantized)
 

@@ -190,12 +190,19 @@ int mxfp8_grouped_gemm(const uint8_t* a, const uint8_t* a_scales, int64_t M, int
  *  gt, gt_scales : COL codes of G, [N, M], MMA scales of [N, M]
  *  xt, xt_scales : COL codes of X, [Kx, M], MMA scales of [Kx, M]
  *  dw            : bf16 [E, N, Kx]; an expert with no rows gets exact zeros.
+ *  expert_rows   : DEVICE int32 [E] or NULL.  The number of token rows at the
+ *                  head of each expert's segment, the rest being padding
+ *                  (0 <= expert_rows[e] <= offsets[e+1] - offsets[e], else
+ *                  nothing is written and MXMOE_ERR_OFFSETS is raised on the
+ *                  device).  The padding's 128-row K blocks are then skipped:
+ *                  the sum runs over the token rows only (with zero pad rows,
+ *                  as the route and gather produce, the result is the same).
  *  Needs N, Kx, M multiples of 128.
  * ------------------------------------------------------------------------- */
 int mxfp8_grouped_gemm_wgrad(const uint8_t* gt, const uint8_t* gt_scales, int64_t N,
                              const uint8_t* xt, const uint8_t* xt_scales, int64_t Kx,
-                             int64_t M, const int32_t* expert_offsets, int E, int pad_multiple,
-                             void* dw, cudaStream_t stream);
+                             int64_t M, const int32_t* expert_offsets, const int32_t* expert_rows,
+                             int E, int pad_multiple, void* dw, cudaStream_t stream);
 
 /* -------------------------------------------------------------------------
  * mxfp8_grouped_gemm_swiglu_quant -- FC1 grouped GEMM with the SwiGLU + dual
@@ -447,6 +454,8 @@ int mxmoe_combine_weight_grad(const void* dout, const void* y, int64_t m_rows, i
  * Backward: gather dout_tokens scaled by the router weights fused with the
  *           dY cast; FC2 dgrad + dSwiGLU + dual quant; dW2; dx rows; dW13;
  *           dx_tokens = sum of a token's dx rows; dweights = <dout, y rows>.
+ *           The weight gradients take each expert's token-row count from the
+ *           saved route tables and skip the all-padding K blocks.
  *
  * The layout capacity is m_cap = mxmoe_route_capacity(T, top_k, E,
  * pad_multiple); every row buffer below has m_cap rows and only the rows

@@ -65,7 +65,7 @@ _SIGS = {
     "mxfp8_swiglu_quant": ([_P, _L, _L, _I, _I, _P, _P, _P, _P, _P], _I),
     "mxfp8_dequantize": ([_P, _P, _L, _L, _P, _P], _I),
     "mxfp8_grouped_gemm": ([_P, _P, _L, _L, _P, _P, _I, _L, _P, _I, _P, _P], _I),
-    "mxfp8_grouped_gemm_wgrad": ([_P, _P, _L, _P, _P, _L, _L, _P, _I, _I, _P, _P], _I),
+    "mxfp8_grouped_gemm_wgrad": ([_P, _P, _L, _P, _P, _L, _L, _P, _P, _I, _I, _P, _P], _I),
     "mxfp8_grouped_gemm_swiglu_quant": ([_P, _P, _L, _L, _P, _P, _I, _L, _P, _I, _P, _P, _P, _P, _P, _P], _I),
     "mxfp8_grouped_gemm_dswiglu_quant": ([_P, _P, _L, _L, _P, _P, _I, _L, _P, _I, _P, _P, _P, _P, _P, _P], _I),
     "mxmoe_workspace_size": ([_L, _L, _I, _L, _I], _S),
@@ -256,8 +256,11 @@ def mxfp8_grouped_gemm(a, a_scales, w, w_scales, offsets, pad_multiple=128, out=
     return out
 
 
-def mxfp8_grouped_gemm_wgrad(gt, gt_scales, xt, xt_scales, offsets, pad_multiple=128, out=None):
-    """Ragged-K grouped GEMM: gt [N, M], xt [Kx, M] COL codes -> dw bf16 [E, N, Kx]."""
+def mxfp8_grouped_gemm_wgrad(gt, gt_scales, xt, xt_scales, offsets, pad_multiple=128, out=None, expert_rows=None):
+    """Ragged-K grouped GEMM: gt [N, M], xt [Kx, M] COL codes -> dw bf16 [E, N, Kx].
+
+    expert_rows (optional, int32 [E] on the device): token rows at the head of
+    each expert's padded segment; the all-padding K blocks are skipped."""
     E = _offs(offsets)
     _need(gt, torch.uint8, "gt")
     _need(xt, torch.uint8, "xt")
@@ -271,8 +274,12 @@ def mxfp8_grouped_gemm_wgrad(gt, gt_scales, xt, xt_scales, offsets, pad_multiple
         out = torch.empty(E, N, Kx, dtype=torch.bfloat16, device=gt.device)
     _need(out, torch.bfloat16, "out")
     _shape(out, (E, N, Kx), "out")
+    if expert_rows is not None:
+        _need(expert_rows, torch.int32, "expert_rows")
+        if expert_rows.numel() != E:
+            raise ValueError(f"expert_rows must hold E={E} counts, got {expert_rows.numel()}")
     _check(lib().mxfp8_grouped_gemm_wgrad(_ptr(gt), _ptr(gt_scales), N, _ptr(xt), _ptr(xt_scales), Kx, M,
-                                          _ptr(offsets), E, pad_multiple, _ptr(out), _stream(gt)))
+                                          _ptr(offsets), _ptr(expert_rows), E, pad_multiple, _ptr(out), _stream(gt)))
     return out
 
 

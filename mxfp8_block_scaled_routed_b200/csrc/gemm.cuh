@@ -48,6 +48,7 @@ struct Params {
   int64_t n_out;      // ragged M: N (B rows per expert; 2F for SwiGLU); ragged K: Kx
   int64_t M;          // token rows of the buffer (bounds the offsets)
   const int32_t* offsets;
+  const int32_t* rows;    // ragged K, optional: real (token) rows at the head of each expert's segment
   int pad;
   const uint8_t* a_scales;
   const uint8_t* b_scales;
@@ -158,8 +159,10 @@ __device__ __forceinline__ Tile get_tile(const Params& p, const int32_t* offs, i
     const int64_t e = t / (nn * nj), rem = t % (nn * nj);
     const int64_t nt = rem / nj, jt = rem % nj;
     T.e = int(e);
-    T.k0 = offs[e];
-    T.nk = int((offs[e + 1] - offs[e]) / 128);
+    // low 7 bits of offs[e]: trailing 128-row K blocks of the segment that
+    // hold only padding (set when the real row counts are given)
+    T.k0 = offs[e] & ~127;
+    T.nk = int(((offs[e + 1] & ~127) - T.k0) / 128) - (offs[e] & 127);
     T.a_row = nt * PM + rank * 128;
     T.b_row0 = jt * BN;
     T.b_row1 = jt * BN + 128;
@@ -402,6 +405,37 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
       if (o < 0 || (o % p.pad) != 0 || int64_t(o) > p.M) bad = true;
       if (i == 0 && o != 0) bad = true;
       if (i < p.E && offs[i + 1] < o) bad = true;
+    }
+  }
+  if constexpr (kMode == kRaggedK) {
+    // real row counts: 0 <= rows[e] <= segment; the padded K blocks past the
+    // last real row are skipped (their codes are zero, they add nothing).
+    // Every thread reads the segments it owns first and tags them after a
+    // barrier, so no read sees a tagged offset.
+    constexpr int kPer = (C::MAX_E + 383) / 384;   // experts per thread (384 threads)
+    int32_t skip[kPer];
+    if (p.rows != nullptr) {
+#pragma unroll
+      for (int j = 0; j < kPer; ++j) {
+        const int i = threadIdx.x + 384 * j;
+        skip[j] = 0;
+        if (!bad && i < p.E) {
+          const int32_t seg = offs[i + 1] - offs[i], r = p.rows[i];
+          if (r < 0 || r > seg) bad = true;
+          else skip[j] = min((seg - ((r + 127) & ~127)) >> 7, 127);
+        }
+      }
+    }
+    if (__syncthreads_or(bad)) {
+      if (threadIdx.x == 0 && blockIdx.x == 0) raise_device_error(kErrOffsets);
+      return;
+    }
+    if (p.rows != nullptr) {
+#pragma unroll
+      for (int j = 0; j < kPer; ++j) {
+        const int i = threadIdx.x + 384 * j;
+        if (i < p.E) offs[i] |= skip[j];
+      }
     }
   }
   if (__syncthreads_or(bad)) {

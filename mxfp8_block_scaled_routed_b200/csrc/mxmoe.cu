@@ -419,8 +419,10 @@ int gemm_ragged_m(const uint8_t* a, const uint8_t* as, int64_t M, int64_t K, con
 }
 
 int gemm_ragged_k(const uint8_t* gt, const uint8_t* gs, int64_t N, const uint8_t* xt, const uint8_t* xs,
-                  int64_t Kx, int64_t M, const int32_t* offsets, int E, int pad, void* dw, cudaStream_t stream) {
+                  int64_t Kx, int64_t M, const int32_t* offsets, const int32_t* rows, int E, int pad, void* dw,
+                  cudaStream_t stream) {
   gemm::Params p{};
+  p.rows = rows;
   p.E = E;
   p.rows_a = N;
   p.kext = M;
@@ -584,12 +586,12 @@ int bwd_core(const void* dy, int64_t M, int64_t D, const mxmoe_qweights& qw, int
   MX_TRY(gemm_dswiglu(w.dy_rc, w.dy_rs, M, D, qw.w2t_codes, qw.w2t_scales, E, F, offsets, pad, saved->h13, w.g_rc,
                       w.g_rs, w.g_cc, w.g_cs, stream));
   // a7: dW2[e] = dY_e^T . h_e
-  MX_TRY(gemm_ragged_k(w.dy_cc, w.dy_cs, D, saved->h_col_codes, saved->h_col_scales, F, M, offsets, E, pad, dw2,
+  MX_TRY(gemm_ragged_k(w.dy_cc, w.dy_cs, D, saved->h_col_codes, saved->h_col_scales, F, M, offsets, nullptr, E, pad, dw2,
                        stream));
   // a8: dx = dh13 . W13[e]
   MX_TRY(gemm_ragged_m(w.g_rc, w.g_rs, M, 2 * F, qw.w13t_codes, qw.w13t_scales, E, D, offsets, pad, dx, stream));
   // a9: dW13[e] = dh13_e^T . x_e
-  return gemm_ragged_k(w.g_cc, w.g_cs, 2 * F, saved->x_col_codes, saved->x_col_scales, D, M, offsets, E, pad, dw13,
+  return gemm_ragged_k(w.g_cc, w.g_cs, 2 * F, saved->x_col_codes, saved->x_col_scales, D, M, offsets, nullptr, E, pad, dw13,
                        stream);
 }
 
@@ -630,6 +632,7 @@ struct LayerFwdWs {
 struct LayerBwdWs {
   BwdWs mlp;
   uint16_t* dx_rows;   // dx of the padded rows, before the unpermute
+  int32_t* rows;       // real rows of each expert (the weight gradients skip the all-pad K blocks)
 };
 
 int64_t route_chunks(int64_t T, int k) { return (T * k + kRouteChunk - 1) / kRouteChunk; }
@@ -658,6 +661,7 @@ size_t carve_layer_bwd(uint8_t* base, int64_t m_cap, int64_t D, int E, int64_t F
   b.g_cs = c.take<uint8_t>(m_cap * 2 * F / 32);
   b.qw = mxmoe_qweights{};
   w->dx_rows = c.take<uint16_t>(m_cap * D * 2);
+  w->rows = c.take<int32_t>(size_t(E) * 4);
   return c.off + 256;
 }
 
@@ -797,14 +801,15 @@ int mxfp8_grouped_gemm(const uint8_t* a, const uint8_t* a_scales, int64_t M, int
 }
 
 int mxfp8_grouped_gemm_wgrad(const uint8_t* gt, const uint8_t* gt_scales, int64_t N, const uint8_t* xt,
-                             const uint8_t* xt_scales, int64_t Kx, int64_t M, const int32_t* expert_offsets, int E,
-                             int pad_multiple, void* dw, cudaStream_t stream) {
+                             const uint8_t* xt_scales, int64_t Kx, int64_t M, const int32_t* expert_offsets,
+                             const int32_t* expert_rows, int E, int pad_multiple, void* dw, cudaStream_t stream) {
   MX_TRY(check_offsets_args(expert_offsets, E, pad_multiple));
   MX_TRY(check_mult("M", M, 128));
   MX_TRY(check_mult("N", N, 128));
   MX_TRY(check_mult("Kx", Kx, 128));
   MX_TRY(check_ptrs({{"gt", gt}, {"gt_scales", gt_scales}, {"xt", xt}, {"xt_scales", xt_scales}, {"dw", dw}}));
-  return gemm_ragged_k(gt, gt_scales, N, xt, xt_scales, Kx, M, expert_offsets, E, pad_multiple, dw, stream);
+  return gemm_ragged_k(gt, gt_scales, N, xt, xt_scales, Kx, M, expert_offsets, expert_rows, E, pad_multiple, dw,
+                       stream);
 }
 
 int mxfp8_grouped_gemm_swiglu_quant(const uint8_t* a, const uint8_t* a_scales, int64_t M, int64_t K,
@@ -1221,14 +1226,17 @@ int moe_layer_bwd_q(const void* dout_tokens, int64_t T, int64_t D, const float* 
                                   w.mlp.dy_rs, w.mlp.dy_cc, w.mlp.dy_cs, rows_dev, stream, &g));
   const BwdWs& b = w.mlp;
   const mxmoe_saved* ms = &saved->mlp;
+  // real rows per expert, from the route tables, for the weight gradients
+  expert_rows_kernel<<<(E + 255) / 256, 256, 0, stream>>>(saved->offsets, saved->row_slot, E, m_cap, w.rows);
+  MX_CHECK_CUDA(cudaGetLastError(), "expert rows launch");
   // a6 - a9
   MX_TRY(gemm_dswiglu(b.dy_rc, b.dy_rs, m_cap, D, qw->w2t_codes, qw->w2t_scales, E, F, saved->offsets, pad_multiple,
                       ms->h13, b.g_rc, b.g_rs, b.g_cc, b.g_cs, stream));
-  MX_TRY(gemm_ragged_k(b.dy_cc, b.dy_cs, D, ms->h_col_codes, ms->h_col_scales, F, m_cap, saved->offsets, E,
+  MX_TRY(gemm_ragged_k(b.dy_cc, b.dy_cs, D, ms->h_col_codes, ms->h_col_scales, F, m_cap, saved->offsets, w.rows, E,
                        pad_multiple, dw2, stream));
   MX_TRY(gemm_ragged_m(b.g_rc, b.g_rs, m_cap, 2 * F, qw->w13t_codes, qw->w13t_scales, E, D, saved->offsets,
                        pad_multiple, w.dx_rows, stream));
-  MX_TRY(gemm_ragged_k(b.g_cc, b.g_cs, 2 * F, ms->x_col_codes, ms->x_col_scales, D, m_cap, saved->offsets, E,
+  MX_TRY(gemm_ragged_k(b.g_cc, b.g_cs, 2 * F, ms->x_col_codes, ms->x_col_scales, D, m_cap, saved->offsets, w.rows, E,
                        pad_multiple, dw13, stream));
   // unpermute dx (sum over a token's copies) and the router-weight gradient
   MX_TRY(mxmoe_unpermute_combine(w.dx_rows, m_cap, D, saved->slot_row, nullptr, T, top_k, dx_tokens, stream));

@@ -198,6 +198,28 @@ combine_kernel(const uint16_t* __restrict__ y, int64_t m_rows, const int32_t* __
   }
 }
 
+// Real (token) rows of each expert's padded segment.  The route lays out a
+// segment's token rows first and its pad rows (row_slot < 0) after them, so
+// the count is the position of the first pad row: a binary search per expert.
+// A segment outside [0, m_rows] counts 0 rows (the GEMMs reject its offsets).
+__global__ void __launch_bounds__(256)
+expert_rows_kernel(const int32_t* __restrict__ offsets, const int32_t* __restrict__ row_slot, int E, int64_t m_rows,
+                   int32_t* __restrict__ rows) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= E) return;
+  const int64_t base = offsets[e], end = offsets[e + 1];
+  if (base < 0 || end > m_rows || end < base) {
+    rows[e] = 0;
+    return;
+  }
+  int64_t lo = base, hi = end;     // first pad row in [base, end]
+  while (lo < hi) {
+    const int64_t mid = (lo + hi) >> 1;
+    if (row_slot[mid] >= 0) lo = mid + 1; else hi = mid;
+  }
+  rows[e] = int32_t(lo - base);
+}
+
 // dw[t*k+j] = <dout[t], y[slot_row[t*k+j]]> in fp32 (0 for an invalid slot).
 __global__ void __launch_bounds__(256)
 combine_weight_grad_kernel(const uint16_t* __restrict__ dout, const uint16_t* __restrict__ y, int64_t m_rows,

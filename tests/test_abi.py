@@ -47,7 +47,8 @@ def test_gemm_rejects_bad_pad_and_shapes(L):
 
 
 def test_wgrad_and_fused_reject(L):
-    s = L.mxfp8_grouped_gemm_wgrad(P(FAKE), P(FAKE), 256, P(FAKE), P(FAKE), 100, 256, P(FAKE), 4, 128, P(FAKE), None)
+    s = L.mxfp8_grouped_gemm_wgrad(P(FAKE), P(FAKE), 256, P(FAKE), P(FAKE), 100, 256, P(FAKE), None, 4, 128, P(FAKE),
+                                   None)
     assert s == 2 and "Kx=100" in _err(L)
     s = L.mxfp8_grouped_gemm_swiglu_quant(P(FAKE), P(FAKE), 256, 256, P(FAKE), P(FAKE), 4, 96, P(FAKE), 128,
                                           None, P(FAKE), P(FAKE), P(FAKE), P(FAKE), None)

@@ -179,6 +179,54 @@ def test_wgrad_exact_closed_form_and_empty_expert(N, Kx):
     assert (got[1] == 0).all() and not np.signbit(got[1]).any()
 
 
+@pytest.mark.parametrize("N,Kx", [(256, 384), (256, 512)])
+def test_wgrad_expert_rows_skip_only_padding(N, Kx):
+    """With each expert's token-row count given, the weight gradient stops at
+    the last 128-row K block holding a token row.  Kx = 384 runs the single-CTA
+    kernel, 512 the CTA pairs.  With zero pad rows the result equals the full
+    sum; codes planted in the all-padding K blocks are ignored with the counts
+    (and seen without them); a count beyond its segment writes nothing and
+    raises the offsets error."""
+    g = synth.rng(9)
+    counts = [300, 0, 129, 256]
+    E, pad = len(counts), 256
+    off = _offsets(counts, pad)
+    M = int(off[-1])
+    G = np.zeros((M, N), np.float32)
+    X = np.zeros((M, Kx), np.float32)
+    for e, c in enumerate(counts):
+        G[off[e]:off[e] + c] = synth.normal(g, (c, N), 1e-2)
+        X[off[e]:off[e] + c] = synth.normal(g, (c, Kx))
+    gc, gs = _mx_cols_dev(_bf16(G))
+    xc, xs = _mx_cols_dev(_bf16(X))
+    rows = _dev(np.array(counts, np.int32))
+    full = mxk.mxfp8_grouped_gemm_wgrad(gc, gs, xc, xs, _dev(off), pad)
+    skip = mxk.mxfp8_grouped_gemm_wgrad(gc, gs, xc, xs, _dev(off), pad, expert_rows=rows)
+    assert torch.equal(full, skip)
+    # plant codes (and unit scales) in the K blocks that hold only padding
+    gc2, xc2, gs2, xs2 = gc.clone(), xc.clone(), gs.clone(), xs.clone()
+    for e, c in enumerate(counts):
+        lo, hi = int(off[e]) + (c + 127) // 128 * 128, int(off[e + 1])
+        if hi > lo:
+            gc2[:, lo:hi] = 0x38      # E4M3 1.0
+            xc2[:, lo:hi] = 0x38
+    gs2.fill_(127)
+    xs2.fill_(127)
+    gs2.copy_(torch.where(gs == 0, gs2, gs))   # real blocks keep their scales
+    xs2.copy_(torch.where(xs == 0, xs2, xs))
+    planted = mxk.mxfp8_grouped_gemm_wgrad(gc2, gs2, xc2, xs2, _dev(off), pad, expert_rows=rows)
+    assert torch.equal(planted, full)
+    unskipped = mxk.mxfp8_grouped_gemm_wgrad(gc2, gs2, xc2, xs2, _dev(off), pad)
+    assert not torch.equal(unskipped, full)
+    # a count larger than its segment
+    out = torch.full((E, N, Kx), 3.0, dtype=torch.bfloat16, device=DEV)
+    bad = _dev(np.array([300, 1, 129, 256], np.int32))
+    assert mxk.device_error() == 0
+    mxk.mxfp8_grouped_gemm_wgrad(gc, gs, xc, xs, _dev(off), pad, out=out, expert_rows=bad)
+    assert mxk.device_error(reset=True) == 4
+    assert (bf16_np(out) == 3.0).all()
+
+
 @pytest.mark.parametrize("pad,N,Kx", [(128, 256, 256), (256, 384, 512), (256, 512, 768)])
 def test_wgrad_random_vs_oracle(pad, N, Kx):
     g = synth.rng(5)
