@@ -20,12 +20,15 @@
 
 using namespace mxmoe;
 
-// Tile width of the wgrad (ragged-K) GEMM when Kx allows both: 256 (one TMEM
-// accumulator) or 128 (two, epilogue overlapped with the next tile's MMAs).
+// Build-time choices, for measuring one tiling against another:
+// tile width of the single-CTA weight-gradient (ragged-K) GEMM when Kx allows
+// both, 256 (one TMEM accumulator) or 128 (two, the epilogue overlapped with
+// the next tile's MMAs) ...
 #ifndef MXMOE_WGRAD_BN
 #define MXMOE_WGRAD_BN 256
 #endif
-// 256 x 256 tiles on CTA pairs (cta_group::2) wherever the shapes allow.
+// ... and 256 x 256 tiles on CTA pairs (cta_group::2) wherever the shapes
+// allow, for the ragged-M GEMMs and for the weight gradients.
 #ifndef MXMOE_USE_PAIRS
 #define MXMOE_USE_PAIRS 1
 #endif
@@ -436,12 +439,9 @@ int gemm_ragged_k(const uint8_t* gt, const uint8_t* gs, int64_t N, const uint8_t
   // CTA pairs (256 x 256 tiles, 128 x 256 per CTA) when N and Kx allow: they
   // halve each SM's B-operand loads; the accumulator hand-off, paid once
   // per tile over each expert's short K, uses a CTA-scope arrive
-  if (MXMOE_WGRAD_PAIRS == 1 && Kx % 256 == 0 && N % 256 == 0)
+  if (MXMOE_WGRAD_PAIRS && Kx % 256 == 0 && N % 256 == 0)
     return launch_gemm<gemm::kRaggedK, gemm::kEpiBF16, 256, true>(gt, N, xt, Kx, p,
                                                                   int64_t(E) * (N / 256) * (Kx / 256), stream, 10);
-  if (MXMOE_WGRAD_PAIRS == 2 && N % 256 == 0)
-    return launch_gemm<gemm::kRaggedK, gemm::kEpiBF16, 128, true>(gt, N, xt, Kx, p,
-                                                                  int64_t(E) * (N / 256) * (Kx / 128), stream, 16);
   if (Kx % 256 == 0 && MXMOE_WGRAD_BN == 256)
     return launch_gemm<gemm::kRaggedK, gemm::kEpiBF16, 256, false>(gt, N, xt, Kx, p,
                                                                    int64_t(E) * (N / 128) * (Kx / 256), stream, 2);
