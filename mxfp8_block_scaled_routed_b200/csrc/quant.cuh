@@ -716,26 +716,29 @@ mx_dequant_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__
 }
 
 // Vector path (cols % 16 == 0, 16-B aligned codes and output): one thread
-// per 16 codes, which share one scale.  The code's exponent and mantissa
-// bits are placed in an fp32 word at the fp32 mantissa's top, so that the
-// word reads as the code's value times 2^-120 (E4M3, exponent bias 7) or
-// 2^-112 (E5M2, bias 15), normals and subnormals alike; multiplying by
-// 2^(byte - bias) -- split in two factors when that power is not an fp32
-// normal -- then rounds the exact product code * 2^(byte-127) once, exactly
-// as the scalar path does.
+// per 16 codes, which share one scale.  Two codes at a time become f16 by
+// cvt.rn.f16x2.{e4m3x2,e5m2x2} (exact: both formats fit in f16), then fp32,
+// and one product with 2^(byte - 127) (exact, the subnormal 2^-127 included:
+// the product of a code of at most 4 significant bits and a power of two is
+// at least 2^-136) is rounded once to bf16 -- the correctly rounded value, as
+// the scalar path gives.
 template <int kElem>
-struct Fp8Bits {
-  static constexpr int kShift = kElem == 0 ? 20 : 21;     // code bit 0 -> fp32 bit
-  static constexpr uint32_t kOff = kElem == 0 ? 120u : 112u;   // 127 - exponent bias
-};
+__device__ __forceinline__ uint32_t fp8x2_to_f16x2(uint32_t pair) {
+  uint32_t h;
+  if constexpr (kElem == 0)
+    asm("{ .reg .b16 c; cvt.u16.u32 c, %1; cvt.rn.f16x2.e4m3x2 %0, c; }" : "=r"(h) : "r"(pair));
+  else
+    asm("{ .reg .b16 c; cvt.u16.u32 c, %1; cvt.rn.f16x2.e5m2x2 %0, c; }" : "=r"(h) : "r"(pair));
+  return h;
+}
 
 template <int kElem>
-__device__ __forceinline__ uint32_t dequant_pair(uint32_t b0, uint32_t b1, float m1, float m2) {
-  constexpr int sh = Fp8Bits<kElem>::kShift;
-  const float y0 = __uint_as_float(((b0 & 0x80u) << 24) | ((b0 & 0x7Fu) << sh)) * m1 * m2;
-  const float y1 = __uint_as_float(((b1 & 0x80u) << 24) | ((b1 & 0x7Fu) << sh)) * m1 * m2;
-  const __nv_bfloat162 h = __floats2bfloat162_rn(y0, y1);
-  return *reinterpret_cast<const uint32_t*>(&h);
+__device__ __forceinline__ uint32_t dequant_pair(uint32_t pair, float s) {
+  const uint32_t h = fp8x2_to_f16x2<kElem>(pair);
+  const float y0 = __half2float(__ushort_as_half(uint16_t(h & 0xFFFFu))) * s;
+  const float y1 = __half2float(__ushort_as_half(uint16_t(h >> 16))) * s;
+  const __nv_bfloat162 b = __floats2bfloat162_rn(y0, y1);
+  return *reinterpret_cast<const uint32_t*>(&b);
 }
 
 // bf16 of a code whose exponent field is all ones: E4M3 S.1111.111 is NaN;
@@ -747,9 +750,9 @@ __device__ __forceinline__ uint32_t special_bf16(uint32_t c) {
 }
 
 template <int kElem>
-__device__ __forceinline__ void dequant_word(uint32_t w, float m1, float m2, uint32_t& lo, uint32_t& hi) {
-  lo = dequant_pair<kElem>(w & 0xFFu, (w >> 8) & 0xFFu, m1, m2);
-  hi = dequant_pair<kElem>((w >> 16) & 0xFFu, w >> 24, m1, m2);
+__device__ __forceinline__ void dequant_word(uint32_t w, float s, uint32_t& lo, uint32_t& hi) {
+  lo = dequant_pair<kElem>(w & 0xFFFFu, s);
+  hi = dequant_pair<kElem>(w >> 16, s);
   // bytes whose special-value field is all ones (E4M3: the low 7 bits; E5M2:
   // the 5 exponent bits) take their value from special_bf16
   constexpr uint32_t f = kElem == 0 ? 0x7Fu : 0x7Cu;
@@ -771,14 +774,11 @@ __device__ __forceinline__ void dequant16(const uint4 q, uint32_t byte, uint4& o
   if (byte == 0xFFu) {
     o0 = o1 = make_uint4(0x7FFF7FFFu, 0x7FFF7FFFu, 0x7FFF7FFFu, 0x7FFF7FFFu);
   } else {
-    constexpr uint32_t off = Fp8Bits<kElem>::kOff;
-    const bool one = byte <= 254u - off;            // 2^(byte - bias) is an fp32 normal
-    const float m1 = __uint_as_float(one ? (byte + off) << 23 : (byte + off - 127u) << 23);
-    const float m2 = one ? 1.0f : __uint_as_float(254u << 23);
-    dequant_word<kElem>(q.x, m1, m2, o0.x, o0.y);
-    dequant_word<kElem>(q.y, m1, m2, o0.z, o0.w);
-    dequant_word<kElem>(q.z, m1, m2, o1.x, o1.y);
-    dequant_word<kElem>(q.w, m1, m2, o1.z, o1.w);
+    const float s = e8m0_to_f32(byte);
+    dequant_word<kElem>(q.x, s, o0.x, o0.y);
+    dequant_word<kElem>(q.y, s, o0.z, o0.w);
+    dequant_word<kElem>(q.z, s, o1.x, o1.y);
+    dequant_word<kElem>(q.w, s, o1.z, o1.w);
   }
 }
 
