@@ -126,13 +126,59 @@ __device__ __forceinline__ int64_t num_tiles(const Params& p, const int32_t* off
   }
 }
 
+// The tiles t0, t0 + step, ... of one CTA (or CTA pair), in order.
+//   ragged M: t = mt * nt + j (m tile, n tile), decoded per tile; e is the
+//             last expert with offs[e] <= the tile's first row.  Its tiles
+//             run the whole K extent, so the decode is a small part of one.
+//   ragged K: t = (e * n1 + nt) * n2 + jt (expert, output row tile, column
+//             tile); the coordinates advance by additions.  Decoding them
+//             with 64-bit divisions took several hundred cycles per tile on
+//             every role's thread, and the weight gradients run tiles of one
+//             or two K blocks (~700 cycles each).
 template <int kMode, int kEpi, int BN, bool kPair>
-__device__ __forceinline__ Tile get_tile(const Params& p, const int32_t* offs, int64_t t, int rank) {
+struct TileIter {
+  static constexpr int PM = kPair ? 256 : 128;
+  int64_t t, step;
+  int64_t n1, n2;      // ragged K: output row tiles per expert, column tiles
+  int64_t c1, c2;      // ragged K: (nt, jt)
+  int64_t d1, d2, d0;  // per-step increments of c1, c2 and e
+  int e;
+
+  __device__ __forceinline__ TileIter(const Params& p, const int32_t* offs, int64_t t0, int64_t step_)
+      : t(t0), step(step_) {
+    if constexpr (kMode == kRaggedK) {
+      // (extents clamped to 1 for the divisions: a zero extent means no tiles)
+      n1 = max(int64_t(1), p.rows_a / PM);
+      n2 = max(int64_t(1), p.n_out / BN);
+      const int64_t q = t0 / n2, qs = step / n2;
+      c2 = t0 % n2;
+      c1 = q % n1;
+      e = int(q / n1);
+      d2 = step % n2;
+      d1 = qs % n1;
+      d0 = qs / n1;
+    }
+  }
+  __device__ __forceinline__ void next(const Params&, const int32_t*) {
+    t += step;
+    if constexpr (kMode == kRaggedK) {
+      c2 += d2;
+      c1 += d1;
+      if (c2 >= n2) { c2 -= n2; ++c1; }
+      e += int(d0);
+      if (c1 >= n1) { c1 -= n1; ++e; }
+    }
+  }
+};
+
+template <int kMode, int kEpi, int BN, bool kPair>
+__device__ __forceinline__ Tile get_tile(const Params& p, const int32_t* offs, const TileIter<kMode, kEpi, BN, kPair>& it,
+                                         int rank) {
   constexpr int PM = kPair ? 256 : 128;
   Tile T;
   if constexpr (kMode == kRaggedM) {
     const int64_t nt = (kEpi == kEpiSwiGLU) ? p.F / 128 : p.n_out / BN;
-    const int64_t mt = t / nt, ntile = t % nt;
+    const int64_t mt = it.t / nt, ntile = it.t % nt;
     const int64_t m0 = mt * PM;
     int lo = 0, hi = p.E;  // last e with offs[e] <= m0
     while (hi - lo > 1) {
@@ -155,19 +201,17 @@ __device__ __forceinline__ Tile get_tile(const Params& p, const int32_t* offs, i
       T.out_c0 = ntile * BN;
     }
   } else {
-    const int64_t nn = p.rows_a / PM, nj = p.n_out / BN;
-    const int64_t e = t / (nn * nj), rem = t % (nn * nj);
-    const int64_t nt = rem / nj, jt = rem % nj;
-    T.e = int(e);
+    const int e = it.e;
+    T.e = e;
     // low 7 bits of offs[e]: trailing 128-row K blocks of the segment that
     // hold only padding (set when the real row counts are given)
     T.k0 = offs[e] & ~127;
     T.nk = int(((offs[e + 1] & ~127) - T.k0) / 128) - (offs[e] & 127);
-    T.a_row = nt * PM + rank * 128;
-    T.b_row0 = jt * BN;
-    T.b_row1 = jt * BN + 128;
+    T.a_row = it.c1 * PM + rank * 128;
+    T.b_row0 = it.c2 * BN;
+    T.b_row1 = it.c2 * BN + 128;
     T.out_r0 = T.a_row;
-    T.out_c0 = jt * BN;
+    T.out_c0 = it.c2 * BN;
   }
   if constexpr (kEpi == kEpiSwiGLU)
     T.b_mine = rank ? T.b_row1 : T.b_row0;          // gate rows on the even CTA, up rows on the odd one
@@ -482,8 +526,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int64_t t = unit; t < ntiles && ok; t += nunits) {
-        const Tile T = get_tile<kMode, kEpi, BN, kPair>(p, offs, t, rank);
+      for (TileIter<kMode, kEpi, BN, kPair> it(p, offs, unit, nunits); it.t < ntiles && ok; it.next(p, offs)) {
+        const Tile T = get_tile(p, offs, it, rank);
         for (int kb = 0; kb < T.nk; ++kb) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1)) { ok = false; break; }
           const int64_t k = T.k0 + int64_t(kb) * 128;
@@ -532,8 +576,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
       bool ok = true;
       const uint32_t sf_col0 = C::ACC_COLS;
       constexpr uint32_t kMmaM = kPair ? 256 : 128;
-      for (int64_t t = unit; t < ntiles && ok; t += nunits) {
-        const Tile T = get_tile<kMode, kEpi, BN, kPair>(p, offs, t, 0);
+      for (TileIter<kMode, kEpi, BN, kPair> it(p, offs, unit, nunits); it.t < ntiles && ok; it.next(p, offs)) {
+        const Tile T = get_tile(p, offs, it, 0);
         if (T.nk == 0) continue;
         if (!(kPair ? mbar_wait_cluster(tempty_bar(acc), acc_phase ^ 1) : mbar_wait(tempty_bar(acc), acc_phase ^ 1))) {
           ok = false;
@@ -596,8 +640,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
     constexpr int kChunks = kHalf / 32;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int64_t t = unit; t < ntiles; t += nunits) {
-      const Tile T = get_tile<kMode, kEpi, BN, kPair>(p, offs, t, rank);
+    for (TileIter<kMode, kEpi, BN, kPair> it(p, offs, unit, nunits); it.t < ntiles; it.next(p, offs)) {
+      const Tile T = get_tile(p, offs, it, rank);
       const int64_t row0 = T.out_r0 + q * 32;              // first row of this warp's 32-row slab
       if constexpr (kMode == kRaggedK) {
         if (T.nk == 0) {
