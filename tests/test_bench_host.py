@@ -75,3 +75,38 @@ def test_reference_arm_under_torchrun_two_ranks():
     assert len(lines) == 1
     line = json.loads(lines[0])
     assert line["impl"] == "reference" and line["n_gpus"] == 2
+
+
+def test_ncu_traffic_only_for_the_sources_it_was_taken_at(tmp_path, monkeypatch):
+    """The roofline's `traffic` comes from a profiles/ summary only while its
+    source stamp matches the kernel sources; otherwise it is reported as null."""
+    sys.path.insert(0, ROOT)
+    import bench
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "profiles" / "cast_w13_dual_dsv3.md").write_text(
+        "# summary\n\ntraffic_bytes_per_launch: 2.964e+10\n\nsource_hash: 0123456789ab\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "src_hash", lambda: "0123456789ab")
+    assert bench.ncu_traffic("cast_w13_dual", "dsv3") == pytest.approx(2.964e10)
+    assert bench.ncu_traffic("wgrad_dw13", "dsv3") is None          # no summary
+    monkeypatch.setattr(bench, "src_hash", lambda: "ba9876543210")
+    assert bench.ncu_traffic("cast_w13_dual", "dsv3") is None       # stale stamp
+
+
+def test_source_hash_changes_with_any_kernel_source(tmp_path, monkeypatch):
+    """Editing any one file of the CUDA sources changes the stamp."""
+    sys.path.insert(0, ROOT)
+    import bench
+    csrc = tmp_path / "mxfp8_block_scaled_routed_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    names = ["gemm.cuh", "mxmoe.cu", "quant.cuh"]
+    for n in names:
+        (csrc / n).write_text(f"// {n}\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    base = bench.src_hash()
+    assert len(base) == 12 and bench.src_hash() == base
+    for n in names:
+        (csrc / n).write_text(f"// {n} edited\n")
+        assert bench.src_hash() != base, n
+        (csrc / n).write_text(f"// {n}\n")
+    assert bench.src_hash() == base
